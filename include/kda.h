@@ -1,0 +1,155 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) library.
+ *
+ * The operation.  KDA is a gated delta-rule recurrence with one forgetting
+ * factor per key channel.  For each (sequence, head), with state S (d_k x d_v):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t          (the query reads the updated state)
+ *
+ * Source: "Kimi K3" open-weights field notes (ailearn.mscapital.top/kimi-k3.html),
+ * panel "KDA 单头递归" (KDA single-head recurrence): alpha_t = exp(g_t) is the
+ * per-channel forgetting, beta_t the per-token write strength, the old state is
+ * decayed per channel first and then corrected and written by the delta rule.
+ * The same page's panel "g ∈ (-5, 0)" bounds the log-decay; the library relies
+ * on g <= 0 (see the preconditions below).  No query scaling or normalisation
+ * happens inside the library: callers pass q and k as they want them used.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *     contiguous, 16-byte aligned (cu_seqlens: 4-byte aligned).  The library never allocates device memory
+ *     and never synchronises the stream in the compute entry points.
+ *   - q, k, g are [.., H, d_k]; v, o are [.., H, d_v]; beta is [.., H];
+ *     states are [N, H, d_k, d_v] fp32 (d_k rows, d_v columns).
+ *   - q, k, v and o share one dtype (kda_dtype); g, beta and states are fp32.
+ *   - Arguments are validated on the host before any launch; a rejected call
+ *     launches nothing and returns a status.  No C++ exception crosses the ABI.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream).  Launch failures are reported as KDA_ERR_CUDA.
+ *   - Supported head sizes: d_k == d_v in {32, 64, 128}.  bf16 with d = 128 runs
+ *     the tensor-core chunkwise path; every other supported combination runs the
+ *     fp32 CUDA-core chunkwise path.
+ */
+#ifndef KDA_B200_H
+#define KDA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,          /* null pointer, negative size, bad dtype     */
+    KDA_ERR_UNSUPPORTED_SHAPE = 2,    /* head size not supported                   */
+    KDA_ERR_MISALIGNED = 3,           /* a pointer is not 16-byte aligned          */
+    KDA_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes < kda_fwd_workspace_size(...)    */
+    KDA_ERR_CUDA = 5,                 /* a CUDA launch or query failed             */
+    KDA_ERR_DEVICE_TIMEOUT = 6,       /* a bounded device-side wait gave up        */
+    KDA_ERR_BAD_SEQLENS = 7           /* cu_seqlens not monotone / out of range    */
+} kda_status;
+
+typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int kda_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *kda_status_string(kda_status s);
+
+/*
+ * Bytes of device workspace that kda_fwd needs for these sizes.  The chunkwise
+ * path stores, per 64-token chunk and head, the intra-chunk transform results
+ * (the delta-rule factors W and U, the decayed keys and queries, the masked
+ * query-key block and the chunk's total decay) that the state pass consumes.
+ * Returns 0 for an invalid or unsupported combination.
+ *   B, T      : fixed-length batch (B sequences of T tokens), or with
+ *               num_seqs > 0 and packed input: B = 1, T = total tokens.
+ *   num_seqs  : 0 for fixed-length input, else the number of packed sequences.
+ */
+size_t kda_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype);
+
+/*
+ * Chunkwise prefill: runs the recurrence over every (sequence, head) from its
+ * initial state and returns all outputs and the final states.
+ *
+ *   q, k     [B, T, H, d_k]  dtype      keys and queries used as given
+ *   v        [B, T, H, d_v]  dtype
+ *   g        [B, T, H, d_k]  fp32       log-decay; precondition g <= 0
+ *                                       (the pages bound it to (-5, 0))
+ *   beta     [B, T, H]       fp32       write strength
+ *   h0       [N, H, d_k, d_v] fp32      initial states; NULL means zeros
+ *   cu_seqlens [num_seqs + 1] int32     NULL for fixed-length input; otherwise
+ *                                       packed sequence offsets (B must be 1,
+ *                                       cu_seqlens[0] = 0, non-decreasing,
+ *                                       cu_seqlens[num_seqs] = T).  Empty
+ *                                       sequences are allowed (hT = h0).
+ *   o        [B, T, H, d_v]  dtype      outputs; must not alias any input
+ *   hT       [N, H, d_k, d_v] fp32      final states, NULL to skip.  hT == h0 is
+ *                                       allowed (the update is then in place).
+ *   workspace, ws_bytes                 device scratch of at least
+ *                                       kda_fwd_workspace_size(...) bytes; its
+ *                                       contents on entry do not matter.
+ *   N = B for fixed-length input, N = num_seqs for packed input.
+ *
+ * The cu_seqlens preconditions are checked on the device; a violation makes
+ * the call write no outputs and is reported by kda_get_last_device_error.
+ * T = 0 (or B = 0) is a valid empty call that only copies h0 to hT.
+ */
+kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, const float *h0, const int32_t *cu_seqlens,
+                   int num_seqs, int B, int T, int H, int dk, int dv, int dtype, void *o,
+                   float *hT, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * The two phases of kda_fwd on the tensor-core path (bf16, d_k = d_v = 128),
+ * exposed so callers can schedule or time them separately.  Calling
+ * kda_fwd_intra and then kda_fwd_inter on the same stream and workspace is
+ * exactly kda_fwd.  Other dtype / head-size combinations return
+ * KDA_ERR_UNSUPPORTED_SHAPE (kda_fwd handles them in a single kernel).
+ *
+ * kda_fwd_intra: everything inside a chunk, in parallel over (chunk, head):
+ *   validates cu_seqlens and lays out the chunks (packed input), then computes
+ *   the in-chunk cumulative log-decay, the strictly-lower key-key block and its
+ *   unit-triangular inverse, the delta-rule factors W and U, the decayed keys
+ *   and queries, the masked query-key block and the chunk's total decay, and
+ *   stores them in `workspace`.  Arguments as for kda_fwd.
+ * kda_fwd_inter: the sequential pass over the chunks of every (sequence, head)
+ *   with the state on chip: reads the records from `workspace`, writes o and hT.
+ *   The size arguments must match the preceding kda_fwd_intra call.
+ */
+kda_status kda_fwd_intra(const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, const int32_t *cu_seqlens, int num_seqs, int B,
+                         int T, int H, int dk, int dv, int dtype, void *workspace,
+                         size_t ws_bytes, void *stream);
+kda_status kda_fwd_inter(const float *h0, const int32_t *cu_seqlens, int num_seqs, int B, int T,
+                         int H, int dk, int dv, int dtype, void *o, float *hT, void *workspace,
+                         size_t ws_bytes, void *stream);
+
+/*
+ * One decode step: every (sequence, head) consumes one token and updates its
+ * state in place (the recurrence above with T = 1).
+ *
+ *   q, k [N, H, d_k] dtype;  v [N, H, d_v] dtype;  g [N, H, d_k] fp32;
+ *   beta [N, H] fp32;  S [N, H, d_k, d_v] fp32, read and overwritten;
+ *   o [N, H, d_v] dtype, the read of the updated state.
+ * Each state is read from HBM once and written once.  N = 0 is a no-op.
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, float *S, void *o, int N, int H, int dk,
+                           int dv, int dtype, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error word
+ * (cu_seqlens violations, bounded waits that gave up).  Returns KDA_OK,
+ * KDA_ERR_BAD_SEQLENS, KDA_ERR_DEVICE_TIMEOUT or KDA_ERR_CUDA.
+ */
+kda_status kda_get_last_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_H */

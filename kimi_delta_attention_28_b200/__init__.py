@@ -1,0 +1,18 @@
+"""Kimi Delta Attention (KDA) on NVIDIA B200 (sm_100a).
+
+The gated delta-rule recurrence with one forgetting factor per key channel,
+S_t = (I - b_t k_t k_t^T) Diag(exp g_t) S_{t-1} + b_t k_t v_t^T, o_t = S_t^T q_t
+("Kimi K3" open-weights field notes, ailearn.mscapital.top/kimi-k3.html,
+panel "KDA 单头递归"), as a C-ABI CUDA library:
+
+* ``kda_fwd``          chunkwise prefill (fixed-length or packed varlen batches,
+                       initial and final states);
+* ``kda_decode_step``  one token per sequence, state updated in place.
+
+This package is the thin Python binding; ``include/kda.h`` is the interface.
+"""
+from ._lib import (KDAError, device_error, kda_decode_step, kda_fwd,  # noqa: F401
+                   kda_fwd_inter, kda_fwd_intra, load_library, workspace_size)
+
+__all__ = ["kda_fwd", "kda_fwd_intra", "kda_fwd_inter", "kda_decode_step", "workspace_size", "device_error", "load_library",
+           "KDAError"]

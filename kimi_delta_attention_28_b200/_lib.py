@@ -1,0 +1,195 @@
+"""ctypes binding of ``libkda_b200.so`` (the C ABI in ``include/kda.h``).
+
+Argument marshalling only: every step of the recurrence runs in the library's
+CUDA kernels.  torch provides device memory (outputs, workspace) and the
+current CUDA stream.  If the library is missing the calls raise; there is no
+other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkda_b200.so")
+
+KDA_DTYPE_F32 = 0
+KDA_DTYPE_BF16 = 1
+
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED_SHAPE",
+          3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_WORKSPACE_TOO_SMALL", 5: "KDA_ERR_CUDA",
+          6: "KDA_ERR_DEVICE_TIMEOUT", 7: "KDA_ERR_BAD_SEQLENS"}
+
+# Every symbol the header declares, with its ctypes signature.
+_VP, _SZ, _I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+SIGNATURES = {
+    "kda_version": ([], _I),
+    "kda_status_string": ([_I], ctypes.c_char_p),
+    "kda_fwd_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
+    "kda_fwd": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP,
+                 _SZ, _VP], _I),
+    "kda_fwd_intra": ([_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP],
+                      _I),
+    "kda_fwd_inter": ([_VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP], _I),
+    "kda_decode_step": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP], _I),
+    "kda_get_last_device_error": ([_VP], _I),
+}
+
+
+class KDAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({_status_string(code)})")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load the CUDA library (built by ``kimi_delta_attention_28_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with "
+                              "`python -m kimi_delta_attention_28_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+    return _lib
+
+
+def _status_string(code: int) -> str:
+    try:
+        return load_library().kda_status_string(code).decode()
+    except Exception:  # noqa: BLE001 - only used to decorate an error message
+        return "?"
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise KDAError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    if dt == torch.float32:
+        return KDA_DTYPE_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {dt}")
+
+
+def _need(t, name, dtype=None, device=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
+                   dtype: torch.dtype) -> int:
+    return int(load_library().kda_fwd_workspace_size(B, T, H, dk, dv, num_seqs,
+                                                      _dtype_code(dtype)))
+
+
+def kda_fwd(q, k, v, g, beta, h0=None, cu_seqlens=None, *, output_final_state: bool = True,
+            o=None, hT=None, workspace=None):
+    """Chunkwise KDA prefill through the C ABI.
+
+    q, k, g: [B, T, H, d_k]; v: [B, T, H, d_v] (q/k/v bf16 or fp32, g fp32);
+    beta: [B, T, H] fp32; h0: [N, H, d_k, d_v] fp32 or None (zeros);
+    cu_seqlens: int32 [N+1] packed offsets (then B == 1) or None.
+    Returns (o, hT); hT is None when output_final_state is False.
+    """
+    lib = load_library()
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q.dtype)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(h0, "h0", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = B if cu_seqlens is None else num_seqs
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=q.dtype, device=dev)
+    if hT is None and output_final_state:
+        hT = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    need = workspace_size(B, T, H, dk, dv, num_seqs, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.kda_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                       _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, dt, _ptr(o), _ptr(hT),
+                       _ptr(workspace), workspace.numel(), _stream(dev)), "kda_fwd")
+    return o, hT
+
+
+def kda_fwd_intra(q, k, v, g, beta, cu_seqlens=None, *, workspace):
+    """Phase 1 of the tensor-core prefill (bf16, d = 128): per-(chunk, head)
+    intra-chunk records into ``workspace``.  Same argument conventions as kda_fwd."""
+    lib = load_library()
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib.kda_fwd_intra(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                             num_seqs, B, T, H, dk, dv, _dtype_code(q.dtype), _ptr(workspace),
+                             workspace.numel(), _stream(dev)), "kda_fwd_intra")
+
+
+def kda_fwd_inter(h0, cu_seqlens, o, hT, *, B, T, H, dk, dv, dtype, workspace):
+    """Phase 2 of the tensor-core prefill: the state pass, writing o and hT."""
+    lib = load_library()
+    dev = o.device
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib.kda_fwd_inter(_ptr(h0), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv,
+                             _dtype_code(dtype), _ptr(o), _ptr(hT), _ptr(workspace),
+                             workspace.numel(), _stream(dev)), "kda_fwd_inter")
+
+
+def kda_decode_step(q, k, v, g, beta, S, o=None):
+    """One decode token per (sequence, head); S [N, H, d_k, d_v] fp32 is updated
+    in place.  q, k, g: [N, H, d_k]; v: [N, H, d_v]; beta: [N, H].  Returns o."""
+    lib = load_library()
+    dev = q.device
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q.dtype)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=q.dtype, device=dev)
+    _check(lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                               N, H, dk, dv, dt, _stream(dev)), "kda_decode_step")
+    return o
+
+
+def device_error(device=None) -> int:
+    """Synchronise and read/clear the library's device error word (0 = none)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda")
+    return int(load_library().kda_get_last_device_error(_stream(dev)))

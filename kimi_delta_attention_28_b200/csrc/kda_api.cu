@@ -1,0 +1,346 @@
+// kda_api.cu -- the library's C ABI (declared in include/kda.h).
+//
+// Host-side argument validation, workspace layout and kernel dispatch.  All
+// kernels are compiled into this one translation unit so they can share the
+// device error word without relocatable device code.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/kda.h"
+#include "kda_common.cuh"
+#include "kda_decode.cuh"
+#include "kda_prefill_simt.cuh"
+#include "kda_prefill_tc.cuh"
+
+// Sticky device error bits; read and cleared by kda_get_last_device_error.
+__device__ int g_kda_device_error = 0;
+
+namespace {
+
+constexpr int ERRBIT_SEQLENS = 1;
+constexpr int ERRBIT_TIMEOUT = 2;
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace layout of kda_fwd (all segments 256-byte aligned):
+//   header   : 2 ints (offsets-valid flag, total chunks)
+//   seq_off  : num_seqs + 1 ints
+//   chunks   : max_chunks ChunkLoc
+//   records  : max_chunks * H records of tc::REC_BYTES (tensor-core path only)
+struct WsLayout {
+    size_t hdr, seq_off, chunks, recs, total;
+    long long max_chunks;
+};
+
+inline bool is_tc_path(int dtype, int dk) { return dtype == KDA_DTYPE_BF16 && dk == 128; }
+
+WsLayout ws_layout(int B, int T, int H, int dk, int num_seqs, int dtype) {
+    WsLayout L{};
+    const bool varlen = num_seqs > 0;
+    const int chunk = is_tc_path(dtype, dk) ? kda::tc::C : kda::simt::C;
+    if (varlen)
+        L.max_chunks = ((long long)T + chunk - 1) / chunk + num_seqs;
+    else
+        L.max_chunks = (long long)B * (((long long)T + chunk - 1) / chunk);
+    L.hdr = 0;
+    L.seq_off = 256;
+    L.chunks = round_up(L.seq_off + sizeof(int) * (size_t)(num_seqs + 1), 256);
+    L.recs = round_up(L.chunks + (varlen ? sizeof(kda::tc::ChunkLoc) * (size_t)L.max_chunks : 0),
+                      256);
+    L.total = L.recs;
+    if (is_tc_path(dtype, dk)) L.total += (size_t)L.max_chunks * H * kda::tc::REC_BYTES;
+    return L;
+}
+
+kda_status check_shape(int H, int dk, int dv, int dtype) {
+    if (H <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (dk != dv) return KDA_ERR_UNSUPPORTED_SHAPE;
+    if (dk != 32 && dk != 64 && dk != 128) return KDA_ERR_UNSUPPORTED_SHAPE;
+    return KDA_OK;
+}
+
+kda_status launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+template <int D, typename TIn>
+kda_status launch_simt(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *h0, float *hT, void *o, int T, int H,
+                       int nunits, const int *hdr, const int *cu, cudaStream_t s) {
+    const size_t smem = sizeof(kda::simt::SimtSmem<D>);
+    auto kern = kda::simt::kda_simt_fwd_kernel<D, TIn>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return KDA_ERR_CUDA;
+    kern<<<nunits, kda::simt::NT, smem, s>>>(
+        static_cast<const TIn *>(q), static_cast<const TIn *>(k), static_cast<const TIn *>(v), g,
+        beta, h0, hT, static_cast<TIn *>(o), T, H, hdr, cu);
+    return launch_status();
+}
+
+template <typename TIn>
+kda_status dispatch_simt(int D, const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, const float *h0, float *hT, void *o, int T, int H,
+                         int nunits, const int *hdr, const int *cu, cudaStream_t s) {
+    switch (D) {
+        case 32: return launch_simt<32, TIn>(q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr, cu, s);
+        case 64: return launch_simt<64, TIn>(q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr, cu, s);
+        case 128:
+            return launch_simt<128, TIn>(q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr, cu, s);
+        default: return KDA_ERR_UNSUPPORTED_SHAPE;
+    }
+}
+
+template <int DVT>
+kda_status launch_state(const uint8_t *recs, const float *h0, float *hT, void *o, int T, int H,
+                        int cps, int nunits, const int *hdr, const int *seq_off, const int *cu,
+                        cudaStream_t s) {
+    using namespace kda::tc;
+    const size_t smem = sizeof(StateSmem<DVT>);
+    auto kern = kda_tc_state_kernel<DVT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return KDA_ERR_CUDA;
+    const unsigned grid = (unsigned)nunits * (D / DVT);
+    kern<<<grid, 128, smem, s>>>(recs, h0, hT, static_cast<__nv_bfloat16 *>(o), T, H, cps, hdr,
+                                 seq_off, cu);
+    return launch_status();
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_version(void) { return 100; }
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: null pointer, negative size or bad dtype";
+        case KDA_ERR_UNSUPPORTED_SHAPE: return "KDA_ERR_UNSUPPORTED_SHAPE: need d_k == d_v in {32, 64, 128}";
+        case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED: tensor pointers must be 16-byte aligned";
+        case KDA_ERR_WORKSPACE_TOO_SMALL: return "KDA_ERR_WORKSPACE_TOO_SMALL";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA launch or query failed";
+        case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
+        case KDA_ERR_BAD_SEQLENS: return "KDA_ERR_BAD_SEQLENS: cu_seqlens not monotone or out of range";
+        default: return "KDA_ERR_UNKNOWN";
+    }
+}
+
+size_t kda_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype) {
+    if (B < 0 || T < 0 || num_seqs < 0) return 0;
+    if (check_shape(H, dk, dv, dtype) != KDA_OK) return 0;
+    if (num_seqs > 0 && B != 1) return 0;
+    return ws_layout(B, T, H, dk, num_seqs, dtype).total;
+}
+
+// Shared validation of the prefill entry points.  Fills N (the number of
+// sequences) and the workspace layout.
+static kda_status validate_fwd(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *h0, const int32_t *cu,
+                               int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
+                               const void *o, const float *hT, const void *workspace,
+                               size_t ws_bytes, bool need_inputs, bool need_outputs, int *N,
+                               WsLayout *L) {
+    if (B < 0 || T < 0 || num_seqs < 0) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_shape(H, dk, dv, dtype);
+    if (st != KDA_OK) return st;
+    const bool varlen = cu != nullptr;
+    if (varlen && (B != 1 || num_seqs <= 0)) return KDA_ERR_INVALID_ARG;
+    if (!varlen && num_seqs != 0) return KDA_ERR_INVALID_ARG;
+    *N = varlen ? num_seqs : B;
+    const long long ntok = (long long)B * T;
+    if (need_inputs && ntok > 0 && (!q || !k || !v || !g || !beta)) return KDA_ERR_INVALID_ARG;
+    if (need_outputs && ntok > 0 && !o) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, h0, o, hT, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    if (cu && (reinterpret_cast<uintptr_t>(cu) & 3u)) return KDA_ERR_MISALIGNED;
+    // outputs must not alias inputs (hT == h0 is the one allowed overlap)
+    if (o && (o == q || o == k || o == v || o == g || o == beta)) return KDA_ERR_INVALID_ARG;
+    *L = ws_layout(B, T, H, dk, varlen ? num_seqs : 0, dtype);
+    if (!workspace || ws_bytes < L->total) return KDA_ERR_WORKSPACE_TOO_SMALL;
+    if ((long long)(*N) * H * 8 > 0x7fffffffLL || L->max_chunks > 0x7fffffffLL)
+        return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
+static int *device_error_word() {
+    int *p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_kda_device_error) != cudaSuccess)
+        return nullptr;
+    return p;
+}
+
+// Tensor-core path, phase 1: chunk map (varlen) and the per-(chunk, head) records.
+static kda_status tc_intra(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const int32_t *cu, int N, int T, int H,
+                           const WsLayout &L, void *workspace, cudaStream_t s) {
+    using namespace kda::tc;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *hdr = reinterpret_cast<int *>(ws + L.hdr);
+    int *seq_off = reinterpret_cast<int *>(ws + L.seq_off);
+    auto *chunks = reinterpret_cast<ChunkLoc *>(ws + L.chunks);
+    kda_status st;
+    int cps = 0;
+    if (cu) {
+        int *err = device_error_word();
+        if (!err) return KDA_ERR_CUDA;
+        kda_chunk_map_kernel<<<1, 1024, 0, s>>>(cu, N, T, hdr, seq_off, chunks, err,
+                                                ERRBIT_SEQLENS);
+        if ((st = launch_status()) != KDA_OK) return st;
+    } else {
+        cps = (T + C - 1) / C;
+    }
+    if (L.max_chunks == 0) return KDA_OK;
+    const size_t smem = sizeof(PrepSmem);
+    if (cudaFuncSetAttribute(kda_tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    dim3 grid((unsigned)L.max_chunks, H);
+    kda_tc_prep_kernel<<<grid, 256, smem, s>>>(
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), g, beta, T, H, cps, hdr, cu ? chunks : nullptr,
+        ws + L.recs);
+    return launch_status();
+}
+
+// Tensor-core path, phase 2: the state pass over the records.
+static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int H,
+                           const WsLayout &L, void *o, float *hT, void *workspace,
+                           cudaStream_t s) {
+    using namespace kda::tc;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *hdr = reinterpret_cast<int *>(ws + L.hdr);
+    int *seq_off = reinterpret_cast<int *>(ws + L.seq_off);
+    const int cps = cu ? 0 : (T + C - 1) / C;
+    const int nunits = N * H;
+    // Narrow column tiles when there are too few chains to fill the GPU.
+    if ((long long)nunits * (D / 32) < 2LL * sm_count())
+        return launch_state<16>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
+    return launch_state<32>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
+}
+
+kda_status kda_fwd_intra(const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, const int32_t *cu_seqlens, int num_seqs, int B,
+                         int T, int H, int dk, int dv, int dtype, void *workspace,
+                         size_t ws_bytes, void *stream) {
+    int N;
+    WsLayout L;
+    kda_status st = validate_fwd(q, k, v, g, beta, nullptr, cu_seqlens, num_seqs, B, T, H, dk, dv,
+                                 dtype, nullptr, nullptr, workspace, ws_bytes, true, false, &N, &L);
+    if (st != KDA_OK) return st;
+    if (!is_tc_path(dtype, dk)) return KDA_ERR_UNSUPPORTED_SHAPE;
+    if (N == 0) return KDA_OK;
+    return tc_intra(q, k, v, g, beta, cu_seqlens, N, T, H, L, workspace,
+                    static_cast<cudaStream_t>(stream));
+}
+
+kda_status kda_fwd_inter(const float *h0, const int32_t *cu_seqlens, int num_seqs, int B, int T,
+                         int H, int dk, int dv, int dtype, void *o, float *hT, void *workspace,
+                         size_t ws_bytes, void *stream) {
+    int N;
+    WsLayout L;
+    kda_status st = validate_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, h0, cu_seqlens,
+                                 num_seqs, B, T, H, dk, dv, dtype, o, hT, workspace, ws_bytes,
+                                 false, true, &N, &L);
+    if (st != KDA_OK) return st;
+    if (!is_tc_path(dtype, dk)) return KDA_ERR_UNSUPPORTED_SHAPE;
+    if (N == 0) return KDA_OK;
+    return tc_inter(h0, cu_seqlens, N, T, H, L, o, hT, workspace,
+                    static_cast<cudaStream_t>(stream));
+}
+
+kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
+                   int B, int T, int H, int dk, int dv, int dtype, void *o, float *hT,
+                   void *workspace, size_t ws_bytes, void *stream) {
+    int N;
+    WsLayout L;
+    kda_status st = validate_fwd(q, k, v, g, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv,
+                                 dtype, o, hT, workspace, ws_bytes, true, true, &N, &L);
+    if (st != KDA_OK) return st;
+    if (N == 0) return KDA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (is_tc_path(dtype, dk)) {
+        if ((st = tc_intra(q, k, v, g, beta, cu_seqlens, N, T, H, L, workspace, s)) != KDA_OK)
+            return st;
+        return tc_inter(h0, cu_seqlens, N, T, H, L, o, hT, workspace, s);
+    }
+    // fp32 / small-head path
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *hdr = reinterpret_cast<int *>(ws + L.hdr);
+    if (cu_seqlens) {
+        int *err = device_error_word();
+        if (!err) return KDA_ERR_CUDA;
+        kda::tc::kda_chunk_map_kernel<<<1, 1024, 0, s>>>(
+            cu_seqlens, N, T, hdr, reinterpret_cast<int *>(ws + L.seq_off),
+            reinterpret_cast<kda::tc::ChunkLoc *>(ws + L.chunks), err, ERRBIT_SEQLENS);
+        if ((st = launch_status()) != KDA_OK) return st;
+    }
+    const int nunits = N * H;
+    if (dtype == KDA_DTYPE_F32)
+        return dispatch_simt<float>(dk, q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr,
+                                    cu_seqlens, s);
+    return dispatch_simt<__nv_bfloat16>(dk, q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr,
+                                        cu_seqlens, s);
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, float *S, void *o, int N, int H, int dk, int dv,
+                           int dtype, void *stream) {
+    if (N < 0) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_shape(H, dk, dv, dtype);
+    if (st != KDA_OK) return st;
+    if (N == 0) return KDA_OK;
+    if (!q || !k || !v || !g || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned grid = (unsigned)(N * H);
+    using namespace kda::dec;
+#define KDA_DEC(DD, TT)                                                                       \
+    kda_decode_kernel<DD, TT><<<grid, NT, 0, s>>>(                                            \
+        static_cast<const TT *>(q), static_cast<const TT *>(k), static_cast<const TT *>(v), g, \
+        beta, S, static_cast<TT *>(o))
+    if (dtype == KDA_DTYPE_BF16) {
+        if (dk == 32) KDA_DEC(32, __nv_bfloat16);
+        else if (dk == 64) KDA_DEC(64, __nv_bfloat16);
+        else KDA_DEC(128, __nv_bfloat16);
+    } else {
+        if (dk == 32) KDA_DEC(32, float);
+        else if (dk == 64) KDA_DEC(64, float);
+        else KDA_DEC(128, float);
+    }
+#undef KDA_DEC
+    return launch_status();
+}
+
+kda_status kda_get_last_device_error(void *stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_kda_device_error, sizeof(int)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_kda_device_error, &zero, sizeof(int)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (word & ERRBIT_SEQLENS) return KDA_ERR_BAD_SEQLENS;
+    if (word & ERRBIT_TIMEOUT) return KDA_ERR_DEVICE_TIMEOUT;
+    return KDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,133 @@
+"""The C-ABI library builds, loads and exports every symbol ``include/kda.h``
+declares; host-side argument validation answers with the documented status
+codes.  CPU only: every call here returns before any kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kimi_delta_attention_28_b200 as kda
+from kimi_delta_attention_28_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, WS_SMALL = 0, 1, 2, 3, 4
+BF16, F32 = 1, 0
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(kda_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("kda_fwd", "kda_decode_step", "kda_fwd_workspace_size", "kda_fwd_intra",
+              "kda_fwd_inter", "kda_get_last_device_error", "kda_status_string", "kda_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks a signature for {name}"
+
+
+def test_binding_declares_nothing_extra():
+    assert set(_lib.SIGNATURES) == set(declared_functions())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.kda_version() >= 100
+    for code in range(8):
+        s = lib.kda_status_string(code).decode()
+        assert s.startswith("KDA_")
+    assert lib.kda_status_string(99).decode() == "KDA_ERR_UNKNOWN"
+
+
+def test_workspace_size(lib):
+    ws = lib.kda_fwd_workspace_size
+    # tensor-core path stores one 74240-byte record per (64-token chunk, head)
+    a = ws(2, 4096, 8, 128, 128, 0, BF16)
+    b = ws(2, 4096 + 64, 8, 128, 128, 0, BF16)
+    assert b - a == 2 * 8 * 74240
+    assert ws(1, 100, 4, 128, 128, 3, BF16) > 0          # packed varlen
+    assert ws(2, 100, 4, 128, 128, 3, BF16) == 0         # packed needs B == 1
+    assert ws(1, 64, 4, 128, 64, 0, BF16) == 0           # d_k != d_v
+    assert ws(1, 64, 4, 96, 96, 0, BF16) == 0            # unsupported head size
+    assert ws(1, 64, 4, 128, 128, 0, 7) == 0             # bad dtype
+    assert 0 < ws(1, 64, 4, 32, 32, 0, F32) < 4096       # CUDA-core path: header only
+
+
+def _fwd(lib, ptr=0x10000, ws=1 << 40, **over):
+    a = dict(q=ptr, k=ptr, v=ptr, g=ptr, beta=ptr, h0=None, cu=None, num_seqs=0, B=1, T=64,
+             H=2, dk=128, dv=128, dtype=BF16, o=ptr + 0x100000, hT=None, work=ptr, ws=ws,
+             stream=None)
+    a.update(over)
+    return lib.kda_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["h0"], a["cu"],
+                       a["num_seqs"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["dtype"],
+                       a["o"], a["hT"], a["work"], a["ws"], a["stream"])
+
+
+def test_fwd_validation_before_launch(lib):
+    assert _fwd(lib, dtype=5) == INVALID
+    assert _fwd(lib, dk=64, dv=128) == UNSUPPORTED
+    assert _fwd(lib, dk=96, dv=96) == UNSUPPORTED
+    assert _fwd(lib, H=0) == INVALID
+    assert _fwd(lib, B=-1) == INVALID
+    assert _fwd(lib, q=None) == INVALID
+    assert _fwd(lib, o=None) == INVALID
+    assert _fwd(lib, q=0x10004) == MISALIGNED
+    assert _fwd(lib, hT=0x20008) == MISALIGNED
+    assert _fwd(lib, o=0x10000) == INVALID               # output aliases an input
+    assert _fwd(lib, ws=16) == WS_SMALL
+    assert _fwd(lib, work=None) == WS_SMALL
+    assert _fwd(lib, num_seqs=2) == INVALID              # offsets count without offsets
+    assert _fwd(lib, cu=0x30000, num_seqs=2, B=2) == INVALID   # packed needs B == 1
+    assert _fwd(lib, cu=0x30002, num_seqs=2) == MISALIGNED
+    # empty batch: valid, nothing to do, no launch
+    assert _fwd(lib, B=0) == OK
+
+
+def test_phase_entry_points_validate(lib):
+    p = 0x10000
+    assert lib.kda_fwd_intra(p, p, p, p, p, None, 0, 1, 64, 2, 32, 32, F32, p, 1 << 40,
+                             None) == UNSUPPORTED
+    assert lib.kda_fwd_inter(None, None, 0, 1, 64, 2, 128, 128, BF16, None, None, p, 1 << 40,
+                             None) == INVALID
+    assert lib.kda_fwd_inter(None, None, 0, 0, 64, 2, 128, 128, BF16, p, None, p, 1 << 40,
+                             None) == OK
+
+
+def test_decode_validation_before_launch(lib):
+    p = 0x10000
+    f = lib.kda_decode_step
+    assert f(p, p, p, p, p, p, p, 4, 2, 128, 64, BF16, None) == UNSUPPORTED
+    assert f(p, p, p, p, p, p, p, 4, 2, 128, 128, 9, None) == INVALID
+    assert f(p, p, p, p, p, None, p, 4, 2, 128, 128, BF16, None) == INVALID
+    assert f(p, p, p, p, p, p + 8, p, 4, 2, 128, 128, BF16, None) == MISALIGNED
+    assert f(p, p, p, p, p, p, p, 0, 2, 128, 128, BF16, None) == OK
+    assert f(p, p, p, p, p, p, p, -1, 2, 128, 128, BF16, None) == INVALID
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        kda.kda_fwd(x, x, x, x.float(), torch.zeros(1, 4, 1), None)
+
+
+def test_library_is_built_for_sm100a():
+    # the build recipe targets sm_100a only
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.FLAGS)
+    assert os.path.exists(build.LIB)
+    ctypes.CDLL(build.LIB)
