@@ -298,6 +298,77 @@ def run_ours(args, world, rank, local):
     return out
 
 
+def run_ours_decode(args, world, rank, local):
+    """Decode workload: 256 sequences x 96 heads x d=128, fp32 state updated in
+    place; each step consumes fresh pre-generated inputs (the state, 1.6 GB, is
+    larger than L2, so no flush is needed)."""
+    import torch
+    import kimi_delta_attention_28_b200 as kda
+    from kimi_delta_attention_28_b200 import workloads as W
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    kda.load_library()
+    w = W.DECODE
+    nsteps = args.warmup + args.steps
+    inp = W.make_decode_inputs(w.B, w.H, w.dk, w.dv, nsteps, w.dtype, w.seed + rank, dev)
+    S = inp["S"]
+    o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(t):
+        kda.kda_decode_step(inp["q"][t], inp["k"][t], inp["v"][t], inp["g"][t], inp["beta"][t],
+                            S, o)
+
+    for t in range(args.warmup):
+        step(t)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.02)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.perf_counter()
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.perf_counter()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.stop()
+    total_ms = ev[0].elapsed_time(ev[-1])
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if rank != 0:
+        return None
+    ms = total_ms / args.steps
+    units = w.B * w.H
+    per_unit = 2 * w.dk * w.dv * 4 + 3 * w.dk * 2 + w.dk * 4 + 4 + w.dv * 2
+    bytes_step = units * per_unit
+    hbm_peak, _, peak_src = load_peaks()
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    return {
+        "metric": "KDA decode steps/s (256 sequences x 96 heads, d=128, fp32 state in place)",
+        "value": world * 1e3 / ms, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "N": w.B, "H": w.H, "dk": w.dk, "dv": w.dv,
+                   "l2": "state (1.6 GB) larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "kernel": "kda_decode_kernel", "achieved": gbs,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                     "traffic": load_traffic("decode"),
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                     "algorithmic_bytes_per_launch": bytes_step},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+
+
 def load_traffic(which):
     """DRAM bytes per launch from the committed ncu summary, if one matches the
     current kernel build (see profiles/)."""
@@ -403,7 +474,8 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "long", "varlen"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "long", "varlen", "decode"],
+                    default="prefill")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -418,9 +490,14 @@ def main():
             return 0
         print(json.dumps(run_reference(args, world, rank)), flush=True)
         return 0
+    if args.impl == "reference" and args.workload == "decode":
+        ap.error("the reference arm covers the prefill workloads")
     world, rank, local = dist_setup(args)
     try:
-        out = run_ours(args, world, rank, local)
+        if args.workload == "decode":
+            out = run_ours_decode(args, world, rank, local)
+        else:
+            out = run_ours(args, world, rank, local)
         if out is not None:
             print(json.dumps(out), flush=True)
     finally:

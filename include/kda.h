@@ -17,8 +17,11 @@
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller, row-major and
- *     contiguous, 16-byte aligned (cu_seqlens: 4-byte aligned).  The library never allocates device memory
- *     and never synchronises the stream in the compute entry points.
+ *     contiguous.  Alignment: prefill q, k, v and the workspace 16 bytes, h0/hT
+ *     8 bytes, o two elements; the decode state S 16 bytes; everything else its
+ *     element size.  A violation returns KDA_ERR_MISALIGNED.  The library never
+ *     allocates device memory and never synchronises the stream in the compute
+ *     entry points.
  *   - q, k, g are [.., H, d_k]; v, o are [.., H, d_v]; beta is [.., H];
  *     states are [N, H, d_k, d_v] fp32 (d_k rows, d_v columns).
  *   - q, k, v and o share one dtype (kda_dtype); g, beta and states are fp32.
@@ -44,7 +47,7 @@ typedef enum {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARG = 1,          /* null pointer, negative size, bad dtype     */
     KDA_ERR_UNSUPPORTED_SHAPE = 2,    /* head size not supported                   */
-    KDA_ERR_MISALIGNED = 3,           /* a pointer is not 16-byte aligned          */
+    KDA_ERR_MISALIGNED = 3,           /* a pointer breaks its alignment rule       */
     KDA_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes < kda_fwd_workspace_size(...)    */
     KDA_ERR_CUDA = 5,                 /* a CUDA launch or query failed             */
     KDA_ERR_DEVICE_TIMEOUT = 6,       /* a bounded device-side wait gave up        */

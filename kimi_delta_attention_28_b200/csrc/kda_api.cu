@@ -22,7 +22,9 @@ namespace {
 constexpr int ERRBIT_SEQLENS = 1;
 constexpr int ERRBIT_TIMEOUT = 2;
 
-inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned_to(const void *p, size_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;  // NULL counts as aligned
+}
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout of kda_fwd (all segments 256-byte aligned):
@@ -129,7 +131,7 @@ const char *kda_status_string(kda_status s) {
         case KDA_OK: return "KDA_OK";
         case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: null pointer, negative size or bad dtype";
         case KDA_ERR_UNSUPPORTED_SHAPE: return "KDA_ERR_UNSUPPORTED_SHAPE: need d_k == d_v in {32, 64, 128}";
-        case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED: tensor pointers must be 16-byte aligned";
+        case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED: a pointer breaks its alignment rule (see kda.h)";
         case KDA_ERR_WORKSPACE_TOO_SMALL: return "KDA_ERR_WORKSPACE_TOO_SMALL";
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA launch or query failed";
         case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
@@ -163,10 +165,12 @@ static kda_status validate_fwd(const void *q, const void *k, const void *v, cons
     const long long ntok = (long long)B * T;
     if (need_inputs && ntok > 0 && (!q || !k || !v || !g || !beta)) return KDA_ERR_INVALID_ARG;
     if (need_outputs && ntok > 0 && !o) return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, g, beta, h0, o, hT, workspace};
-    for (const void *p : ptrs)
-        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
-    if (cu && (reinterpret_cast<uintptr_t>(cu) & 3u)) return KDA_ERR_MISALIGNED;
+    // 16 B: rows staged with 16-byte copies; 8 B: float2 state access; else natural.
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    if (!aligned_to(q, 16) || !aligned_to(k, 16) || !aligned_to(v, 16) ||
+        !aligned_to(workspace, 16) || !aligned_to(h0, 8) || !aligned_to(hT, 8) ||
+        !aligned_to(g, 4) || !aligned_to(beta, 4) || !aligned_to(cu, 4) || !aligned_to(o, 2 * es))
+        return KDA_ERR_MISALIGNED;
     // outputs must not alias inputs (hT == h0 is the one allowed overlap)
     if (o && (o == q || o == k || o == v || o == g || o == beta)) return KDA_ERR_INVALID_ARG;
     *L = ws_layout(B, T, H, dk, varlen ? num_seqs : 0, dtype);
@@ -305,9 +309,10 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
     if (st != KDA_OK) return st;
     if (N == 0) return KDA_OK;
     if (!q || !k || !v || !g || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, g, beta, S, o};
-    for (const void *p : ptrs)
-        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    if (!aligned_to(S, 16) || !aligned_to(q, es) || !aligned_to(k, es) || !aligned_to(v, es) ||
+        !aligned_to(o, es) || !aligned_to(g, 4) || !aligned_to(beta, 4))
+        return KDA_ERR_MISALIGNED;
     if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const unsigned grid = (unsigned)(N * H);
@@ -344,3 +349,4 @@ kda_status kda_get_last_device_error(void *stream) {
 }
 
 }  // extern "C"
+

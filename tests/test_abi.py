@@ -87,7 +87,9 @@ def test_fwd_validation_before_launch(lib):
     assert _fwd(lib, q=None) == INVALID
     assert _fwd(lib, o=None) == INVALID
     assert _fwd(lib, q=0x10004) == MISALIGNED
-    assert _fwd(lib, hT=0x20008) == MISALIGNED
+    assert _fwd(lib, hT=0x20004) == MISALIGNED
+    assert _fwd(lib, g=0x10002) == MISALIGNED
+    assert _fwd(lib, o=0x20002) == MISALIGNED            # bf16 o needs 4 bytes
     assert _fwd(lib, o=0x10000) == INVALID               # output aliases an input
     assert _fwd(lib, ws=16) == WS_SMALL
     assert _fwd(lib, work=None) == WS_SMALL
@@ -115,6 +117,7 @@ def test_decode_validation_before_launch(lib):
     assert f(p, p, p, p, p, p, p, 4, 2, 128, 128, 9, None) == INVALID
     assert f(p, p, p, p, p, None, p, 4, 2, 128, 128, BF16, None) == INVALID
     assert f(p, p, p, p, p, p + 8, p, 4, 2, 128, 128, BF16, None) == MISALIGNED
+    assert f(p, p, p, p, p + 2, p, p, 4, 2, 128, 128, BF16, None) == MISALIGNED
     assert f(p, p, p, p, p, p, p, 0, 2, 128, 128, BF16, None) == OK
     assert f(p, p, p, p, p, p, p, -1, 2, 128, 128, BF16, None) == INVALID
 
