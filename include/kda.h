@@ -51,7 +51,8 @@ typedef enum {
     KDA_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes < kda_fwd_workspace_size(...)    */
     KDA_ERR_CUDA = 5,                 /* a CUDA launch or query failed             */
     KDA_ERR_DEVICE_TIMEOUT = 6,       /* a bounded device-side wait gave up        */
-    KDA_ERR_BAD_SEQLENS = 7           /* cu_seqlens not monotone / out of range    */
+    KDA_ERR_BAD_SEQLENS = 7,          /* cu_seqlens not monotone / out of range    */
+    KDA_ERR_EXCEEDS_STATIC_SCRATCH = 8 /* kda_fwd_noalloc: problem too large       */
 } kda_status;
 
 typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
@@ -143,6 +144,44 @@ kda_status kda_fwd_inter(const float *h0, const int32_t *cu_seqlens, int num_seq
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const float *g,
                            const float *beta, float *S, void *o, int N, int H, int dk,
                            int dv, int dtype, void *stream);
+
+/*
+ * Allocation-free prefill.  The source pages have no counterpart to this entry
+ * point: it is a convenience of this library, not part of the method.
+ *
+ * Some callers cannot allocate device memory on the call path: code that a
+ * host framework or plugin interface hands only its input and output buffers,
+ * with no way to ask for scratch space, and code whose device-memory budget is
+ * fixed up front so that a per-call allocation (and the chance of it failing
+ * mid-request) is not allowed.  kda_fwd needs a caller-provided workspace; this
+ * variant instead uses one scratch array compiled into the library -- a
+ * file-scope __device__ array of KDA_NOALLOC_SCRATCH_BYTES (32 MiB) that every
+ * GPU which loads the library keeps until the process exits.  It calls no
+ * cudaMalloc or cudaFree and no allocating library routine.
+ *
+ * Arguments and results are those of kda_fwd without the workspace arguments.
+ * Only the tensor-core path is offered (bf16, d_k = d_v = 128); other dtypes or
+ * head sizes return KDA_ERR_UNSUPPORTED_SHAPE.
+ *
+ *   - Size limit: kda_fwd_workspace_size(B, T, H, 128, 128, num_seqs,
+ *     KDA_DTYPE_BF16) must not exceed KDA_NOALLOC_SCRATCH_BYTES, otherwise the
+ *     call returns KDA_ERR_EXCEEDS_STATIC_SCRATCH and launches nothing.  32 MiB
+ *     holds 451 (64-token chunk, head) records, e.g. B = 1, H = 8, T = 3,584.
+ *   - Set-up: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it.  Make that
+ *     first call on each device before any stream capture begins.
+ *   - Sharing: every call on a device uses the same array, which keeps whatever
+ *     the previous call left in it.  Nothing in it has to start at zero, because
+ *     each call writes every scratch byte it later reads.  Calls whose work
+ *     overlaps on the GPU (issued on different streams, or from different host
+ *     threads without ordering) race on the array and corrupt each other's
+ *     results: order them on one stream or with events.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (32u << 20)
+kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const float *h0, const int32_t *cu_seqlens,
+                           int num_seqs, int B, int T, int H, int dk, int dv, int dtype, void *o,
+                           float *hT, void *stream);
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error word

@@ -12,7 +12,8 @@ panel "KDA 单头递归"), as a C-ABI CUDA library:
 This package is the thin Python binding; ``include/kda.h`` is the interface.
 """
 from ._lib import (KDAError, device_error, kda_decode_step, kda_fwd,  # noqa: F401
-                   kda_fwd_inter, kda_fwd_intra, load_library, workspace_size)
+                   kda_fwd_inter, kda_fwd_intra, kda_fwd_noalloc, load_library,
+                   workspace_size)
 
-__all__ = ["kda_fwd", "kda_fwd_intra", "kda_fwd_inter", "kda_decode_step",
+__all__ = ["kda_fwd", "kda_fwd_intra", "kda_fwd_inter", "kda_fwd_noalloc", "kda_decode_step",
            "workspace_size", "device_error", "load_library", "KDAError"]

@@ -20,7 +20,11 @@ KDA_DTYPE_BF16 = 1
 
 STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED_SHAPE",
           3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_WORKSPACE_TOO_SMALL", 5: "KDA_ERR_CUDA",
-          6: "KDA_ERR_DEVICE_TIMEOUT", 7: "KDA_ERR_BAD_SEQLENS"}
+          6: "KDA_ERR_DEVICE_TIMEOUT", 7: "KDA_ERR_BAD_SEQLENS",
+          8: "KDA_ERR_EXCEEDS_STATIC_SCRATCH"}
+
+# Size of the static scratch array behind kda_fwd_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 # Every symbol the header declares, with its ctypes signature.
 _VP, _SZ, _I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
@@ -35,6 +39,8 @@ SIGNATURES = {
     "kda_fwd_inter": ([_VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP], _I),
     "kda_decode_step": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP], _I),
     "kda_get_last_device_error": ([_VP], _I),
+    "kda_fwd_noalloc": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP,
+                         _VP], _I),
 }
 
 
@@ -187,6 +193,30 @@ def kda_decode_step(q, k, v, g, beta, S, o=None):
     _check(lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
                                N, H, dk, dv, dt, _stream(dev)), "kda_decode_step")
     return o
+
+
+def kda_fwd_noalloc(q, k, v, g, beta, h0, cu_seqlens, o, hT):
+    """Prefill through the allocation-free entry point: the library uses its
+    built-in static scratch array instead of a workspace.  For callers that
+    cannot allocate device memory per call; the caller passes every buffer,
+    including the outputs o and hT (hT may be None), and this wrapper allocates
+    nothing.  bf16, d = 128 only; the problem must fit the 32 MiB scratch."""
+    lib = load_library()
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, n, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(h0, "h0", torch.float32, dev)
+    _need(hT, "hT", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _check(lib.kda_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                               _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, _dtype_code(q.dtype),
+                               _ptr(o), _ptr(hT), _stream(dev)), "kda_fwd_noalloc")
+    return o, hT
 
 
 def device_error(device=None) -> int:

@@ -7,6 +7,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/kda.h"
 #include "kda_common.cuh"
@@ -136,6 +137,9 @@ const char *kda_status_string(kda_status s) {
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA launch or query failed";
         case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
         case KDA_ERR_BAD_SEQLENS: return "KDA_ERR_BAD_SEQLENS: cu_seqlens not monotone or out of range";
+        case KDA_ERR_EXCEEDS_STATIC_SCRATCH:
+            return "KDA_ERR_EXCEEDS_STATIC_SCRATCH: problem needs more scratch than the 32 MiB "
+                   "static array of kda_fwd_noalloc; use kda_fwd with a workspace";
         default: return "KDA_ERR_UNKNOWN";
     }
 }
@@ -350,3 +354,52 @@ kda_status kda_get_last_device_error(void *stream) {
 
 }  // extern "C"
 
+// ---------------------------------------------------------------------------
+// kda_fwd_noalloc: the tensor-core prefill with its scratch in a static array.
+// ---------------------------------------------------------------------------
+// In host code this name is only a host-side stand-in for the device array; its
+// device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t g_kda_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoallocMaxDevices = 64;
+std::once_flag g_noalloc_once[kNoallocMaxDevices];
+void *g_noalloc_ptr[kNoallocMaxDevices];
+cudaError_t g_noalloc_err[kNoallocMaxDevices];
+
+// Device address of the static scratch on the current device (nullptr on error).
+void *noalloc_scratch() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices)
+        return nullptr;
+    std::call_once(g_noalloc_once[dev], [dev]() {
+        g_noalloc_err[dev] =
+            cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_kda_noalloc_scratch);
+    });
+    return g_noalloc_err[dev] == cudaSuccess ? g_noalloc_ptr[dev] : nullptr;
+}
+}  // namespace
+
+extern "C" kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v,
+                                      const float *g, const float *beta, const float *h0,
+                                      const int32_t *cu_seqlens, int num_seqs, int B, int T,
+                                      int H, int dk, int dv, int dtype, void *o, float *hT,
+                                      void *stream) {
+    // Host-side checks first, with a placeholder (aligned, non-null) workspace of
+    // unbounded size, so bad arguments return before any CUDA call.
+    int N;
+    WsLayout L;
+    void *placeholder = reinterpret_cast<void *>(uintptr_t(256));
+    kda_status st = validate_fwd(q, k, v, g, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv,
+                                 dtype, o, hT, placeholder, SIZE_MAX, true, true, &N, &L);
+    if (st != KDA_OK) return st;
+    if (!is_tc_path(dtype, dk)) return KDA_ERR_UNSUPPORTED_SHAPE;
+    if (L.total > (size_t)KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_EXCEEDS_STATIC_SCRATCH;
+    if (N == 0) return KDA_OK;
+    void *scratch = noalloc_scratch();
+    if (!scratch) return KDA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = tc_intra(q, k, v, g, beta, cu_seqlens, N, T, H, L, scratch, s)) != KDA_OK)
+        return st;
+    return tc_inter(h0, cu_seqlens, N, T, H, L, o, hT, scratch, s);
+}
