@@ -369,14 +369,29 @@ def run_ours_decode(args, world, rank, local):
     }
 
 
+def kernel_source_sha():
+    """sha256 over the CUDA sources of the library (identifies a kernel build)."""
+    import hashlib
+    src = os.path.join(ROOT, "kimi_delta_attention_28_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(src)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(src, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
 def load_traffic(which):
-    """DRAM bytes per launch from the committed ncu summary, if one matches the
-    current kernel build (see profiles/)."""
+    """DRAM bytes (read + write) per launch of kernel `which`, from the committed
+    ncu summary profiles/traffic.json -- only if it was taken on the current
+    kernel sources (same sha256), else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        return d.get(which)
+        if d.get("kernel_source_sha256") != kernel_source_sha():
+            return None
+        return d["per_launch_dram_bytes"].get(which)
     except Exception:  # noqa: BLE001
         return None
 

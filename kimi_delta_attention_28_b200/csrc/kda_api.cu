@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -66,6 +67,32 @@ kda_status check_shape(int H, int dk, int dv, int dtype) {
     return KDA_OK;
 }
 
+int *device_error_word() {
+    int *p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_kda_device_error) != cudaSuccess)
+        return nullptr;
+    return p;
+}
+
+// Test hook: KDA_TEST_DROP_FIRST_COPY=1 (read once per process) makes the state
+// pass skip the bulk copy of its first chunk, so its bounded wait runs out and
+// the call reports KDA_ERR_DEVICE_TIMEOUT.  Used only by the failure-path test.
+int debug_drop_first_copy() {
+    static const int v = [] {
+        const char *e = getenv("KDA_TEST_DROP_FIRST_COPY");
+        return (e && atoi(e) != 0) ? 1 : 0;
+    }();
+    return v;
+}
+
+int state_tile_override() {
+    static const int v = [] {
+        const char *e = getenv("KDA_STATE_TILE");
+        return e ? atoi(e) : 0;
+    }();
+    return v;
+}
+
 kda_status launch_status() {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -109,9 +136,11 @@ kda_status launch_state(const uint8_t *recs, const float *h0, float *hT, void *o
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return KDA_ERR_CUDA;
+    int *err = device_error_word();
+    if (!err) return KDA_ERR_CUDA;
     const unsigned grid = (unsigned)nunits * (D / DVT);
-    kern<<<grid, 128, smem, s>>>(recs, h0, hT, static_cast<__nv_bfloat16 *>(o), T, H, cps, hdr,
-                                 seq_off, cu);
+    kern<<<grid, 256, smem, s>>>(recs, h0, hT, static_cast<__nv_bfloat16 *>(o), T, H, cps, hdr,
+                                 seq_off, cu, err, debug_drop_first_copy());
     return launch_status();
 }
 
@@ -173,7 +202,7 @@ static kda_status validate_fwd(const void *q, const void *k, const void *v, cons
     const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
     if (!aligned_to(q, 16) || !aligned_to(k, 16) || !aligned_to(v, 16) ||
         !aligned_to(workspace, 16) || !aligned_to(h0, 8) || !aligned_to(hT, 8) ||
-        !aligned_to(g, 4) || !aligned_to(beta, 4) || !aligned_to(cu, 4) || !aligned_to(o, 2 * es))
+        !aligned_to(g, 8) || !aligned_to(beta, 4) || !aligned_to(cu, 4) || !aligned_to(o, 2 * es))
         return KDA_ERR_MISALIGNED;
     // outputs must not alias inputs (hT == h0 is the one allowed overlap)
     if (o && (o == q || o == k || o == v || o == g || o == beta)) return KDA_ERR_INVALID_ARG;
@@ -182,13 +211,6 @@ static kda_status validate_fwd(const void *q, const void *k, const void *v, cons
     if ((long long)(*N) * H * 8 > 0x7fffffffLL || L->max_chunks > 0x7fffffffLL)
         return KDA_ERR_INVALID_ARG;
     return KDA_OK;
-}
-
-static int *device_error_word() {
-    int *p = nullptr;
-    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_kda_device_error) != cudaSuccess)
-        return nullptr;
-    return p;
 }
 
 // Tensor-core path, phase 1: chunk map (varlen) and the per-(chunk, head) records.
@@ -234,8 +256,10 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
     int *seq_off = reinterpret_cast<int *>(ws + L.seq_off);
     const int cps = cu ? 0 : (T + C - 1) / C;
     const int nunits = N * H;
-    // Narrow column tiles when there are too few chains to fill the GPU.
-    if ((long long)nunits * (D / 32) < 2LL * sm_count())
+    // Narrow column tiles when there are too few chains to fill the GPU;
+    // KDA_STATE_TILE=16|32 overrides the choice (tuning knob).
+    const int forced = state_tile_override();
+    if (forced == 16 || (forced != 32 && (long long)nunits * (D / 32) < 2LL * sm_count()))
         return launch_state<16>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
     return launch_state<32>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
 }

@@ -81,3 +81,56 @@ KDA_DEVINL int frag_bk_row(int lane) { return (lane & 7) + (((lane >> 3) & 1) <<
 KDA_DEVINL int frag_bk_col(int lane) { return (lane >> 4) << 3; }                       // n off
 
 }  // namespace kda
+
+namespace kda {
+
+// ---- mbarrier / bulk-copy (TMA engine) primitives ----
+KDA_DEVINL void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+KDA_DEVINL void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::); }
+KDA_DEVINL void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::); }
+KDA_DEVINL void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+KDA_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+KDA_DEVINL uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+    return t;
+}
+// Wait for the barrier phase with a wall-clock limit.  Returns false on timeout.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
+KDA_DEVINL bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+KDA_DEVINL void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+        ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ---- swizzled tile layouts (16-byte chunks XOR-permuted by row) ----
+// Byte offset of bf16 element (r, c) in a [rows][128] tile with 256-byte rows.
+KDA_DEVINL int swz128(int r, int c) { return r * 256 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1); }
+// Byte offset of bf16 element (r, c) in a [rows][64] tile with 128-byte rows.
+KDA_DEVINL int swz64(int r, int c) { return r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1); }
+
+}  // namespace kda
