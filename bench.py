@@ -126,6 +126,14 @@ def workload_inputs(name, device, seed_offset=0):
     return w, W.make_workload(w, device)
 
 
+def record_bytes():
+    """Bytes of one (64-token chunk, head) record of the tensor-core path."""
+    import torch
+    import kimi_delta_attention_28_b200 as kda
+    return (kda.workspace_size(1, 64, 1, 128, 128, 0, torch.bfloat16)
+            - kda.workspace_size(1, 0, 1, 128, 128, 0, torch.bfloat16))
+
+
 def algorithmic(w, inp):
     """Units and algorithmic byte / flop counts of one prefill step."""
     ntok = inp["q"].shape[0] * inp["q"].shape[1]          # tokens (each with H heads)
@@ -138,7 +146,7 @@ def algorithmic(w, inp):
     per_unit_out = w.dv * io                                 # o
     compulsory = units * (per_unit_in + per_unit_out) + chains * state_bytes * (
         2 if inp["h0"] is not None else 1)
-    rec_per_unit = 74240 / 64                                # intra-chunk record bytes per token-head
+    rec_per_unit = record_bytes() / 64                       # intra-chunk record bytes per token-head
     intra_bytes = units * (per_unit_in + rec_per_unit)
     inter_bytes = units * (rec_per_unit + per_unit_out) + chains * state_bytes * (
         2 if inp["h0"] is not None else 1)

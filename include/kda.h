@@ -64,10 +64,10 @@ int kda_version(void);
 const char *kda_status_string(kda_status s);
 
 /*
- * Bytes of device workspace that kda_fwd needs for these sizes.  The chunkwise
- * path stores, per 64-token chunk and head, the intra-chunk transform results
- * (the delta-rule factors W and U, the decayed keys and queries, the masked
- * query-key block and the chunk's total decay) that the state pass consumes.
+ * Bytes of device workspace that kda_fwd needs for these sizes.  The
+ * tensor-core path stores, per 64-token chunk and head, the chunk's affine map
+ * on the state (98,816 bytes: the state transition and offset, the output
+ * read-out and offset, and the chunk's total decay) that the state pass consumes.
  * Returns 0 for an invalid or unsupported combination.
  *   B, T      : fixed-length batch (B sequences of T tokens), or with
  *               num_seqs > 0 and packed input: B = 1, T = total tokens.
@@ -166,7 +166,7 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
  *   - Size limit: kda_fwd_workspace_size(B, T, H, 128, 128, num_seqs,
  *     KDA_DTYPE_BF16) must not exceed KDA_NOALLOC_SCRATCH_BYTES, otherwise the
  *     call returns KDA_ERR_EXCEEDS_STATIC_SCRATCH and launches nothing.  32 MiB
- *     holds 451 (64-token chunk, head) records, e.g. B = 1, H = 8, T = 3,584.
+ *     holds 339 (64-token chunk, head) records, e.g. B = 1, H = 8, T = 2,688.
  *   - Set-up: the first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it.  Make that
  *     first call on each device before any stream capture begins.

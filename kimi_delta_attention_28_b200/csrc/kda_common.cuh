@@ -134,3 +134,8 @@ KDA_DEVINL int swz128(int r, int c) { return r * 256 + ((((c >> 3) ^ (r & 7))) <
 KDA_DEVINL int swz64(int r, int c) { return r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1); }
 
 }  // namespace kda
+
+namespace kda {
+// Byte offset of bf16 element (r, c) in a [rows][256] tile with 512-byte rows.
+KDA_DEVINL int swz256(int r, int c) { return r * 512 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1); }
+}  // namespace kda

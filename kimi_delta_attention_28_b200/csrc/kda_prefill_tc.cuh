@@ -16,11 +16,12 @@
 // blocks with the pairwise decays factored through 16-token sub-tile reference
 // rows so no factor overflows (the same page's panel "g ∈ (-5, 0)" bounds a
 // 16-token decay by e^-80); [W|U] by blocked forward substitution (fp32 inverses
-// of the 16x16 diagonal blocks, tensor-core products elsewhere); the decayed keys
-// and queries.  It writes one record per (chunk, head).  Kernel 2
-// (kda_tc_state_kernel) walks the chunks of each (sequence, head) in order with
-// the fp32 state on chip, split over d_v column tiles (state columns evolve
-// independently); records arrive by bulk copies into a 3-stage ring.
+// of the 16x16 diagonal blocks, tensor-core products elsewhere); and from them
+// the chunk's affine map on the state (below), one record per (chunk, head).
+// Kernel 2 (kda_tc_state_kernel) walks the chunks of each (sequence, head) in
+// order with the fp32 state on chip, split over d_v column tiles (state columns
+// evolve independently), one product chain per chunk; records arrive by bulk
+// copies into a 3-stage ring.
 #pragma once
 
 #include "kda_common.cuh"
@@ -32,26 +33,35 @@ constexpr int D = 128;          // head size (d_k = d_v)
 constexpr int C = 64;           // chunk length
 constexpr int ST = 16;          // sub-tile length for the decay reference rows
 constexpr int NST = C / ST;     // sub-tiles per chunk
-constexpr int LD = D + 8;       // padded bf16 row stride of staged inputs (272 B)
-constexpr int LDY = 2 * D + 8;  // padded bf16 row stride of the [W|U] solution (528 B)
-constexpr int LDA = C + 8;      // padded bf16 row stride of the key-key block (144 B)
 
-// Per (chunk, head) record, written by kernel 1 and read by kernel 2.  The
-// [C][D] tiles use the swz128 layout (16-byte chunks XOR-permuted by row) so a
-// plain bulk copy lands them in shared memory ready for conflict-free ldmatrix.
-constexpr int REC_W = 0;                    // W                 [C][D] bf16, swz128
-constexpr int REC_KT = REC_W + C * D * 2;   // K*exp(G_C - G)    [C][D] bf16, swz128
-constexpr int REC_QG = REC_KT + C * D * 2;  // Q*exp(G)          [C][D] bf16, swz128
-constexpr int REC_AQK = REC_QG + C * D * 2; // masked query-key  [C][C] bf16, swz64
-constexpr int REC_GC = REC_AQK + C * C * 2; // exp(G_C)          [D] fp32
-constexpr int REC_SHARED = REC_GC + D * 4;  // bytes every column tile reads (57,856)
-constexpr int REC_U = REC_SHARED;           // U as 8 column tiles [8][C][16] bf16
-constexpr int UT = 16;                      // U tile width
-constexpr int REC_BYTES = REC_U + C * D * 2;  // 74,240
-static_assert(REC_BYTES % 256 == 0 && REC_SHARED % 16 == 0, "record alignment");
+// Per (chunk, head) record, written by kernel 1 and read by kernel 2: the
+// chunk's affine map.  With W, U, Kt = K*exp(G_C - G), Qg = Q*exp(G) and the
+// masked query-key block Aqk, a chunk takes the state S_in to
+//   S_out = Diag(exp G_C) S_in + M' S_in + R,   M' = -Kt^T W,  R = Kt^T U
+//   O     = Q' S_in + O0,                      Q' = Qg - Aqk W,  O0 = Aqk U
+// [rows][128] tiles use the swz128 layout (16-byte chunks XOR-permuted by row)
+// so a plain bulk copy lands them in shared memory ready for conflict-free
+// ldmatrix; R and O0 are stored as 16-column tiles so each column slice of the
+// state reads one contiguous block.
+constexpr int REC_M = 0;                     // M'        [D][D] bf16, swz128
+constexpr int REC_QP = REC_M + D * D * 2;    // Q'        [C][D] bf16, swz128
+constexpr int REC_GC = REC_QP + C * D * 2;   // exp(G_C)  [D] fp32
+constexpr int REC_SHARED = REC_GC + D * 4;   // bytes every column slice reads (49,664)
+constexpr int UT = 16;                       // column tile width of R and O0
+constexpr int REC_R = REC_SHARED;            // R   [D/UT][D][UT] bf16
+constexpr int REC_O0 = REC_R + D * D * 2;    // O0  [D/UT][C][UT] bf16
+constexpr int REC_BYTES = REC_O0 + C * D * 2;  // 98,816
+// Kt and Qg pass through the R and O0 areas of the record (swz128) before
+// those are written: kernel 1 needs them after its shared memory has been reused.
+constexpr int REC_KT_SCRATCH = REC_R;
+constexpr int REC_QG_SCRATCH = REC_O0;
+static_assert(REC_BYTES % 256 == 0 && REC_SHARED % 16 == 0 && REC_O0 % 16 == 0, "alignment");
 
-KDA_DEVINL int rec_u_off(int r, int c) {
-    return REC_U + (c >> 4) * (C * UT * 2) + r * (UT * 2) + (c & 15) * 2;
+KDA_DEVINL int rec_r_off(int r, int c) {
+    return REC_R + (c >> 4) * (D * UT * 2) + r * (UT * 2) + (c & 15) * 2;
+}
+KDA_DEVINL int rec_o0_off(int r, int c) {
+    return REC_O0 + (c >> 4) * (C * UT * 2) + r * (UT * 2) + (c & 15) * 2;
 }
 
 struct ChunkLoc {
@@ -118,22 +128,33 @@ __global__ void __launch_bounds__(1024) kda_chunk_map_kernel(const int *__restri
 // ---------------------------------------------------------------------------
 // Kernel 1: intra-chunk transform.  grid = (chunk slots, H), 256 threads.
 // ---------------------------------------------------------------------------
+constexpr int LDA = C + 8;      // padded bf16 row stride of the 64x64 blocks (144 B)
+constexpr int ZLD = 40;         // row stride of the per-warp substitution scratch
+
+// The six sub-tile pairs (a, b), b < a, of a 64-token chunk.
+__constant__ int2 kPairs[6] = {{1, 0}, {2, 0}, {3, 0}, {2, 1}, {3, 1}, {3, 2}};
+
 struct PrepSmem {
-    // kL/qL: raw k/q, then scaled left operands; afterwards the [W|U] solution
-    // (64 x LDY bf16 = 33,792 B spans both arrays, which are adjacent).
-    __nv_bfloat16 kL[C * LD];      // k * exp(G_r - G_ref(a))
-    __nv_bfloat16 qL[C * LD];      // q * exp(G_r - G_ref(a))
-    __nv_bfloat16 v[C * LD];       // raw v
-    __nv_bfloat16 kR[C * LD];      // k * exp(G_ref(b) - G_i); afterwards per-warp scratch
-    __nv_bfloat16 kG[C * LD];      // k * exp(G_r)
-    __nv_bfloat16 akkn[C * LDA];   // -b_r A_ri for sub-tile blocks b < a (bf16)
-    float akd[NST][ST][ST + 1];    //  b_r A_ri inside diagonal sub-tile blocks (fp32)
+    // Five 16 KB tiles in swz128 layout, reused across phases:
+    //   r0: k -> k*exp(G_r - G_ref(a)) ; then, with r1, the [W|U] solution (swz256)
+    //   r1: q -> q*exp(G_r - G_ref(a))
+    //   r2: v
+    //   r3: k*exp(G_ref(b) - G_i) ; then per-warp scratch ; then Kt
+    //   r4: k*exp(G_r) ; then Qg
+    uint8_t r0[C * D * 2], r1[C * D * 2], r2[C * D * 2], r3[C * D * 2], r4[C * D * 2];
+    __nv_bfloat16 akkn[C * LDA];   // -b_r A_ri, sub-tile blocks b < a (bf16)
+    __nv_bfloat16 aqk[C * LDA];    // masked query-key block (bf16)
     __nv_bfloat16 taa[NST][ST * (ST + 8)];  // (I + A_aa)^-1, bf16
-    float gref[NST][D];            // G at each sub-tile's reference row (log2 units)
-    float xch[NST][D];             // sub-tile decay totals
+    float mfac[6][D];              // exp(G_ref(a) - G_ref(b)) per pair and channel
+    union {
+        struct {
+            float tot[NST][D];     // sub-tile decay totals   (log2 units)
+            float ref[NST][D];     // sub-tile-local G at the reference row
+        } p1;
+        float akd[NST][ST][ST];    // b_r A_ri inside the diagonal sub-tile blocks
+    } u;
     float beta[C];
 };
-static_assert(sizeof(__nv_bfloat16) * C * LDY <= 2 * sizeof(__nv_bfloat16) * C * LD, "Y fits");
 
 __global__ void __launch_bounds__(256, 2)
 kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -160,6 +181,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     uint8_t *rec = recs + ((size_t)cid * H + h) * REC_BYTES;
     const size_t rowstride = (size_t)H * D;  // elements between consecutive tokens
     const size_t base = ((size_t)t0 * H + h) * D;
+    const uint32_t s0 = smem_u32(sm.r0), s1 = smem_u32(sm.r1), s2 = smem_u32(sm.r2);
+    const uint32_t s3 = smem_u32(sm.r3), s4 = smem_u32(sm.r4);
 
     // ---- P0: stage k, q, v rows (zero-filled past len) and beta ----
 #pragma unroll
@@ -169,7 +192,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         const int rem = i % (C * (D / 8));
         const int r = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
         const __nv_bfloat16 *src = (m == 0 ? k : (m == 1 ? q : v));
-        __nv_bfloat16 *dst = (m == 0 ? sm.kL : (m == 1 ? sm.qL : sm.v)) + r * LD + c8;
+        uint8_t *dst = (m == 0 ? sm.r0 : (m == 1 ? sm.r1 : sm.r2)) + swz128(r, c8);
         const bool ok = r < len;
         cp_async16(dst, ok ? (src + base + r * rowstride + c8) : src, ok ? 16 : 0);
     }
@@ -177,8 +200,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     if (tid < C) sm.beta[tid] = tid < len ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
 
     // ---- P1: cumulative decay and the scaled operands ----
-    // thread -> channel pair (2cp, 2cp+1) x sub-tile a (rows 16a..16a+15); log2 units.
-    const int cp = tid & 63, a1 = tid >> 6, c0 = 2 * cp;
+    // thread -> channel pair (c0, c0+1) x sub-tile a1 (rows 16a1..16a1+15).  gam holds
+    // the cumsum local to the sub-tile, in log2 units.
+    const int c0 = 2 * (tid & 63), a1 = tid >> 6;
     float2 gam[ST];
     {
         float2 run = make_float2(0.f, 0.f);
@@ -192,15 +216,25 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             run.y += gv.y * kLog2e;
             gam[j] = run;
         }
-        *reinterpret_cast<float2 *>(&sm.xch[a1][c0]) = run;
+        *reinterpret_cast<float2 *>(&sm.u.p1.tot[a1][c0]) = run;
+        *reinterpret_cast<float2 *>(&sm.u.p1.ref[a1][c0]) = gam[ST / 2 - 1];
     }
     cp_async_wait<0>();
     __syncthreads();
+    // pair factors exp(G_ref(a) - G_ref(b)) <= 1 for the off-diagonal sub-tile blocks
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+        const int e = tid + 256 * m, p = e >> 7, c = e & (D - 1);
+        const int pa = kPairs[p].x, pb = kPairs[p].y;
+        float d = sm.u.p1.ref[pa][c] - sm.u.p1.ref[pb][c];
+        for (int a = pb; a < pa; ++a) d += sm.u.p1.tot[a][c];
+        sm.mfac[p][c] = exp2f(d);
+    }
     {
         float2 Ba = make_float2(0.f, 0.f), GC = make_float2(0.f, 0.f);
 #pragma unroll
         for (int a = 0; a < NST; ++a) {
-            const float2 x = *reinterpret_cast<const float2 *>(&sm.xch[a][c0]);
+            const float2 x = *reinterpret_cast<const float2 *>(&sm.u.p1.tot[a][c0]);
             if (a < a1) {
                 Ba.x += x.x;
                 Ba.y += x.y;
@@ -208,38 +242,31 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             GC.x += x.x;
             GC.y += x.y;
         }
-#pragma unroll
-        for (int j = 0; j < ST; ++j) {
-            gam[j].x += Ba.x;
-            gam[j].y += Ba.y;
-        }
-        const float2 Gref = gam[ST / 2 - 1], Gend = gam[ST - 1];
-        *reinterpret_cast<float2 *>(&sm.gref[a1][c0]) = Gref;
-        // per-(sub-tile, channel) factors; every product below stays in [e^-80, e^40]
-        const float2 f1 = make_float2(exp2f(Ba.x - Gref.x), exp2f(Ba.y - Gref.y));      // >= 1
-        const float2 f2 = make_float2(exp2f(Gref.x - Gend.x), exp2f(Gref.y - Gend.y));  // >= 1
-        const float2 eB = make_float2(exp2f(Ba.x), exp2f(Ba.y));                        // <= 1
-        const float2 fC = make_float2(exp2f(GC.x - Gend.x), exp2f(GC.y - Gend.y));      // <= 1
+        const float2 Gref = gam[ST / 2 - 1], Gend = gam[ST - 1];   // local to the sub-tile
+        const float2 f1 = make_float2(exp2f(-Gref.x), exp2f(-Gref.y));                   // >= 1
+        const float2 f2 = make_float2(exp2f(Gref.x - Gend.x), exp2f(Gref.y - Gend.y));   // >= 1
+        const float2 eB = make_float2(exp2f(Ba.x), exp2f(Ba.y));                         // <= 1
+        const float2 fC = make_float2(exp2f(GC.x - Ba.x - Gend.x), exp2f(GC.y - Ba.y - Gend.y));
 #pragma unroll
         for (int j = 0; j < ST; ++j) {
             const int r = a1 * ST + j;
-            const float2 E1 = make_float2(exp2f(gam[j].x - Ba.x), exp2f(gam[j].y - Ba.y));
+            const int off = swz128(r, c0);
+            // every factor below lies in [e^-80, e^40] for g in (-5, 0]
+            const float2 E1 = make_float2(exp2f(gam[j].x), exp2f(gam[j].y));
             const float2 E2 = make_float2(exp2f(Gend.x - gam[j].x), exp2f(Gend.y - gam[j].y));
-            const float2 kf =
-                unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.kL + r * LD + c0));
-            const float2 qf =
-                unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.qL + r * LD + c0));
-            *reinterpret_cast<uint32_t *>(sm.kL + r * LD + c0) =
+            const float2 kf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.r0 + off));
+            const float2 qf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.r1 + off));
+            *reinterpret_cast<uint32_t *>(sm.r0 + off) =
                 pack_bf16x2(kf.x * E1.x * f1.x, kf.y * E1.y * f1.y);
-            *reinterpret_cast<uint32_t *>(sm.qL + r * LD + c0) =
+            *reinterpret_cast<uint32_t *>(sm.r1 + off) =
                 pack_bf16x2(qf.x * E1.x * f1.x, qf.y * E1.y * f1.y);
-            *reinterpret_cast<uint32_t *>(sm.kR + r * LD + c0) =
+            *reinterpret_cast<uint32_t *>(sm.r3 + off) =
                 pack_bf16x2(kf.x * E2.x * f2.x, kf.y * E2.y * f2.y);
-            *reinterpret_cast<uint32_t *>(sm.kG + r * LD + c0) =
+            *reinterpret_cast<uint32_t *>(sm.r4 + off) =
                 pack_bf16x2(kf.x * E1.x * eB.x, kf.y * E1.y * eB.y);
-            *reinterpret_cast<uint32_t *>(rec + REC_QG + swz128(r, c0)) =
+            *reinterpret_cast<uint32_t *>(rec + REC_QG_SCRATCH + off) =
                 pack_bf16x2(qf.x * E1.x * eB.x, qf.y * E1.y * eB.y);
-            *reinterpret_cast<uint32_t *>(rec + REC_KT + swz128(r, c0)) =
+            *reinterpret_cast<uint32_t *>(rec + REC_KT_SCRATCH + off) =
                 pack_bf16x2(kf.x * E2.x * fC.x, kf.y * E2.y * fC.y);
         }
         if (a1 == NST - 1)
@@ -248,92 +275,115 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     __syncthreads();
 
-    // ---- P2: A blocks.  warp -> (row sub-tile a, kind: 0 keys, 1 queries) ----
-    {
-        const int a = warp >> 1, kind = warp & 1;
-        const __nv_bfloat16 *left = kind ? sm.qL : sm.kL;
-        for (int b = 0; b <= a; ++b) {
-            float acc[2][4] = {};
+    // ---- P2: key-key and query-key blocks ----
+    // warps 0-5: one off-diagonal sub-tile pair each (both products share the
+    // rescaled right operand); warps 6-7: two diagonal blocks each, whose
+    // key-key blocks they also invert.
+    if (warp < 6) {
+        const int a = kPairs[warp].x, b = kPairs[warp].y;
+        float ak[2][4] = {}, aq[2][4] = {};
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            uint32_t lk[4], lq[4], bfr[4];
+            ldsm_x4(lk, s0 + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+            ldsm_x4(lq, s1 + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+            ldsm_x4(bfr, s3 + swz128(b * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
+            // right rows of sub-tile b move their reference from G_ref(b) to G_ref(a)
+            const int cc = ks * 16 + 2 * tig;
+            const float2 m01 = *reinterpret_cast<const float2 *>(&sm.mfac[warp][cc]);
+            const float2 m89 = *reinterpret_cast<const float2 *>(&sm.mfac[warp][cc + 8]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 x = unpack_bf16x2(bfr[u]);
+                bfr[u] = (u & 1) ? pack_bf16x2(x.x * m89.x, x.y * m89.y)
+                                 : pack_bf16x2(x.x * m01.x, x.y * m01.y);
+            }
+            mma_bf16_16816(ak[0], lk, bfr[0], bfr[1]);
+            mma_bf16_16816(ak[1], lk, bfr[2], bfr[3]);
+            mma_bf16_16816(aq[0], lq, bfr[0], bfr[1]);
+            mma_bf16_16816(aq[1], lq, bfr[2], bfr[3]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int r = a * ST + gid + 8 * hh, i = b * ST + nt * 8 + 2 * tig;
+                const float br = sm.beta[r];
+                *reinterpret_cast<uint32_t *>(sm.akkn + r * LDA + i) =
+                    pack_bf16x2(-ak[nt][2 * hh] * br, -ak[nt][2 * hh + 1] * br);
+                *reinterpret_cast<uint32_t *>(sm.aqk + r * LDA + i) =
+                    pack_bf16x2(aq[nt][2 * hh], aq[nt][2 * hh + 1]);
+            }
+    } else {
+        const int a0 = 2 * (warp - 6);
+        float aq[2][2][4] = {};
+#pragma unroll
+        for (int d = 0; d < 2; ++d) {
+            const int a = a0 + d;
+            float ak[2][4] = {};
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
-                uint32_t af[4], bfr[4];
-                ldsm_x4(af, smem_u32(left + (a * ST + frag_a_row(lane)) * LD + ks * 16 +
-                                     frag_a_col(lane)));
-                ldsm_x4(bfr, smem_u32(sm.kR + (b * ST + frag_bn_row(lane)) * LD + ks * 16 +
-                                      frag_bn_col(lane)));
-                if (b < a) {
-                    // right rows of sub-tile b move their reference from G_ref(b) to G_ref(a)
-                    const int cc = ks * 16 + 2 * tig;
-                    const float m0 = exp2f(sm.gref[a][cc] - sm.gref[b][cc]);
-                    const float m1 = exp2f(sm.gref[a][cc + 1] - sm.gref[b][cc + 1]);
-                    const float m8 = exp2f(sm.gref[a][cc + 8] - sm.gref[b][cc + 8]);
-                    const float m9 = exp2f(sm.gref[a][cc + 9] - sm.gref[b][cc + 9]);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 x = unpack_bf16x2(bfr[u]);
-                        bfr[u] = (u & 1) ? pack_bf16x2(x.x * m8, x.y * m9)
-                                         : pack_bf16x2(x.x * m0, x.y * m1);
-                    }
-                }
-                mma_bf16_16816(acc[0], af, bfr[0], bfr[1]);
-                mma_bf16_16816(acc[1], af, bfr[2], bfr[3]);
+                uint32_t lk[4], lq[4], bfr[4];
+                ldsm_x4(lk, s0 + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+                ldsm_x4(lq, s1 + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+                ldsm_x4(bfr, s3 + swz128(a * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
+                mma_bf16_16816(ak[0], lk, bfr[0], bfr[1]);
+                mma_bf16_16816(ak[1], lk, bfr[2], bfr[3]);
+                mma_bf16_16816(aq[d][0], lq, bfr[0], bfr[1]);
+                mma_bf16_16816(aq[d][1], lq, bfr[2], bfr[3]);
             }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const int rl = gid + 8 * hh, r = a * ST + rl;
-                    const int il = nt * 8 + 2 * tig, i = b * ST + il;
-                    float x0 = acc[nt][2 * hh], x1 = acc[nt][2 * hh + 1];
-                    if (kind == 0) {
-                        const float br = sm.beta[r];
-                        if (b == a) {
-                            sm.akd[a][rl][il] = (il < rl) ? x0 * br : 0.f;
-                            sm.akd[a][rl][il + 1] = (il + 1 < rl) ? x1 * br : 0.f;
-                        } else {
-                            *reinterpret_cast<uint32_t *>(sm.akkn + r * LDA + i) =
-                                pack_bf16x2(-x0 * br, -x1 * br);
-                        }
-                    } else {
-                        if (b == a) {
-                            x0 = (il <= rl) ? x0 : 0.f;
-                            x1 = (il + 1 <= rl) ? x1 : 0.f;
-                        }
-                        *reinterpret_cast<uint32_t *>(rec + REC_AQK + swz64(r, i)) =
-                            pack_bf16x2(x0, x1);
-                    }
+                    const int rl = gid + 8 * hh, il = nt * 8 + 2 * tig;
+                    const float br = sm.beta[a * ST + rl];
+                    sm.u.akd[a][rl][il] = (il < rl) ? ak[nt][2 * hh] * br : 0.f;
+                    sm.u.akd[a][rl][il + 1] = (il + 1 < rl) ? ak[nt][2 * hh + 1] * br : 0.f;
                 }
         }
-    }
-    __syncthreads();
-
-    // ---- P3: inverses of the 16x16 unit-lower diagonal blocks, fp32 ----
-    if (tid < C) {
-        const int a = tid >> 4, j = tid & 15;   // block a, column j: solve (I + A_aa) x = e_j
-        float x[ST];
+        __syncwarp();
+        {   // lane -> (block a0 + lane/16, column j): solve (I + A_aa) x = e_j in fp32
+            const int a = a0 + (lane >> 4), j = lane & 15;
+            float x[ST];
 #pragma unroll
-        for (int r = 0; r < ST; ++r) {
-            float s = (r == j) ? 1.f : 0.f;
-            if (r > j) {
+            for (int r = 0; r < ST; ++r) {
+                float sacc = (r == j) ? 1.f : 0.f;
+                if (r > j) {
 #pragma unroll
-                for (int i = 0; i < r; ++i)
-                    if (i >= j) s -= sm.akd[a][r][i] * x[i];
+                    for (int i = 0; i < r; ++i)
+                        if (i >= j) sacc -= sm.u.akd[a][r][i] * x[i];
+                }
+                x[r] = sacc;
             }
-            x[r] = s;
+#pragma unroll
+            for (int r = 0; r < ST; ++r) sm.taa[a][r * (ST + 8) + j] = f2bf(x[r]);
         }
 #pragma unroll
-        for (int r = 0; r < ST; ++r) sm.taa[a][r * (ST + 8) + j] = f2bf(x[r]);
+        for (int d = 0; d < 2; ++d)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int rl = gid + 8 * hh, il = nt * 8 + 2 * tig;
+                    const int r = (a0 + d) * ST + rl, i = (a0 + d) * ST + il;
+                    *reinterpret_cast<uint32_t *>(sm.aqk + r * LDA + i) =
+                        pack_bf16x2(il <= rl ? aq[d][nt][2 * hh] : 0.f,
+                                    il + 1 <= rl ? aq[d][nt][2 * hh + 1] : 0.f);
+                }
     }
     __syncthreads();
 
-    // ---- P4: [W|U] by blocked forward substitution, warp-local column slices ----
-    // warp w owns 32 columns: W[:, 32w..] (w < 4) or U[:, 32(w-4)..] (w >= 4).
+    // ---- P3: [W|U] = (I + A)^-1 Diag(b) [K*exp G | V] by blocked forward substitution ----
+    // warp w owns 32 columns of the solution Y (swz256 over r0..r1): W[:, 32w..] for
+    // w < 4, U[:, 32(w-4)..] for w >= 4.  Only warp-level syncs are needed.
     {
-        __nv_bfloat16 *Y = sm.kL;                       // [C][LDY]: solution rows so far
-        __nv_bfloat16 *Z = sm.kR + warp * (ST * 40);    // warp scratch [16][40]
-        const __nv_bfloat16 *X = warp < 4 ? sm.kG : sm.v;
-        const int xc = (warp & 3) * 32;                 // column base inside X / W / U
-        const int yc = warp * 32;                       // column base inside Y
+        const uint32_t sY = s0;
+        uint8_t *Yb = sm.r0;
+        __nv_bfloat16 *Z = reinterpret_cast<__nv_bfloat16 *>(sm.r3) + warp * (ST * ZLD);
+        const uint8_t *X = warp < 4 ? sm.r4 : sm.r2;
+        const int xc = (warp & 3) * 32;   // column base inside X
+        const int yc = warp * 32;         // column base inside Y
         for (int a = 0; a < NST; ++a) {
             float acc[4][4];
 #pragma unroll
@@ -341,8 +391,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int r = a * ST + gid + 8 * hh;
-                    const float2 x = unpack_bf16x2(
-                        *reinterpret_cast<const uint32_t *>(X + r * LD + xc + nt * 8 + 2 * tig));
+                    const float2 x = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
+                        X + swz128(r, xc + nt * 8 + 2 * tig)));
                     acc[nt][2 * hh] = sm.beta[r] * x.x;
                     acc[nt][2 * hh + 1] = sm.beta[r] * x.y;
                 }
@@ -353,8 +403,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
                 for (int np = 0; np < 2; ++np) {
                     uint32_t bb[4];
-                    ldsm_x4_t(bb, smem_u32(Y + (b * ST + frag_bk_row(lane)) * LDY + yc +
-                                           np * 16 + frag_bk_col(lane)));
+                    ldsm_x4_t(bb, sY + swz256(b * ST + frag_bk_row(lane),
+                                              yc + np * 16 + frag_bk_col(lane)));
                     mma_bf16_16816(acc[2 * np], af, bb[0], bb[1]);
                     mma_bf16_16816(acc[2 * np + 1], af, bb[2], bb[3]);
                 }
@@ -363,7 +413,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh)
-                    *reinterpret_cast<uint32_t *>(Z + (gid + 8 * hh) * 40 + nt * 8 + 2 * tig) =
+                    *reinterpret_cast<uint32_t *>(Z + (gid + 8 * hh) * ZLD + nt * 8 + 2 * tig) =
                         pack_bf16x2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
             __syncwarp();
             float y[4][4] = {};
@@ -372,7 +422,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t bz[4];
-                ldsm_x4_t(bz, smem_u32(Z + frag_bk_row(lane) * 40 + np * 16 + frag_bk_col(lane)));
+                ldsm_x4_t(bz, smem_u32(Z + frag_bk_row(lane) * ZLD + np * 16 + frag_bk_col(lane)));
                 mma_bf16_16816(y[2 * np], at, bz[0], bz[1]);
                 mma_bf16_16816(y[2 * np + 1], at, bz[2], bz[3]);
             }
@@ -381,34 +431,117 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int r = a * ST + gid + 8 * hh;
-                    const int cl = nt * 8 + 2 * tig;
-                    const uint32_t pk = pack_bf16x2(y[nt][2 * hh], y[nt][2 * hh + 1]);
-                    *reinterpret_cast<uint32_t *>(Y + r * LDY + yc + cl) = pk;
-                    if (warp < 4)
-                        *reinterpret_cast<uint32_t *>(rec + REC_W + swz128(r, xc + cl)) = pk;
-                    else
-                        *reinterpret_cast<uint32_t *>(rec + rec_u_off(r, xc + cl)) = pk;
+                    *reinterpret_cast<uint32_t *>(Yb + swz256(r, yc + nt * 8 + 2 * tig)) =
+                        pack_bf16x2(y[nt][2 * hh], y[nt][2 * hh + 1]);
                 }
             __syncwarp();
         }
+    }
+    __syncthreads();
+
+    // ---- P4: Kt and Qg back from the record's scratch area into r3 / r4 ----
+#pragma unroll
+    for (int it = 0; it < 2 * C * D * 2 / 16 / 256; ++it) {
+        const int i = tid + it * 256;                  // 16-byte chunk index
+        const int m = i / (C * D * 2 / 16), off = (i % (C * D * 2 / 16)) * 16;
+        cp_async16((m == 0 ? sm.r3 : sm.r4) + off,
+                   rec + (m == 0 ? REC_KT_SCRATCH : REC_QG_SCRATCH) + off);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // ---- P5: the chunk's affine map ----
+    // (a) M' = -Kt^T W and R = Kt^T U: warp w owns key rows 16w..16w+15.
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+        float acc[16][4] = {};
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks) {
+            uint32_t ak[4];
+            ldsm_x4_t(ak, s3 + swz128(ks * 16 + frag_at_row(lane), warp * 16 + frag_at_col(lane)));
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t bb[4];
+                ldsm_x4_t(bb, s0 + swz256(ks * 16 + frag_bk_row(lane),
+                                          half * D + np * 16 + frag_bk_col(lane)));
+                mma_bf16_16816(acc[2 * np], ak, bb[0], bb[1]);
+                mma_bf16_16816(acc[2 * np + 1], ak, bb[2], bb[3]);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int r = warp * 16 + gid + 8 * hh, c = nt * 8 + 2 * tig;
+                if (half == 0)
+                    *reinterpret_cast<uint32_t *>(rec + REC_M + swz128(r, c)) =
+                        pack_bf16x2(-acc[nt][2 * hh], -acc[nt][2 * hh + 1]);
+                else
+                    *reinterpret_cast<uint32_t *>(rec + rec_r_off(r, c)) =
+                        pack_bf16x2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+            }
+    }
+    // (b) Q' = Qg - Aqk W and O0 = Aqk U: warp -> chunk rows 16(w&3).., half w>>2.
+    {
+        const int mt = warp & 3, half = warp >> 2;
+        float acc[16][4];
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float2 x = make_float2(0.f, 0.f);
+                if (half == 0)
+                    x = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
+                        sm.r4 + swz128(mt * 16 + gid + 8 * hh, nt * 8 + 2 * tig)));
+                acc[nt][2 * hh] = -x.x;     // -Qg (negated back on store)
+                acc[nt][2 * hh + 1] = -x.y;
+            }
+        for (int ks = 0; ks <= mt; ++ks) {
+            uint32_t aa[4];
+            ldsm_x4(aa, smem_u32(sm.aqk + (mt * 16 + frag_a_row(lane)) * LDA + ks * 16 +
+                                 frag_a_col(lane)));
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t bb[4];
+                ldsm_x4_t(bb, s0 + swz256(ks * 16 + frag_bk_row(lane),
+                                          half * D + np * 16 + frag_bk_col(lane)));
+                mma_bf16_16816(acc[2 * np], aa, bb[0], bb[1]);
+                mma_bf16_16816(acc[2 * np + 1], aa, bb[2], bb[3]);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int r = mt * 16 + gid + 8 * hh, c = nt * 8 + 2 * tig;
+                if (half == 0)
+                    *reinterpret_cast<uint32_t *>(rec + REC_QP + swz128(r, c)) =
+                        pack_bf16x2(-acc[nt][2 * hh], -acc[nt][2 * hh + 1]);
+                else
+                    *reinterpret_cast<uint32_t *>(rec + rec_o0_off(r, c)) =
+                        pack_bf16x2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+            }
     }
 }
 
 // ---------------------------------------------------------------------------
 // Kernel 2: inter-chunk state pass.  grid = N * H * (D / DVT), 256 threads.
-// Warp w owns key rows 16w..16w+15 of the fp32 state tile S[:, col0:col0+DVT],
-// held in MMA accumulator registers; a bf16 copy in smem feeds W S and Qg S.
-// Chunk records arrive by bulk copies into a 3-stage mbarrier ring; every wait
-// is bounded (a wait that runs out sets the timeout bit and the CTA returns).
+// Per chunk: S <- Diag(exp G_C) S + M' S + R and O = Q' S + O0, one product
+// chain and one barrier.  Warp w owns key rows 16w..16w+15 of the fp32 state
+// tile S[:, col0:col0+DVT] (MMA accumulator registers); a double-buffered bf16
+// copy in smem is the B operand.  Warps w and w+4 share output rows 16(w&3)..
+// and split the tile's columns.  Records arrive by bulk copies into a 3-stage
+// mbarrier ring; every wait is bounded (on expiry: timeout bit, drain, return).
 // ---------------------------------------------------------------------------
 constexpr int NSTAGE = 3;
 
 template <int DVT>
 struct StateSmem {
-    static constexpr int STAGE_BYTES = REC_SHARED + C * DVT * 2;
-    uint8_t stage[NSTAGE][STAGE_BYTES];        // [W|Kt|Qg|Aqk|gC] + U tile(s)
-    __nv_bfloat16 sb[D * (DVT + 8)];           // bf16 copy of the state tile
-    __nv_bfloat16 db[C * (DVT + 8)];           // bf16 Delta tile
+    static constexpr int R_BYTES = D * DVT * 2, O0_BYTES = C * DVT * 2;
+    static constexpr int STAGE_BYTES = REC_SHARED + R_BYTES + O0_BYTES;
+    uint8_t stage[NSTAGE][STAGE_BYTES];        // [M'|Q'|gC] + R tile + O0 tile
+    __nv_bfloat16 sb[2][D * (DVT + 8)];        // bf16 copies of the state tile
     uint64_t full[NSTAGE];
 };
 
@@ -420,10 +553,10 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
                     const int *__restrict__ cu, int *err_word, int debug_drop_first_copy) {
     constexpr int NT = DVT / 8;    // n-tiles of the column tile
     constexpr int LDV = DVT + 8;
-    constexpr int STAGE_BYTES = StateSmem<DVT>::STAGE_BYTES;
-    static_assert(STAGE_BYTES % 128 == 0, "stage alignment");
+    using SM = StateSmem<DVT>;
+    static_assert(SM::STAGE_BYTES % 128 == 0, "stage alignment");
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    StateSmem<DVT> &sm = *reinterpret_cast<StateSmem<DVT> *>(smem_raw);
+    SM &sm = *reinterpret_cast<SM *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
     // 1-D grid, column tile fastest so the tiles of one chain run side by side
@@ -455,15 +588,17 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
         uint64_t *bar = &sm.full[j % NSTAGE];
         const uint8_t *rec = recs + ((size_t)(c_begin + j) * H + h) * REC_BYTES;
         uint8_t *dst = sm.stage[j % NSTAGE];
-        mbar_arrive_expect_tx(bar, STAGE_BYTES);
+        mbar_arrive_expect_tx(bar, SM::STAGE_BYTES);
         if (debug_drop_first_copy && j == 0) return;   // test hook: the wait must run out
         bulk_g2s(dst, rec, REC_SHARED, bar);
-        bulk_g2s(dst + REC_SHARED, rec + REC_U + tile * (C * DVT * 2), C * DVT * 2, bar);
+        bulk_g2s(dst + REC_SHARED, rec + REC_R + tile * SM::R_BYTES, SM::R_BYTES, bar);
+        bulk_g2s(dst + REC_SHARED + SM::R_BYTES, rec + REC_O0 + tile * SM::O0_BYTES,
+                 SM::O0_BYTES, bar);
     };
     if (tid == 0)
         for (int j = 0; j < NSTAGE && j < nchunks; ++j) issue(j);
 
-    // state rows 16w..16w+15 -> accumulator registers
+    // state rows 16w..16w+15 -> registers
     float S[NT][4];
     const size_t sbase = (size_t)chain * D * D;
 #pragma unroll
@@ -477,19 +612,21 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
             S[nt][2 * hh] = x.x;
             S[nt][2 * hh + 1] = x.y;
         }
-    auto store_sb = [&]() {
+    auto store_sb = [&](int buf) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int r = warp * 16 + gid + 8 * hh;
-                *reinterpret_cast<uint32_t *>(sm.sb + r * LDV + nt * 8 + 2 * tig) =
+                *reinterpret_cast<uint32_t *>(sm.sb[buf] + r * LDV + nt * 8 + 2 * tig) =
                     pack_bf16x2(S[nt][2 * hh], S[nt][2 * hh + 1]);
             }
     };
-    store_sb();
+    store_sb(0);
     __syncthreads();
 
+    const int rq = (warp & 3) * 16;       // output rows of this warp
+    const int oq = (warp >> 2) * (NT / 2);  // first output n-tile of this warp
     for (int j = 0; j < nchunks; ++j) {
         const int s = j % NSTAGE;
         if (!mbar_wait_bounded(&sm.full[s], (j / NSTAGE) & 1)) {
@@ -503,102 +640,77 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
             return;
         }
         const uint8_t *st = sm.stage[s];
-        const uint32_t sW = smem_u32(st + REC_W), sKt = smem_u32(st + REC_KT);
-        const uint32_t sQg = smem_u32(st + REC_QG), sA = smem_u32(st + REC_AQK);
+        const uint32_t sM = smem_u32(st + REC_M), sQ = smem_u32(st + REC_QP);
         const float *gc = reinterpret_cast<const float *>(st + REC_GC);
-        const __nv_bfloat16 *u = reinterpret_cast<const __nv_bfloat16 *>(st + REC_SHARED);
+        const uint8_t *rt = st + REC_SHARED;                 // R tile   [DVT/16][D][16]
+        const uint8_t *ot = st + REC_SHARED + SM::R_BYTES;   // O0 tile  [DVT/16][C][16]
+        const uint32_t sB = smem_u32(sm.sb[j & 1]);
         const int t0 = seq_t0 + j * C;
         const int len = min(C, seq_len - j * C);
 
-        // Phase A: warps 0-3 -> Delta = U - W S (rows 16w..), warps 4-7 -> Oq = Qg S
-        const int rw = (warp & 3) * 16;
-        const uint32_t sL = warp < 4 ? sW : sQg;
-        float P[NT][4] = {};
+        float acc[NT][4], oacc[NT / 2][4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = warp * 16 + gid + 8 * hh;
+            const float gr = gc[r];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int cl = nt * 8 + 2 * tig;
+                const float2 rr = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
+                    rt + (cl >> 4) * (D * UT * 2) + r * (UT * 2) + (cl & 15) * 2));
+                acc[nt][2 * hh] = gr * S[nt][2 * hh] + rr.x;
+                acc[nt][2 * hh + 1] = gr * S[nt][2 * hh + 1] + rr.y;
+            }
+            const int ro = rq + gid + 8 * hh;
+#pragma unroll
+            for (int i = 0; i < NT / 2; ++i) {
+                const int cl = (oq + i) * 8 + 2 * tig;
+                const float2 oo = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
+                    ot + (cl >> 4) * (C * UT * 2) + ro * (UT * 2) + (cl & 15) * 2));
+                oacc[i][2 * hh] = oo.x;
+                oacc[i][2 * hh + 1] = oo.y;
+            }
+        }
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-            uint32_t af[4];
-            ldsm_x4(af, sL + swz128(rw + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+            uint32_t am[4], aq[4];
+            ldsm_x4(am, sM + swz128(warp * 16 + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+            ldsm_x4(aq, sQ + swz128(rq + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
 #pragma unroll
             for (int np = 0; np < NT / 2; ++np) {
                 uint32_t b[4];
-                ldsm_x4_t(b, smem_u32(sm.sb + (ks * 16 + frag_bk_row(lane)) * LDV + np * 16 +
-                                      frag_bk_col(lane)));
-                mma_bf16_16816(P[2 * np], af, b[0], b[1]);
-                mma_bf16_16816(P[2 * np + 1], af, b[2], b[3]);
-            }
-        }
-        if (warp < 4) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int r = rw + gid + 8 * hh;
-                    const int cl = nt * 8 + 2 * tig;
-                    const float2 uu = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
-                        u + (cl >> 4) * (C * UT) + r * UT + (cl & 15)));
-                    *reinterpret_cast<uint32_t *>(sm.db + r * LDV + cl) =
-                        pack_bf16x2(uu.x - P[nt][2 * hh], uu.y - P[nt][2 * hh + 1]);
-                }
-        }
-        __syncthreads();
-
-        // Phase B: all warps update their 16 state rows: S = Diag(exp G_C) S + Kt^T Delta
-        {
-            const float g0 = gc[warp * 16 + gid], g8 = gc[warp * 16 + gid + 8];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                S[nt][0] *= g0;
-                S[nt][1] *= g0;
-                S[nt][2] *= g8;
-                S[nt][3] *= g8;
-            }
-#pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks) {
-                uint32_t ak[4];
-                ldsm_x4_t(ak, sKt + swz128(ks * 16 + frag_at_row(lane),
-                                           warp * 16 + frag_at_col(lane)));
-#pragma unroll
-                for (int np = 0; np < NT / 2; ++np) {
-                    uint32_t bd[4];
-                    ldsm_x4_t(bd, smem_u32(sm.db + (ks * 16 + frag_bk_row(lane)) * LDV +
-                                           np * 16 + frag_bk_col(lane)));
-                    mma_bf16_16816(S[2 * np], ak, bd[0], bd[1]);
-                    mma_bf16_16816(S[2 * np + 1], ak, bd[2], bd[3]);
-                }
-            }
-        }
-        // warps 4-7: O = Qg S + Aqk Delta (lower triangular: k-steps 0..rw/16)
-        if (warp >= 4) {
-            const int wr = warp - 4;
-#pragma unroll
-            for (int ks = 0; ks < C / 16; ++ks) {
-                if (ks <= wr) {
-                    uint32_t aa[4];
-                    ldsm_x4(aa, sA + swz64(rw + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-#pragma unroll
-                    for (int np = 0; np < NT / 2; ++np) {
-                        uint32_t bd[4];
-                        ldsm_x4_t(bd, smem_u32(sm.db + (ks * 16 + frag_bk_row(lane)) * LDV +
-                                               np * 16 + frag_bk_col(lane)));
-                        mma_bf16_16816(P[2 * np], aa, bd[0], bd[1]);
-                        mma_bf16_16816(P[2 * np + 1], aa, bd[2], bd[3]);
+                ldsm_x4_t(b, sB + 2 * ((ks * 16 + frag_bk_row(lane)) * LDV + np * 16 +
+                                       frag_bk_col(lane)));
+                mma_bf16_16816(acc[2 * np], am, b[0], b[1]);
+                mma_bf16_16816(acc[2 * np + 1], am, b[2], b[3]);
+                if constexpr (NT == 2) {
+                    if (oq == 0) mma_bf16_16816(oacc[0], aq, b[0], b[1]);
+                    else mma_bf16_16816(oacc[0], aq, b[2], b[3]);
+                } else {
+                    if (2 * np == oq) {
+                        mma_bf16_16816(oacc[0], aq, b[0], b[1]);
+                        mma_bf16_16816(oacc[1], aq, b[2], b[3]);
                     }
                 }
             }
+        }
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = rw + gid + 8 * hh;
-                if (r < len) {
-                    __nv_bfloat16 *orow = o + ((size_t)(t0 + r) * H + h) * D + col0;
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-                        *reinterpret_cast<uint32_t *>(orow + nt * 8 + 2 * tig) =
-                            pack_bf16x2(P[nt][2 * hh], P[nt][2 * hh + 1]);
-                }
+            for (int e = 0; e < 4; ++e) S[nt][e] = acc[nt][e];
+        store_sb((j + 1) & 1);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int r = rq + gid + 8 * hh;
+            if (r < len) {
+                __nv_bfloat16 *orow = o + ((size_t)(t0 + r) * H + h) * D + col0;
+#pragma unroll
+                for (int i = 0; i < NT / 2; ++i)
+                    *reinterpret_cast<uint32_t *>(orow + (oq + i) * 8 + 2 * tig) =
+                        pack_bf16x2(oacc[i][2 * hh], oacc[i][2 * hh + 1]);
             }
         }
-        store_sb();
-        __syncthreads();   // state copy ready; stage s and db free
+        __syncthreads();   // new state copy ready; stage s consumed
         if (tid == 0 && j + NSTAGE < nchunks) {
             fence_proxy_async_smem();   // order this chunk's generic reads before the refill
             issue(j + NSTAGE);

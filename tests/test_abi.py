@@ -56,10 +56,10 @@ def test_version_and_status_strings(lib):
 
 def test_workspace_size(lib):
     ws = lib.kda_fwd_workspace_size
-    # tensor-core path stores one 74240-byte record per (64-token chunk, head)
+    # tensor-core path stores one 98,816-byte record per (64-token chunk, head)
     a = ws(2, 4096, 8, 128, 128, 0, BF16)
     b = ws(2, 4096 + 64, 8, 128, 128, 0, BF16)
-    assert b - a == 2 * 8 * 74240
+    assert b - a == 2 * 8 * 98816
     assert ws(1, 100, 4, 128, 128, 3, BF16) > 0          # packed varlen
     assert ws(2, 100, 4, 128, 128, 3, BF16) == 0         # packed needs B == 1
     assert ws(1, 64, 4, 128, 64, 0, BF16) == 0           # d_k != d_v

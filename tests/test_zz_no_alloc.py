@@ -61,7 +61,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    # 57 chunks x 8 heads of 74,240-byte records exceed the 32 MiB array
+    # 57 chunks x 8 heads of 98,816-byte records exceed the 32 MiB array
     inp = W.make_prefill_inputs(1, 57 * 64, 8, 128, 128, torch.bfloat16, False, seed=23,
                                 device=DEV)
     o = torch.full((1, 57 * 64, 8, 128), 3.0, dtype=torch.bfloat16, device=DEV)
