@@ -17,8 +17,8 @@
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller, row-major and
- *     contiguous.  Alignment: prefill q, k, v and the workspace 16 bytes, g,
- *     h0 and hT 8 bytes, o two elements; the decode state S 16 bytes; everything
+ *     contiguous.  Alignment: prefill q, k, v, h0, hT and the workspace 16
+ *     bytes, g 8 bytes, o two elements; the decode state S 16 bytes; everything
  *     else its element size.  A violation returns KDA_ERR_MISALIGNED.  The library never
  *     allocates device memory and never synchronises the stream in the compute
  *     entry points.

@@ -131,7 +131,7 @@ kda_status launch_state(const uint8_t *recs, const float *h0, float *hT, void *o
                         int cps, int nunits, const int *hdr, const int *seq_off, const int *cu,
                         cudaStream_t s) {
     using namespace kda::tc;
-    const size_t smem = sizeof(StateSmem<DVT>);
+    const size_t smem = T5Layout<DVT>::BYTES;
     auto kern = kda_tc_state_kernel<DVT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
@@ -139,7 +139,7 @@ kda_status launch_state(const uint8_t *recs, const float *h0, float *hT, void *o
     int *err = device_error_word();
     if (!err) return KDA_ERR_CUDA;
     const unsigned grid = (unsigned)nunits * (D / DVT);
-    kern<<<grid, 256, smem, s>>>(recs, h0, hT, static_cast<__nv_bfloat16 *>(o), T, H, cps, hdr,
+    kern<<<grid, 128, smem, s>>>(recs, h0, hT, static_cast<__nv_bfloat16 *>(o), T, H, cps, hdr,
                                  seq_off, cu, err, debug_drop_first_copy());
     return launch_status();
 }
@@ -201,7 +201,7 @@ static kda_status validate_fwd(const void *q, const void *k, const void *v, cons
     // 16 B: rows staged with 16-byte copies; 8 B: float2 state access; else natural.
     const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
     if (!aligned_to(q, 16) || !aligned_to(k, 16) || !aligned_to(v, 16) ||
-        !aligned_to(workspace, 16) || !aligned_to(h0, 8) || !aligned_to(hT, 8) ||
+        !aligned_to(workspace, 16) || !aligned_to(h0, 16) || !aligned_to(hT, 16) ||
         !aligned_to(g, 8) || !aligned_to(beta, 4) || !aligned_to(cu, 4) || !aligned_to(o, 2 * es))
         return KDA_ERR_MISALIGNED;
     // outputs must not alias inputs (hT == h0 is the one allowed overlap)
@@ -234,7 +234,7 @@ static kda_status tc_intra(const void *q, const void *k, const void *v, const fl
         cps = (T + C - 1) / C;
     }
     if (L.max_chunks == 0) return KDA_OK;
-    const size_t smem = sizeof(PrepSmem);
+    const size_t smem = sizeof(PrepSmem) + 1024;   // + slack for 1024-byte alignment
     if (cudaFuncSetAttribute(kda_tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return KDA_ERR_CUDA;
@@ -242,7 +242,7 @@ static kda_status tc_intra(const void *q, const void *k, const void *v, const fl
     kda_tc_prep_kernel<<<grid, 256, smem, s>>>(
         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
         static_cast<const __nv_bfloat16 *>(v), g, beta, T, H, cps, hdr, cu ? chunks : nullptr,
-        ws + L.recs);
+        ws + L.recs, device_error_word());
     return launch_status();
 }
 
@@ -257,11 +257,11 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
     const int cps = cu ? 0 : (T + C - 1) / C;
     const int nunits = N * H;
     // Narrow column tiles when there are too few chains to fill the GPU;
-    // KDA_STATE_TILE=16|32 overrides the choice (tuning knob).
+    // KDA_STATE_TILE=32|64 overrides the choice (tuning knob).
     const int forced = state_tile_override();
-    if (forced == 16 || (forced != 32 && (long long)nunits * (D / 32) < 2LL * sm_count()))
-        return launch_state<16>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
-    return launch_state<32>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
+    if (forced == 32 || (forced != 64 && (long long)nunits * (D / 64) < (long long)sm_count()))
+        return launch_state<32>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
+    return launch_state<64>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
 }
 
 kda_status kda_fwd_intra(const void *q, const void *k, const void *v, const float *g,

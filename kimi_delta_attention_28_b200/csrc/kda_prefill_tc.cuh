@@ -20,8 +20,8 @@
 // the chunk's affine map on the state (below), one record per (chunk, head).
 // Kernel 2 (kda_tc_state_kernel) walks the chunks of each (sequence, head) in
 // order with the fp32 state on chip, split over d_v column tiles (state columns
-// evolve independently), one product chain per chunk; records arrive by bulk
-// copies into a 3-stage ring.
+// evolve independently): per chunk one pair of tcgen05 products (accumulated in
+// tensor memory) and one barrier; records arrive by bulk copies into a ring.
 #pragma once
 
 #include "kda_common.cuh"
@@ -39,29 +39,37 @@ constexpr int NST = C / ST;     // sub-tiles per chunk
 // masked query-key block Aqk, a chunk takes the state S_in to
 //   S_out = Diag(exp G_C) S_in + M' S_in + R,   M' = -Kt^T W,  R = Kt^T U
 //   O     = Q' S_in + O0,                      Q' = Qg - Aqk W,  O0 = Aqk U
-// [rows][128] tiles use the swz128 layout (16-byte chunks XOR-permuted by row)
-// so a plain bulk copy lands them in shared memory ready for conflict-free
-// ldmatrix; R and O0 are stored as 16-column tiles so each column slice of the
-// state reads one contiguous block.
-constexpr int REC_M = 0;                     // M'        [D][D] bf16, swz128
-constexpr int REC_QP = REC_M + D * D * 2;    // Q'        [C][D] bf16, swz128
+// The four matrices use the core-matrix layout (core_off): 8-column chunks
+// outermost, rows inside, 16 bytes per (row, chunk).  A warp whose lanes hold
+// consecutive rows writes 512 contiguous bytes per 16-byte store, the layout is
+// the tensor core's non-swizzled K-major operand layout (M' and Q' are A
+// operands of the state pass), and any 8-column-aligned slice of R or O0 is one
+// contiguous block.
+constexpr int REC_M = 0;                     // M'        [D][D] bf16, core_off(D, ...)
+constexpr int REC_QP = REC_M + D * D * 2;    // Q'        [C][D] bf16, core_off(C, ...)
 constexpr int REC_GC = REC_QP + C * D * 2;   // exp(G_C)  [D] fp32
 constexpr int REC_SHARED = REC_GC + D * 4;   // bytes every column slice reads (49,664)
-constexpr int UT = 16;                       // column tile width of R and O0
-constexpr int REC_R = REC_SHARED;            // R   [D/UT][D][UT] bf16
-constexpr int REC_O0 = REC_R + D * D * 2;    // O0  [D/UT][C][UT] bf16
+constexpr int REC_R = REC_SHARED;            // R         [D][D] bf16, core_off(D, ...)
+constexpr int REC_O0 = REC_R + D * D * 2;    // O0        [C][D] bf16, core_off(C, ...)
 constexpr int REC_BYTES = REC_O0 + C * D * 2;  // 98,816
-// Kt and Qg pass through the R and O0 areas of the record (swz128) before
-// those are written: kernel 1 needs them after its shared memory has been reused.
+// Kt and Qg pass through the R and O0 areas of the record (swizzled layouts)
+// before those are written: kernel 1 needs them after its shared memory has been reused.
 constexpr int REC_KT_SCRATCH = REC_R;
 constexpr int REC_QG_SCRATCH = REC_O0;
 static_assert(REC_BYTES % 256 == 0 && REC_SHARED % 16 == 0 && REC_O0 % 16 == 0, "alignment");
 
-KDA_DEVINL int rec_r_off(int r, int c) {
-    return REC_R + (c >> 4) * (D * UT * 2) + r * (UT * 2) + (c & 15) * 2;
+// Byte offset of bf16 element (r, c) of a [rows][D] matrix in the core-matrix layout.
+KDA_DEVINL int core_off(int rows, int r, int c) {
+    return (c >> 3) * (rows * 16) + r * 16 + ((c & 7) << 1);
 }
-KDA_DEVINL int rec_o0_off(int r, int c) {
-    return REC_O0 + (c >> 4) * (C * UT * 2) + r * (UT * 2) + (c & 15) * 2;
+
+// Byte offset of element (r, c) of a [rows][128] bf16 tile stored as two planes
+// (columns 0-63, then 64-127), each with 128-byte rows and the 16-byte chunks of
+// row r XOR-permuted by (r & 7): the K-major (or N-major) 128-byte-swizzled operand
+// layout the tcgen05 tensor core reads from shared memory (8-row groups 1024
+// bytes apart).
+KDA_DEVINL int umma_k128(int rows, int r, int c) {
+    return (c >> 6) * (rows * 128) + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
 }
 
 struct ChunkLoc {
@@ -143,7 +151,7 @@ struct PrepSmem {
     //   r4: k*exp(G_r) ; then Qg
     uint8_t r0[C * D * 2], r1[C * D * 2], r2[C * D * 2], r3[C * D * 2], r4[C * D * 2];
     __nv_bfloat16 akkn[C * LDA];   // -b_r A_ri, sub-tile blocks b < a (bf16)
-    __nv_bfloat16 aqk[C * LDA];    // masked query-key block (bf16)
+    uint8_t aqk[C * C * 2];        // masked query-key block, umma_k128 plane (bf16)
     __nv_bfloat16 taa[NST][ST * (ST + 8)];  // (I + A_aa)^-1, bf16
     float mfac[6][D];              // exp(G_ref(a) - G_ref(b)) per pair and channel
     union {
@@ -154,6 +162,8 @@ struct PrepSmem {
         float akd[NST][ST][ST];    // b_r A_ri inside the diagonal sub-tile blocks
     } u;
     float beta[C];
+    uint64_t mma_bar;              // tcgen05 completion barrier
+    uint32_t tmem_slot;            // tensor-memory base address (written by tcgen05.alloc)
 };
 
 __global__ void __launch_bounds__(256, 2)
@@ -161,9 +171,12 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
                    const float *__restrict__ beta, int T, int H, int cps,
                    const int *__restrict__ hdr, const ChunkLoc *__restrict__ chunks,
-                   uint8_t *__restrict__ recs) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    PrepSmem &sm = *reinterpret_cast<PrepSmem *>(smem_raw);
+                   uint8_t *__restrict__ recs, int *err_word) {
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment: the swizzled operand tiles are read by the tensor core
+    PrepSmem &sm = *reinterpret_cast<PrepSmem *>(
+        smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    uint32_t *tmem_slot = &sm.tmem_slot;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
     const int cid = blockIdx.x, h = blockIdx.y;
@@ -183,6 +196,15 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     const size_t base = ((size_t)t0 * H + h) * D;
     const uint32_t s0 = smem_u32(sm.r0), s1 = smem_u32(sm.r1), s2 = smem_u32(sm.r2);
     const uint32_t s3 = smem_u32(sm.r3), s4 = smem_u32(sm.r4);
+
+    if (warp == 0) {   // 256 tensor-memory columns for the P5 accumulators
+        t5::alloc(tmem_slot, 2 * D);
+        t5::relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(&sm.mma_bar, 1);
+        fence_mbar_init();
+    }
 
     // ---- P0: stage k, q, v rows (zero-filled past len) and beta ----
 #pragma unroll
@@ -266,7 +288,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 pack_bf16x2(kf.x * E1.x * eB.x, kf.y * E1.y * eB.y);
             *reinterpret_cast<uint32_t *>(rec + REC_QG_SCRATCH + off) =
                 pack_bf16x2(qf.x * E1.x * eB.x, qf.y * E1.y * eB.y);
-            *reinterpret_cast<uint32_t *>(rec + REC_KT_SCRATCH + off) =
+            *reinterpret_cast<uint32_t *>(rec + REC_KT_SCRATCH + umma_k128(C, r, c0)) =
                 pack_bf16x2(kf.x * E2.x * fC.x, kf.y * E2.y * fC.y);
         }
         if (a1 == NST - 1)
@@ -274,6 +296,14 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 make_float2(exp2f(GC.x), exp2f(GC.y));
     }
     __syncthreads();
+
+    // the query-key block is read whole by the tensor core: zero its upper blocks
+    if (tid < 6 * ST * 2) {
+        const int p = tid / (ST * 2), rr = (tid / 2) % ST, half = tid & 1;
+        const int ba = kPairs[p].y, bb = kPairs[p].x;   // block (row ba, column bb), bb > ba
+        *reinterpret_cast<uint4 *>(sm.aqk + umma_k128(C, ba * ST + rr, bb * ST + half * 8)) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
 
     // ---- P2: key-key and query-key blocks ----
     // warps 0-5: one off-diagonal sub-tile pair each (both products share the
@@ -311,7 +341,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 const float br = sm.beta[r];
                 *reinterpret_cast<uint32_t *>(sm.akkn + r * LDA + i) =
                     pack_bf16x2(-ak[nt][2 * hh] * br, -ak[nt][2 * hh + 1] * br);
-                *reinterpret_cast<uint32_t *>(sm.aqk + r * LDA + i) =
+                *reinterpret_cast<uint32_t *>(sm.aqk + umma_k128(C, r, i)) =
                     pack_bf16x2(aq[nt][2 * hh], aq[nt][2 * hh + 1]);
             }
     } else {
@@ -367,7 +397,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 for (int hh = 0; hh < 2; ++hh) {
                     const int rl = gid + 8 * hh, il = nt * 8 + 2 * tig;
                     const int r = (a0 + d) * ST + rl, i = (a0 + d) * ST + il;
-                    *reinterpret_cast<uint32_t *>(sm.aqk + r * LDA + i) =
+                    *reinterpret_cast<uint32_t *>(sm.aqk + umma_k128(C, r, i)) =
                         pack_bf16x2(il <= rl ? aq[d][nt][2 * hh] : 0.f,
                                     il + 1 <= rl ? aq[d][nt][2 * hh + 1] : 0.f);
                 }
@@ -375,7 +405,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     __syncthreads();
 
     // ---- P3: [W|U] = (I + A)^-1 Diag(b) [K*exp G | V] by blocked forward substitution ----
-    // warp w owns 32 columns of the solution Y (swz256 over r0..r1): W[:, 32w..] for
+    // warp w owns 32 columns of the solution Y (over r0..r1, four 64-column planes in
+    // the umma_k128 layout, the tensor core's N-contiguous B operand): W[:, 32w..] for
     // w < 4, U[:, 32(w-4)..] for w >= 4.  Only warp-level syncs are needed.
     {
         const uint32_t sY = s0;
@@ -403,8 +434,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
                 for (int np = 0; np < 2; ++np) {
                     uint32_t bb[4];
-                    ldsm_x4_t(bb, sY + swz256(b * ST + frag_bk_row(lane),
-                                              yc + np * 16 + frag_bk_col(lane)));
+                    ldsm_x4_t(bb, sY + umma_k128(C, b * ST + frag_bk_row(lane),
+                                                 yc + np * 16 + frag_bk_col(lane)));
                     mma_bf16_16816(acc[2 * np], af, bb[0], bb[1]);
                     mma_bf16_16816(acc[2 * np + 1], af, bb[2], bb[3]);
                 }
@@ -431,7 +462,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int r = a * ST + gid + 8 * hh;
-                    *reinterpret_cast<uint32_t *>(Yb + swz256(r, yc + nt * 8 + 2 * tig)) =
+                    *reinterpret_cast<uint32_t *>(Yb + umma_k128(C, r, yc + nt * 8 + 2 * tig)) =
                         pack_bf16x2(y[nt][2 * hh], y[nt][2 * hh + 1]);
                 }
             __syncwarp();
@@ -451,114 +482,168 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     cp_async_wait<0>();
     __syncthreads();
 
-    // ---- P5: the chunk's affine map ----
-    // (a) M' = -Kt^T W and R = Kt^T U: warp w owns key rows 16w..16w+15.
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-        float acc[16][4] = {};
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks) {
-            uint32_t ak[4];
-            ldsm_x4_t(ak, s3 + swz128(ks * 16 + frag_at_row(lane), warp * 16 + frag_at_col(lane)));
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                uint32_t bb[4];
-                ldsm_x4_t(bb, s0 + swz256(ks * 16 + frag_bk_row(lane),
-                                          half * D + np * 16 + frag_bk_col(lane)));
-                mma_bf16_16816(acc[2 * np], ak, bb[0], bb[1]);
-                mma_bf16_16816(acc[2 * np + 1], ak, bb[2], bb[3]);
-            }
-        }
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = warp * 16 + gid + 8 * hh, c = nt * 8 + 2 * tig;
-                if (half == 0)
-                    *reinterpret_cast<uint32_t *>(rec + REC_M + swz128(r, c)) =
-                        pack_bf16x2(-acc[nt][2 * hh], -acc[nt][2 * hh + 1]);
-                else
-                    *reinterpret_cast<uint32_t *>(rec + rec_r_off(r, c)) =
-                        pack_bf16x2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
-            }
-    }
-    // (b) Q' = Qg - Aqk W and O0 = Aqk U: warp -> chunk rows 16(w&3).., half w>>2.
+    // ---- P5: the chunk's affine map, on tcgen05 (accumulators in tensor memory) ----
+    //   D1 = Kt^T [W|U]  (M = 128 key rows, N = 256, K = 64): M' = -D1[:, :128], R = D1[:, 128:]
+    //   D2 = Aqk  [W|U]  (M = 64 chunk rows):                 Q' = Qg - D2[:, :128], O0 = D2[:, 128:]
+    // Both reuse the same 256 tensor-memory columns, one after the other.
     {
-        const int mt = warp & 3, half = warp >> 2;
-        float acc[16][4];
+        fence_proxy_async_smem();   // Y and aqk (generic stores), Kt (cp.async) -> tensor core
+        t5::fence_before_sync();
+        __syncthreads();
+        const uint32_t tmem = *tmem_slot;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint64_t ydesc = t5::smem_desc(s0, C * 128, 1024, t5::kSwz128);   // [W|U], N-major
+        if (warp == 0) {
+            if (t5::elect_one()) {
+                t5::fence_after_sync();
+                const uint64_t kdesc = t5::smem_desc(s3, C * 128, 1024, t5::kSwz128);  // Kt^T, M-major
+                constexpr uint32_t id = t5::idesc_bf16(128, 2 * D, 1, 1);
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float2 x = make_float2(0.f, 0.f);
-                if (half == 0)
-                    x = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
-                        sm.r4 + swz128(mt * 16 + gid + 8 * hh, nt * 8 + 2 * tig)));
-                acc[nt][2 * hh] = -x.x;     // -Qg (negated back on store)
-                acc[nt][2 * hh + 1] = -x.y;
+                for (int ks = 0; ks < C / 16; ++ks)
+                    t5::mma_bf16(tmem, kdesc + (uint64_t)((ks * 2048) >> 4),
+                                 ydesc + (uint64_t)((ks * 2048) >> 4), id, ks > 0);
+                t5::commit(&sm.mma_bar);
             }
-        for (int ks = 0; ks <= mt; ++ks) {
-            uint32_t aa[4];
-            ldsm_x4(aa, smem_u32(sm.aqk + (mt * 16 + frag_a_row(lane)) * LDA + ks * 16 +
-                                 frag_a_col(lane)));
+            __syncwarp();
+        }
+        bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 0));
+        t5::fence_after_sync();
+        if (ok) {   // lane = key row; warps 0-3 -> M' (columns 0..127), warps 4-7 -> R
+            const int m = (warp & 3) * 32 + lane, cb = (warp >> 2) * D;
 #pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                uint32_t bb[4];
-                ldsm_x4_t(bb, s0 + swz256(ks * 16 + frag_bk_row(lane),
-                                          half * D + np * 16 + frag_bk_col(lane)));
-                mma_bf16_16816(acc[2 * np], aa, bb[0], bb[1]);
-                mma_bf16_16816(acc[2 * np + 1], aa, bb[2], bb[3]);
+            for (int q = 0; q < D / 32; ++q) {
+                float v[32];
+                t5::ld32(tmem + lane_base + cb + q * 32, v);
+#pragma unroll
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    const int c = q * 32 + c8 * 8;
+                    const float sg = warp < 4 ? -1.f : 1.f;
+                    uint4 pk;
+                    pk.x = pack_bf16x2(sg * v[c8 * 8 + 0], sg * v[c8 * 8 + 1]);
+                    pk.y = pack_bf16x2(sg * v[c8 * 8 + 2], sg * v[c8 * 8 + 3]);
+                    pk.z = pack_bf16x2(sg * v[c8 * 8 + 4], sg * v[c8 * 8 + 5]);
+                    pk.w = pack_bf16x2(sg * v[c8 * 8 + 6], sg * v[c8 * 8 + 7]);
+                    uint8_t *dst = rec + (warp < 4 ? REC_M : REC_R) + core_off(D, m, c);
+                    *reinterpret_cast<uint4 *>(dst) = pk;
+                }
             }
         }
+        t5::fence_before_sync();
+        ok = __syncthreads_and(ok) != 0;
+        if (ok && warp == 0) {
+            if (t5::elect_one()) {
+                t5::fence_after_sync();
+                const uint64_t adesc = t5::smem_desc(smem_u32(sm.aqk), 16, 1024, t5::kSwz128);
+                constexpr uint32_t id = t5::idesc_bf16(64, 2 * D, 0, 1);
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = mt * 16 + gid + 8 * hh, c = nt * 8 + 2 * tig;
-                if (half == 0)
-                    *reinterpret_cast<uint32_t *>(rec + REC_QP + swz128(r, c)) =
-                        pack_bf16x2(-acc[nt][2 * hh], -acc[nt][2 * hh + 1]);
-                else
-                    *reinterpret_cast<uint32_t *>(rec + rec_o0_off(r, c)) =
-                        pack_bf16x2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+                for (int ks = 0; ks < C / 16; ++ks)
+                    t5::mma_bf16(tmem, adesc + (uint64_t)((ks * 32) >> 4),
+                                 ydesc + (uint64_t)((ks * 2048) >> 4), id, ks > 0);
+                t5::commit(&sm.mma_bar);
             }
+            __syncwarp();
+        }
+        ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 1));
+        t5::fence_after_sync();
+        if (ok) {   // rows r = 16(w&3) + lane (lanes 0..15); warps 0-3 -> Q', warps 4-7 -> O0
+            const int r = (warp & 3) * 16 + lane, cb = (warp >> 2) * D;
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) {
+                float v[32];
+                t5::ld32(tmem + lane_base + cb + q * 32, v);
+                if (lane < 16) {
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        const int c = q * 32 + c8 * 8;
+                        float x[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[e] = v[c8 * 8 + e];
+                        if (warp < 4) {   // Q' = Qg - Aqk W
+                            const uint4 qg = *reinterpret_cast<const uint4 *>(sm.r4 + swz128(r, c));
+                            const uint32_t u[4] = {qg.x, qg.y, qg.z, qg.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = unpack_bf16x2(u[e]);
+                                x[2 * e] = f.x - x[2 * e];
+                                x[2 * e + 1] = f.y - x[2 * e + 1];
+                            }
+                        }
+                        uint4 pk;
+                        pk.x = pack_bf16x2(x[0], x[1]);
+                        pk.y = pack_bf16x2(x[2], x[3]);
+                        pk.z = pack_bf16x2(x[4], x[5]);
+                        pk.w = pack_bf16x2(x[6], x[7]);
+                        uint8_t *dst = rec + (warp < 4 ? REC_QP : REC_O0) + core_off(C, r, c);
+                        *reinterpret_cast<uint4 *>(dst) = pk;
+                    }
+                }
+            }
+        }
+        if (!ok && tid == 0) atomicOr(err_word, ERR_TIMEOUT_BIT);
+        t5::fence_before_sync();
+        __syncthreads();
+        t5::fence_after_sync();
+        if (warp == 0) t5::dealloc(tmem, 2 * D);
     }
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 2: inter-chunk state pass.  grid = N * H * (D / DVT), 256 threads.
-// Per chunk: S <- Diag(exp G_C) S + M' S + R and O = Q' S + O0, one product
-// chain and one barrier.  Warp w owns key rows 16w..16w+15 of the fp32 state
-// tile S[:, col0:col0+DVT] (MMA accumulator registers); a double-buffered bf16
-// copy in smem is the B operand.  Warps w and w+4 share output rows 16(w&3)..
-// and split the tile's columns.  Records arrive by bulk copies into a 3-stage
-// mbarrier ring; every wait is bounded (on expiry: timeout bit, drain, return).
+// Kernel 2: inter-chunk state pass on tcgen05.  grid = N * H * (D / DVT), 128 threads.
+//
+// Thread t owns key row t of the fp32 state tile S[:, col0:col0+DVT] in registers.
+// Per chunk, one elected lane of warp 0 issues two tcgen05 products whose B
+// operand is a bf16 copy of the state in shared memory (double-buffered):
+//   D_S = M' S   (M = 128 key rows, N = DVT, K = 128) -> tensor memory columns [0, DVT)
+//   D_O = Q' S   (M = 64 chunk rows)                  -> columns [DVT, 2 DVT)
+// with separate completion barriers, so the state update S <- exp(G_C) S + R + D_S
+// (the loop-carried path) waits only for the first product while the second runs
+// behind it; rows 16w..16w+15 of warp w then form O = D_O + O0.  Records arrive by
+// bulk copies into a ring of stages, refilled by warp 1 so warp 0 can go straight
+// on to the next products.  Every wait is bounded; a wait that runs out makes the
+// whole CTA stop (block-wide vote), drain what it issued, free its tensor memory,
+// set the timeout bit and return.
 // ---------------------------------------------------------------------------
-constexpr int NSTAGE = 3;
-
 template <int DVT>
-struct StateSmem {
+struct T5Layout {
+    static_assert(DVT == 32 || DVT == 64, "column tile");
+    // the column tile's slices of R and O0: DVT/8 contiguous 8-column chunks each
     static constexpr int R_BYTES = D * DVT * 2, O0_BYTES = C * DVT * 2;
-    static constexpr int STAGE_BYTES = REC_SHARED + R_BYTES + O0_BYTES;
-    uint8_t stage[NSTAGE][STAGE_BYTES];        // [M'|Q'|gC] + R tile + O0 tile
-    __nv_bfloat16 sb[2][D * (DVT + 8)];        // bf16 copies of the state tile
-    uint64_t full[NSTAGE];
+    static constexpr int STAGE_RAW = REC_SHARED + R_BYTES + O0_BYTES;
+    static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
+    static constexpr int SB_BYTES = D * DVT * 2;        // one bf16 state copy (B operand)
+    static constexpr int SMEM_MAX = 232448;             // opt-in limit per CTA
+    static constexpr int NSTG_FIT = (SMEM_MAX - 2 * SB_BYTES - 2048) / STAGE_BYTES;
+    static constexpr int NSTG = NSTG_FIT > 4 ? 4 : NSTG_FIT;
+    static constexpr int OFF_SB = NSTG * STAGE_BYTES;
+    static constexpr int OFF_BAR = OFF_SB + 2 * SB_BYTES;   // full[NSTG], done_s, done_o
+    static constexpr int OFF_TMEM = OFF_BAR + 8 * (NSTG + 2);
+    static constexpr int BYTES = OFF_TMEM + 16 + 1024;      // + slack for 1024-byte alignment
+    static constexpr uint32_t TMEM_COLS = 2 * DVT;
+    // B operand (the state copy), MN-major: row k (key) holds DVT bf16 values.
+    // DVT = 64: 128-byte rows, 128-byte swizzle; DVT = 32: 64-byte rows, 64-byte swizzle.
+    static constexpr uint32_t SB_ROW = DVT * 2;
+    static constexpr uint32_t SB_SWZ = DVT == 64 ? t5::kSwz128 : t5::kSwz64;
+    KDA_DEVINL static int sb_off(int k, int n) {
+        const int chunk = (n >> 3) ^ (DVT == 64 ? (k & 7) : ((k >> 1) & 3));
+        return k * SB_ROW + (chunk << 4) + ((n & 7) << 1);
+    }
+    static_assert(NSTG >= 2 && BYTES <= SMEM_MAX + 1024, "shared memory budget");
 };
 
 template <int DVT>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(128, 1)
 kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT,
                     __nv_bfloat16 *__restrict__ o, int T, int H, int cps,
                     const int *__restrict__ hdr, const int *__restrict__ seq_off,
                     const int *__restrict__ cu, int *err_word, int debug_drop_first_copy) {
-    constexpr int NT = DVT / 8;    // n-tiles of the column tile
-    constexpr int LDV = DVT + 8;
-    using SM = StateSmem<DVT>;
-    static_assert(SM::STAGE_BYTES % 128 == 0, "stage alignment");
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    SM &sm = *reinterpret_cast<SM *>(smem_raw);
+    using L = T5Layout<DVT>;
+    constexpr int NSTG = L::NSTG;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
+    uint64_t *done_s = full + NSTG, *done_o = full + NSTG + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_TMEM);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gid = lane >> 2, tig = lane & 3;
     // 1-D grid, column tile fastest so the tiles of one chain run side by side
     // and share the chunk records through L2.
     const int tile = blockIdx.x % (D / DVT), col0 = tile * DVT;
@@ -580,154 +665,178 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
     const int nchunks = c_end - c_begin;
 
     if (tid == 0) {
-        for (int s = 0; s < NSTAGE; ++s) mbar_init(&sm.full[s], 1);
+        for (int s = 0; s < NSTG + 2; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
+    if (warp == 0) {
+        t5::alloc(tmem_slot, L::TMEM_COLS);
+        t5::relinquish();
+    }
+    t5::fence_before_sync();
     __syncthreads();
-    auto issue = [&](int j) {   // thread 0 only: bring chunk j into stage j % NSTAGE
-        uint64_t *bar = &sm.full[j % NSTAGE];
+    t5::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;   // this warp's TMEM lane quarter
+
+    auto issue = [&](int j) {   // one thread: bring chunk j into stage j % NSTG
+        uint64_t *bar = &full[j % NSTG];
         const uint8_t *rec = recs + ((size_t)(c_begin + j) * H + h) * REC_BYTES;
-        uint8_t *dst = sm.stage[j % NSTAGE];
-        mbar_arrive_expect_tx(bar, SM::STAGE_BYTES);
+        uint8_t *dst = sm + (j % NSTG) * L::STAGE_BYTES;
+        mbar_arrive_expect_tx(bar, L::STAGE_RAW);
         if (debug_drop_first_copy && j == 0) return;   // test hook: the wait must run out
         bulk_g2s(dst, rec, REC_SHARED, bar);
-        bulk_g2s(dst + REC_SHARED, rec + REC_R + tile * SM::R_BYTES, SM::R_BYTES, bar);
-        bulk_g2s(dst + REC_SHARED + SM::R_BYTES, rec + REC_O0 + tile * SM::O0_BYTES,
-                 SM::O0_BYTES, bar);
+        bulk_g2s(dst + REC_SHARED, rec + REC_R + core_off(D, 0, col0), L::R_BYTES, bar);
+        bulk_g2s(dst + REC_SHARED + L::R_BYTES, rec + REC_O0 + core_off(C, 0, col0), L::O0_BYTES,
+                 bar);
     };
     if (tid == 0)
-        for (int j = 0; j < NSTAGE && j < nchunks; ++j) issue(j);
+        for (int j = 0; j < NSTG && j < nchunks; ++j) issue(j);
 
-    // state rows 16w..16w+15 -> registers
-    float S[NT][4];
-    const size_t sbase = (size_t)chain * D * D;
+    // key row tid of the state tile -> registers
+    float S[DVT];
+    const size_t sbase = (size_t)chain * D * D + (size_t)tid * D + col0;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int i = 0; i < DVT; i += 4) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (h0) x = *reinterpret_cast<const float4 *>(h0 + sbase + i);
+        S[i] = x.x;
+        S[i + 1] = x.y;
+        S[i + 2] = x.z;
+        S[i + 3] = x.w;
+    }
+    auto write_sb = [&](int buf) {   // bf16 copy of row tid, 16 bytes at a time
+        uint8_t *sb = sm + L::OFF_SB + buf * L::SB_BYTES;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int r = warp * 16 + gid + 8 * hh;
-            const int col = col0 + nt * 8 + 2 * tig;
-            float2 x = make_float2(0.f, 0.f);
-            if (h0) x = *reinterpret_cast<const float2 *>(h0 + sbase + (size_t)r * D + col);
-            S[nt][2 * hh] = x.x;
-            S[nt][2 * hh + 1] = x.y;
+        for (int c8 = 0; c8 < DVT; c8 += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(S[c8], S[c8 + 1]);
+            pk.y = pack_bf16x2(S[c8 + 2], S[c8 + 3]);
+            pk.z = pack_bf16x2(S[c8 + 4], S[c8 + 5]);
+            pk.w = pack_bf16x2(S[c8 + 6], S[c8 + 7]);
+            *reinterpret_cast<uint4 *>(sb + L::sb_off(tid, c8)) = pk;
         }
-    auto store_sb = [&](int buf) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = warp * 16 + gid + 8 * hh;
-                *reinterpret_cast<uint32_t *>(sm.sb[buf] + r * LDV + nt * 8 + 2 * tig) =
-                    pack_bf16x2(S[nt][2 * hh], S[nt][2 * hh + 1]);
-            }
+        fence_proxy_async_smem();   // generic writes -> tensor-core reads
     };
-    store_sb(0);
+    write_sb(0);
+    t5::fence_before_sync();
     __syncthreads();
+    t5::fence_after_sync();
 
-    const int rq = (warp & 3) * 16;       // output rows of this warp
-    const int oq = (warp >> 2) * (NT / 2);  // first output n-tile of this warp
-    for (int j = 0; j < nchunks; ++j) {
-        const int s = j % NSTAGE;
-        if (!mbar_wait_bounded(&sm.full[s], (j / NSTAGE) & 1)) {
-            // Give up on this chain: report, let the copies already issued for later
-            // chunks land (bounded) so none writes into freed shared memory, return.
-            if (tid == 0) {
-                atomicOr(err_word, ERR_TIMEOUT_BIT);
-                for (int jj = j + 1; jj < j + NSTAGE && jj < nchunks; ++jj)
-                    mbar_wait_bounded(&sm.full[jj % NSTAGE], (jj / NSTAGE) & 1);
+    constexpr uint32_t idS = t5::idesc_bf16(128, DVT, 0, 1);
+    constexpr uint32_t idO = t5::idesc_bf16(64, DVT, 0, 1);
+    const uint32_t sm_addr = smem_u32(sm);
+    const int orow = warp * 16 + lane;   // output row of lanes 0..15
+    bool abort = false;
+    int j = 0;
+    for (; j < nchunks; ++j) {
+        const int s = j % NSTG;
+        const uint32_t par = (j / NSTG) & 1;
+        const uint8_t *st = sm + s * L::STAGE_BYTES;
+        const uint32_t st_addr = sm_addr + s * L::STAGE_BYTES;
+        if (warp == 0) {
+            // Warp 0 waits for the stage; one elected lane issues both products.
+            // Descriptors are a base plus compile-time offsets (in 16-byte units).
+            const bool ready = __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], par));
+            if (ready && t5::elect_one()) {
+                t5::fence_after_sync();
+                const uint32_t sb_addr = sm_addr + L::OFF_SB + (j & 1) * L::SB_BYTES;
+                const uint64_t bd0 = t5::smem_desc(sb_addr, 4096, 8 * L::SB_ROW, L::SB_SWZ);
+                // A operands in the core-matrix layout: 8-row groups 128 B apart (SBO),
+                // 8-column chunks rows*16 B apart (LBO), no swizzle.
+                const uint64_t am0 = t5::smem_desc(st_addr + REC_M, D * 16, 128, 0);
+                const uint64_t aq0 = t5::smem_desc(st_addr + REC_QP, C * 16, 128, 0);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    t5::mma_bf16(tmem, am0 + (uint64_t)((ks * 2 * D * 16) >> 4),
+                                 bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idS, ks > 0);
+                t5::commit(done_s);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    t5::mma_bf16(tmem + DVT, aq0 + (uint64_t)((ks * 2 * C * 16) >> 4),
+                                 bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idO, ks > 0);
+                t5::commit(done_o);
             }
-            return;
+            __syncwarp();
         }
-        const uint8_t *st = sm.stage[s];
-        const uint32_t sM = smem_u32(st + REC_M), sQ = smem_u32(st + REC_QP);
-        const float *gc = reinterpret_cast<const float *>(st + REC_GC);
-        const uint8_t *rt = st + REC_SHARED;                 // R tile   [DVT/16][D][16]
-        const uint8_t *ot = st + REC_SHARED + SM::R_BYTES;   // O0 tile  [DVT/16][C][16]
-        const uint32_t sB = smem_u32(sm.sb[j & 1]);
-        const int t0 = seq_t0 + j * C;
-        const int len = min(C, seq_len - j * C);
-
-        float acc[NT][4], oacc[NT / 2][4];
+        // stage bytes this thread needs, read while the products run
+        bool ok = mbar_wait_bounded(&full[s], par);
+        const float gam = reinterpret_cast<const float *>(st + REC_GC)[tid];
+        uint4 rv[DVT / 8];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int r = warp * 16 + gid + 8 * hh;
-            const float gr = gc[r];
+        for (int i = 0; i < DVT / 8; ++i)   // row tid of the R slice
+            rv[i] = *reinterpret_cast<const uint4 *>(st + REC_SHARED + core_off(D, tid, 8 * i));
+        ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(done_s, j & 1));
+        t5::fence_after_sync();
+        if (ok) {   // S <- exp(G_C) S + R + M' S
+            float v[DVT];
+            t5::ld_cols<DVT>(tmem + lane_base, v);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int cl = nt * 8 + 2 * tig;
-                const float2 rr = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
-                    rt + (cl >> 4) * (D * UT * 2) + r * (UT * 2) + (cl & 15) * 2));
-                acc[nt][2 * hh] = gr * S[nt][2 * hh] + rr.x;
-                acc[nt][2 * hh + 1] = gr * S[nt][2 * hh + 1] + rr.y;
+            for (int i = 0; i < DVT / 8; ++i) {
+                const uint32_t u[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 r2 = unpack_bf16x2(u[e]);
+                    const int c = i * 8 + 2 * e;
+                    S[c] = fmaf(gam, S[c], r2.x + v[c]);
+                    S[c + 1] = fmaf(gam, S[c + 1], r2.y + v[c + 1]);
+                }
             }
-            const int ro = rq + gid + 8 * hh;
-#pragma unroll
-            for (int i = 0; i < NT / 2; ++i) {
-                const int cl = (oq + i) * 8 + 2 * tig;
-                const float2 oo = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
-                    ot + (cl >> 4) * (C * UT * 2) + ro * (UT * 2) + (cl & 15) * 2));
-                oacc[i][2 * hh] = oo.x;
-                oacc[i][2 * hh + 1] = oo.y;
-            }
+            write_sb((j + 1) & 1);
         }
+        ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(done_o, j & 1));
+        t5::fence_after_sync();
+        if (ok) {   // O = Q' S + O0 for rows 16w..16w+15 (lanes 0..15)
+            float w[DVT];
+            t5::ld_cols<DVT>(tmem + lane_base + DVT, w);
+            const int t0 = seq_t0 + j * C;
+            const int len = min(C, seq_len - j * C);
+            if (lane < 16 && orow < len) {
+                const uint8_t *op0 = st + REC_SHARED + L::R_BYTES;
+                __nv_bfloat16 *op = o + ((size_t)(t0 + orow) * H + h) * D + col0;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            uint32_t am[4], aq[4];
-            ldsm_x4(am, sM + swz128(warp * 16 + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-            ldsm_x4(aq, sQ + swz128(rq + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+                for (int i = 0; i < DVT / 8; ++i) {
+                    const uint4 ov = *reinterpret_cast<const uint4 *>(op0 + core_off(C, orow, 8 * i));
+                    const uint32_t u[4] = {ov.x, ov.y, ov.z, ov.w};
+                    uint4 res;
+                    uint32_t *rr = reinterpret_cast<uint32_t *>(&res);
 #pragma unroll
-            for (int np = 0; np < NT / 2; ++np) {
-                uint32_t b[4];
-                ldsm_x4_t(b, sB + 2 * ((ks * 16 + frag_bk_row(lane)) * LDV + np * 16 +
-                                       frag_bk_col(lane)));
-                mma_bf16_16816(acc[2 * np], am, b[0], b[1]);
-                mma_bf16_16816(acc[2 * np + 1], am, b[2], b[3]);
-                if constexpr (NT == 2) {
-                    if (oq == 0) mma_bf16_16816(oacc[0], aq, b[0], b[1]);
-                    else mma_bf16_16816(oacc[0], aq, b[2], b[3]);
-                } else {
-                    if (2 * np == oq) {
-                        mma_bf16_16816(oacc[0], aq, b[0], b[1]);
-                        mma_bf16_16816(oacc[1], aq, b[2], b[3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 o2 = unpack_bf16x2(u[e]);
+                        rr[e] = pack_bf16x2(w[i * 8 + 2 * e] + o2.x, w[i * 8 + 2 * e + 1] + o2.y);
                     }
+                    *reinterpret_cast<uint4 *>(op + i * 8) = res;
                 }
             }
         }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) S[nt][e] = acc[nt][e];
-        store_sb((j + 1) & 1);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int r = rq + gid + 8 * hh;
-            if (r < len) {
-                __nv_bfloat16 *orow = o + ((size_t)(t0 + r) * H + h) * D + col0;
-#pragma unroll
-                for (int i = 0; i < NT / 2; ++i)
-                    *reinterpret_cast<uint32_t *>(orow + (oq + i) * 8 + 2 * tig) =
-                        pack_bf16x2(oacc[i][2 * hh], oacc[i][2 * hh + 1]);
-            }
-        }
-        __syncthreads();   // new state copy ready; stage s consumed
-        if (tid == 0 && j + NSTAGE < nchunks) {
+        t5::fence_before_sync();
+        abort = __syncthreads_or(!ok) != 0;
+        if (abort) break;
+        t5::fence_after_sync();
+        if (warp == 1 && j + NSTG < nchunks && t5::elect_one()) {
             fence_proxy_async_smem();   // order this chunk's generic reads before the refill
-            issue(j + NSTAGE);
+            issue(j + NSTG);
         }
     }
 
-    if (hT) {
+    if (abort) {
+        if (tid == 0) {
+            atomicOr(err_word, ERR_TIMEOUT_BIT);
+            // let what this CTA issued finish (bounded) before its shared memory goes
+            for (int jj = j + 1; jj < j + NSTG && jj < nchunks; ++jj)
+                mbar_wait_bounded(&full[jj % NSTG], (jj / NSTG) & 1);
+            mbar_wait_bounded(done_s, j & 1);
+            mbar_wait_bounded(done_o, j & 1);
+        }
+    } else if (hT) {
+        float *dst = hT + sbase;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int r = warp * 16 + gid + 8 * hh;
-                const int col = col0 + nt * 8 + 2 * tig;
-                *reinterpret_cast<float2 *>(hT + sbase + (size_t)r * D + col) =
-                    make_float2(S[nt][2 * hh], S[nt][2 * hh + 1]);
-            }
+        for (int i = 0; i < DVT; i += 4)
+            *reinterpret_cast<float4 *>(dst + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
     }
+    t5::fence_before_sync();
+    __syncthreads();
+    t5::fence_after_sync();
+    if (warp == 0) t5::dealloc(tmem, L::TMEM_COLS);
 }
 
 }  // namespace tc

@@ -87,7 +87,7 @@ def test_fwd_validation_before_launch(lib):
     assert _fwd(lib, q=None) == INVALID
     assert _fwd(lib, o=None) == INVALID
     assert _fwd(lib, q=0x10004) == MISALIGNED
-    assert _fwd(lib, hT=0x20004) == MISALIGNED
+    assert _fwd(lib, hT=0x20008) == MISALIGNED           # states are read as float4
     assert _fwd(lib, g=0x10004) == MISALIGNED            # g is read as float pairs
     assert _fwd(lib, o=0x20002) == MISALIGNED            # bf16 o needs 4 bytes
     assert _fwd(lib, o=0x10000) == INVALID               # output aliases an input
