@@ -85,14 +85,6 @@ int debug_drop_first_copy() {
     return v;
 }
 
-int state_tile_override() {
-    static const int v = [] {
-        const char *e = getenv("KDA_STATE_TILE");
-        return e ? atoi(e) : 0;
-    }();
-    return v;
-}
-
 kda_status launch_status() {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -139,16 +131,11 @@ kda_status launch_state(const uint8_t *recs, const float *h0, float *hT, void *o
     int *err = device_error_word();
     if (!err) return KDA_ERR_CUDA;
     const unsigned grid = (unsigned)nunits * (D / DVT);
-    kern<<<grid, 128, smem, s>>>(recs, h0, hT, static_cast<__nv_bfloat16 *>(o), T, H, cps, hdr,
+    kern<<<grid, 320, smem, s>>>(recs, h0, hT, static_cast<__nv_bfloat16 *>(o), T, H, cps, hdr,
                                  seq_off, cu, err, debug_drop_first_copy());
     return launch_status();
 }
 
-int sm_count() {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
-}
 
 }  // namespace
 
@@ -256,12 +243,7 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
     int *seq_off = reinterpret_cast<int *>(ws + L.seq_off);
     const int cps = cu ? 0 : (T + C - 1) / C;
     const int nunits = N * H;
-    // Narrow column tiles when there are too few chains to fill the GPU;
-    // KDA_STATE_TILE=32|64 overrides the choice (tuning knob).
-    const int forced = state_tile_override();
-    if (forced == 32 || (forced != 64 && (long long)nunits * (D / 64) < (long long)sm_count()))
-        return launch_state<32>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
-    return launch_state<64>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
+    return launch_state<32>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
 }
 
 kda_status kda_fwd_intra(const void *q, const void *k, const void *v, const float *g,

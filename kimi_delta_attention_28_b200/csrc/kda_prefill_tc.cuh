@@ -19,9 +19,11 @@
 // of the 16x16 diagonal blocks, tensor-core products elsewhere); and from them
 // the chunk's affine map on the state (below), one record per (chunk, head).
 // Kernel 2 (kda_tc_state_kernel) walks the chunks of each (sequence, head) in
-// order with the fp32 state on chip, split over d_v column tiles (state columns
-// evolve independently): per chunk one pair of tcgen05 products (accumulated in
-// tensor memory) and one barrier; records arrive by bulk copies into a ring.
+// order with the fp32 state on chip, split over 32-column slices of the state
+// (state columns evolve independently).  Its warps are specialised (state
+// update, tcgen05 issue, output, bulk-copy producer) and hand off through
+// mbarriers, so the loop-carried path per chunk is one tcgen05 product plus the
+// register update of the state; the outputs and copies run beside it.
 #pragma once
 
 #include "kda_common.cuh"
@@ -588,37 +590,45 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 2: inter-chunk state pass on tcgen05.  grid = N * H * (D / DVT), 128 threads.
-//
-// Thread t owns key row t of the fp32 state tile S[:, col0:col0+DVT] in registers.
-// Per chunk, one elected lane of warp 0 issues two tcgen05 products whose B
-// operand is a bf16 copy of the state in shared memory (double-buffered):
-//   D_S = M' S   (M = 128 key rows, N = DVT, K = 128) -> tensor memory columns [0, DVT)
-//   D_O = Q' S   (M = 64 chunk rows)                  -> columns [DVT, 2 DVT)
-// with separate completion barriers, so the state update S <- exp(G_C) S + R + D_S
-// (the loop-carried path) waits only for the first product while the second runs
-// behind it; rows 16w..16w+15 of warp w then form O = D_O + O0.  Records arrive by
-// bulk copies into a ring of stages, refilled by warp 1 so warp 0 can go straight
-// on to the next products.  Every wait is bounded; a wait that runs out makes the
-// whole CTA stop (block-wide vote), drain what it issued, free its tensor memory,
-// set the timeout bit and return.
+// Kernel 2: inter-chunk state pass on tcgen05, warp-specialised.
+// grid = N * H * (D / DVT) CTAs of 320 threads (10 warps):
+//   warps 0-3  state:    thread t owns key row t of the fp32 state tile
+//                        S[:, col0:col0+DVT] in registers; per chunk it applies
+//                        S <- exp(G_C) S + R + (M' S) and writes the bf16 copy of
+//                        the new state that the next products read;
+//   warp 4     MMA:      one elected lane issues, per chunk,
+//                          D_S        = M'(j) S   (M = 128 key rows, N = DVT, K = 128)
+//                          D_O[j & 1] = Q'(j) S   (M = 64 chunk rows)
+//                        on tcgen05, accumulating in tensor memory;
+//   warps 5-8  output:   O = D_O + O0 for the chunk's rows (warp w reads tensor-memory
+//                        lane quarter w % 4), stored as bf16;
+//   warp 9     producer: bulk copies of the chunk records into two rings, the state
+//                        ring (M', exp(G_C), R slice) and the output ring (Q', O0 slice),
+//                        refilling a slot once its consumers release it.
+// The roles hand off through mbarriers only, so the loop-carried path per chunk is
+// M' S on the tensor core -> state update -> bf16 copy -> next M' S.  Every wait is
+// bounded; a wait that runs out sets the shared abort flag and the timeout bit, all
+// roles stop, the CTA drains what it issued, frees its tensor memory and returns.
 // ---------------------------------------------------------------------------
 template <int DVT>
 struct T5Layout {
     static_assert(DVT == 32 || DVT == 64, "column tile");
-    // the column tile's slices of R and O0: DVT/8 contiguous 8-column chunks each
     static constexpr int R_BYTES = D * DVT * 2, O0_BYTES = C * DVT * 2;
-    static constexpr int STAGE_RAW = REC_SHARED + R_BYTES + O0_BYTES;
-    static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
-    static constexpr int SB_BYTES = D * DVT * 2;        // one bf16 state copy (B operand)
-    static constexpr int SMEM_MAX = 232448;             // opt-in limit per CTA
-    static constexpr int NSTG_FIT = (SMEM_MAX - 2 * SB_BYTES - 2048) / STAGE_BYTES;
-    static constexpr int NSTG = NSTG_FIT > 4 ? 4 : NSTG_FIT;
-    static constexpr int OFF_SB = NSTG * STAGE_BYTES;
-    static constexpr int OFF_BAR = OFF_SB + 2 * SB_BYTES;   // full[NSTG], done_s, done_o
-    static constexpr int OFF_TMEM = OFF_BAR + 8 * (NSTG + 2);
-    static constexpr int BYTES = OFF_TMEM + 16 + 1024;      // + slack for 1024-byte alignment
-    static constexpr uint32_t TMEM_COLS = 2 * DVT;
+    static constexpr int A_RAW = D * D * 2 + D * 4 + R_BYTES;            // M' | exp(G_C) | R
+    static constexpr int A_BYTES = (A_RAW + 1023) / 1024 * 1024;
+    static constexpr int A_GC = D * D * 2, A_R = A_GC + D * 4;
+    static constexpr int B_BYTES = C * D * 2 + O0_BYTES;                 // Q' | O0
+    static constexpr int B_O0 = C * D * 2;
+    static constexpr int NA = DVT == 32 ? 3 : 2, NB = 3;
+    static constexpr int SB_BYTES = D * DVT * 2;                         // one bf16 state copy
+    static constexpr int OFF_B = NA * A_BYTES;
+    static constexpr int OFF_SB = OFF_B + NB * B_BYTES;
+    // barriers: full_a[NA] full_b[NB] a_free[NA] b_free[NB] done_s done_o[2] sb_full do_free[2]
+    static constexpr int OFF_BAR = OFF_SB + 2 * SB_BYTES;
+    static constexpr int NBAR = 2 * (NA + NB) + 6;
+    static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;   // tmem slot, abort flag, counters
+    static constexpr int BYTES = OFF_MISC + 32 + 1024;    // + slack for 1024-byte alignment
+    static constexpr uint32_t TMEM_COLS = DVT == 32 ? 128 : 256;   // D_S | D_O[0] | D_O[1]
     // B operand (the state copy), MN-major: row k (key) holds DVT bf16 values.
     // DVT = 64: 128-byte rows, 128-byte swizzle; DVT = 32: 64-byte rows, 64-byte swizzle.
     static constexpr uint32_t SB_ROW = DVT * 2;
@@ -627,22 +637,30 @@ struct T5Layout {
         const int chunk = (n >> 3) ^ (DVT == 64 ? (k & 7) : ((k >> 1) & 3));
         return k * SB_ROW + (chunk << 4) + ((n & 7) << 1);
     }
-    static_assert(NSTG >= 2 && BYTES <= SMEM_MAX + 1024, "shared memory budget");
+    static_assert(BYTES <= 232448, "shared memory budget");
 };
 
 template <int DVT>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(320, 1)
 kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT,
                     __nv_bfloat16 *__restrict__ o, int T, int H, int cps,
                     const int *__restrict__ hdr, const int *__restrict__ seq_off,
                     const int *__restrict__ cu, int *err_word, int debug_drop_first_copy) {
     using L = T5Layout<DVT>;
-    constexpr int NSTG = L::NSTG;
+    constexpr int NA = L::NA, NB = L::NB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
-    uint64_t *done_s = full + NSTG, *done_o = full + NSTG + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_TMEM);
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
+    uint64_t *full_b = full_a + NA;
+    uint64_t *a_free = full_b + NB;
+    uint64_t *b_free = a_free + NA;
+    uint64_t *done_s = b_free + NB;
+    uint64_t *done_o = done_s + 1;     // [2] by chunk parity
+    uint64_t *sb_full = done_o + 2;
+    uint64_t *do_free = sb_full + 1;   // [2] by chunk parity
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 4);
+    int *cnt = reinterpret_cast<int *>(sm + L::OFF_MISC + 8);   // [0] ring A issued, [1] ring B issued, [2] MMA issued
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // 1-D grid, column tile fastest so the tiles of one chain run side by side
     // and share the chunk records through L2.
@@ -665,7 +683,16 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
     const int nchunks = c_end - c_begin;
 
     if (tid == 0) {
-        for (int s = 0; s < NSTG + 2; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < NA; ++s) { mbar_init(&full_a[s], 1); mbar_init(&a_free[s], 128); }
+        for (int s = 0; s < NB; ++s) { mbar_init(&full_b[s], 1); mbar_init(&b_free[s], 128); }
+        mbar_init(done_s, 1);
+        mbar_init(&done_o[0], 1);
+        mbar_init(&done_o[1], 1);
+        mbar_init(sb_full, 128);
+        mbar_init(&do_free[0], 128);
+        mbar_init(&do_free[1], 128);
+        *abort_flag = 0;
+        cnt[0] = cnt[1] = cnt[2] = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -676,100 +703,62 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
     __syncthreads();
     t5::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;   // this warp's TMEM lane quarter
-
-    auto issue = [&](int j) {   // one thread: bring chunk j into stage j % NSTG
-        uint64_t *bar = &full[j % NSTG];
-        const uint8_t *rec = recs + ((size_t)(c_begin + j) * H + h) * REC_BYTES;
-        uint8_t *dst = sm + (j % NSTG) * L::STAGE_BYTES;
-        mbar_arrive_expect_tx(bar, L::STAGE_RAW);
-        if (debug_drop_first_copy && j == 0) return;   // test hook: the wait must run out
-        bulk_g2s(dst, rec, REC_SHARED, bar);
-        bulk_g2s(dst + REC_SHARED, rec + REC_R + core_off(D, 0, col0), L::R_BYTES, bar);
-        bulk_g2s(dst + REC_SHARED + L::R_BYTES, rec + REC_O0 + core_off(C, 0, col0), L::O0_BYTES,
-                 bar);
-    };
-    if (tid == 0)
-        for (int j = 0; j < NSTG && j < nchunks; ++j) issue(j);
-
-    // key row tid of the state tile -> registers
-    float S[DVT];
-    const size_t sbase = (size_t)chain * D * D + (size_t)tid * D + col0;
-#pragma unroll
-    for (int i = 0; i < DVT; i += 4) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (h0) x = *reinterpret_cast<const float4 *>(h0 + sbase + i);
-        S[i] = x.x;
-        S[i + 1] = x.y;
-        S[i + 2] = x.z;
-        S[i + 3] = x.w;
-    }
-    auto write_sb = [&](int buf) {   // bf16 copy of row tid, 16 bytes at a time
-        uint8_t *sb = sm + L::OFF_SB + buf * L::SB_BYTES;
-#pragma unroll
-        for (int c8 = 0; c8 < DVT; c8 += 8) {
-            uint4 pk;
-            pk.x = pack_bf16x2(S[c8], S[c8 + 1]);
-            pk.y = pack_bf16x2(S[c8 + 2], S[c8 + 3]);
-            pk.z = pack_bf16x2(S[c8 + 4], S[c8 + 5]);
-            pk.w = pack_bf16x2(S[c8 + 6], S[c8 + 7]);
-            *reinterpret_cast<uint4 *>(sb + L::sb_off(tid, c8)) = pk;
-        }
-        fence_proxy_async_smem();   // generic writes -> tensor-core reads
-    };
-    write_sb(0);
-    t5::fence_before_sync();
-    __syncthreads();
-    t5::fence_after_sync();
-
-    constexpr uint32_t idS = t5::idesc_bf16(128, DVT, 0, 1);
-    constexpr uint32_t idO = t5::idesc_bf16(64, DVT, 0, 1);
     const uint32_t sm_addr = smem_u32(sm);
-    const int orow = warp * 16 + lane;   // output row of lanes 0..15
-    bool abort = false;
-    int j = 0;
-    for (; j < nchunks; ++j) {
-        const int s = j % NSTG;
-        const uint32_t par = (j / NSTG) & 1;
-        const uint8_t *st = sm + s * L::STAGE_BYTES;
-        const uint32_t st_addr = sm_addr + s * L::STAGE_BYTES;
-        if (warp == 0) {
-            // Warp 0 waits for the stage; one elected lane issues both products.
-            // Descriptors are a base plus compile-time offsets (in 16-byte units).
-            const bool ready = __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], par));
-            if (ready && t5::elect_one()) {
-                t5::fence_after_sync();
-                const uint32_t sb_addr = sm_addr + L::OFF_SB + (j & 1) * L::SB_BYTES;
-                const uint64_t bd0 = t5::smem_desc(sb_addr, 4096, 8 * L::SB_ROW, L::SB_SWZ);
-                // A operands in the core-matrix layout: 8-row groups 128 B apart (SBO),
-                // 8-column chunks rows*16 B apart (LBO), no swizzle.
-                const uint64_t am0 = t5::smem_desc(st_addr + REC_M, D * 16, 128, 0);
-                const uint64_t aq0 = t5::smem_desc(st_addr + REC_QP, C * 16, 128, 0);
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    t5::mma_bf16(tmem, am0 + (uint64_t)((ks * 2 * D * 16) >> 4),
-                                 bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idS, ks > 0);
-                t5::commit(done_s);
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    t5::mma_bf16(tmem + DVT, aq0 + (uint64_t)((ks * 2 * C * 16) >> 4),
-                                 bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idO, ks > 0);
-                t5::commit(done_o);
-            }
-            __syncwarp();
+    auto fail = [&]() {
+        if (*abort_flag == 0) {
+            *abort_flag = 1;
+            atomicOr(err_word, ERR_TIMEOUT_BIT);
         }
-        // stage bytes this thread needs, read while the products run
-        bool ok = mbar_wait_bounded(&full[s], par);
-        const float gam = reinterpret_cast<const float *>(st + REC_GC)[tid];
-        uint4 rv[DVT / 8];
+    };
+    auto rec_of = [&](int j) { return recs + ((size_t)(c_begin + j) * H + h) * REC_BYTES; };
+
+    if (warp < 4) {
+        // ---------------- state warps ----------------
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        float S[DVT];
+        const size_t sbase = (size_t)chain * D * D + (size_t)tid * D + col0;
 #pragma unroll
-        for (int i = 0; i < DVT / 8; ++i)   // row tid of the R slice
-            rv[i] = *reinterpret_cast<const uint4 *>(st + REC_SHARED + core_off(D, tid, 8 * i));
-        ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(done_s, j & 1));
-        t5::fence_after_sync();
-        if (ok) {   // S <- exp(G_C) S + R + M' S
+        for (int i = 0; i < DVT; i += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (h0) x = *reinterpret_cast<const float4 *>(h0 + sbase + i);
+            S[i] = x.x;
+            S[i + 1] = x.y;
+            S[i + 2] = x.z;
+            S[i + 3] = x.w;
+        }
+        auto write_sb = [&](int buf) {   // bf16 copy of row tid, then signal it
+            uint8_t *sb = sm + L::OFF_SB + buf * L::SB_BYTES;
+#pragma unroll
+            for (int c8 = 0; c8 < DVT; c8 += 8) {
+                uint4 pk;
+                pk.x = pack_bf16x2(S[c8], S[c8 + 1]);
+                pk.y = pack_bf16x2(S[c8 + 2], S[c8 + 3]);
+                pk.z = pack_bf16x2(S[c8 + 4], S[c8 + 5]);
+                pk.w = pack_bf16x2(S[c8 + 6], S[c8 + 7]);
+                *reinterpret_cast<uint4 *>(sb + L::sb_off(tid, c8)) = pk;
+            }
+            fence_proxy_async_smem();   // generic writes -> tensor-core reads
+            mbar_arrive(sb_full);
+        };
+        write_sb(0);
+        int j = 0;
+        for (; j < nchunks && !*abort_flag; ++j) {
+            const int sa = j % NA;
+            const uint8_t *st = sm + sa * L::A_BYTES;
+            bool ok = mbar_wait_bounded(&full_a[sa], (j / NA) & 1);
+            const float gam = reinterpret_cast<const float *>(st + L::A_GC)[tid];
+            uint4 rv[DVT / 8];
+#pragma unroll
+            for (int i = 0; i < DVT / 8; ++i)   // row tid of the R slice
+                rv[i] = *reinterpret_cast<const uint4 *>(st + L::A_R + core_off(D, tid, 8 * i));
+            // the tensor-memory load below is warp-collective: decide as a warp
+            ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(done_s, j & 1));
+            if (!ok) { fail(); break; }
+            t5::fence_after_sync();
             float v[DVT];
             t5::ld_cols<DVT>(tmem + lane_base, v);
+            t5::fence_before_sync();
+            mbar_arrive(&a_free[sa]);   // this thread is done with the slot and with D_S
 #pragma unroll
             for (int i = 0; i < DVT / 8; ++i) {
                 const uint32_t u[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
@@ -781,17 +770,70 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
                     S[c + 1] = fmaf(gam, S[c + 1], r2.y + v[c + 1]);
                 }
             }
-            write_sb((j + 1) & 1);
+            if (j + 1 < nchunks) write_sb((j + 1) & 1);
         }
-        ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(done_o, j & 1));
-        t5::fence_after_sync();
-        if (ok) {   // O = Q' S + O0 for rows 16w..16w+15 (lanes 0..15)
+        if (!*abort_flag && hT && j == nchunks) {
+            float *dst = hT + sbase;
+#pragma unroll
+            for (int i = 0; i < DVT; i += 4)
+                *reinterpret_cast<float4 *>(dst + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
+        }
+    } else if (warp == 4) {
+        // ---------------- MMA warp ----------------
+        constexpr uint32_t idS = t5::idesc_bf16(128, DVT, 0, 1);
+        constexpr uint32_t idO = t5::idesc_bf16(64, DVT, 0, 1);
+        for (int j = 0; j < nchunks && !*abort_flag; ++j) {
+            const int sa = j % NA, sbb = j % NB;
+            bool ok = mbar_wait_bounded(&full_a[sa], (j / NA) & 1) &&
+                      mbar_wait_bounded(&full_b[sbb], (j / NB) & 1) &&
+                      mbar_wait_bounded(sb_full, j & 1) &&
+                      (j < 2 || mbar_wait_bounded(&do_free[j & 1], ((j - 2) >> 1) & 1));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) { fail(); break; }
+            if (t5::elect_one()) {
+                t5::fence_after_sync();
+                const uint32_t sb_addr = sm_addr + L::OFF_SB + (j & 1) * L::SB_BYTES;
+                const uint64_t bd0 = t5::smem_desc(sb_addr, 4096, 8 * L::SB_ROW, L::SB_SWZ);
+                // A operands in the core-matrix layout: 8-row groups 128 B apart (SBO),
+                // 8-column chunks rows*16 B apart (LBO), no swizzle.
+                const uint64_t am0 = t5::smem_desc(sm_addr + sa * L::A_BYTES, D * 16, 128, 0);
+                const uint64_t aq0 = t5::smem_desc(sm_addr + L::OFF_B + sbb * L::B_BYTES,
+                                                   C * 16, 128, 0);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    t5::mma_bf16(tmem, am0 + (uint64_t)((ks * 2 * D * 16) >> 4),
+                                 bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idS, ks > 0);
+                t5::commit(done_s);
+                const uint32_t dO = tmem + DVT + (j & 1) * DVT;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    t5::mma_bf16(dO, aq0 + (uint64_t)((ks * 2 * C * 16) >> 4),
+                                 bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idO, ks > 0);
+                t5::commit(&done_o[j & 1]);
+                cnt[2] = j + 1;
+            }
+            __syncwarp();
+        }
+    } else if (warp < 9) {
+        // ---------------- output warps ----------------
+        const int q = warp & 3;                          // tensor-memory lane quarter
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const int orow = q * 16 + lane;                  // output row of lanes 0..15
+        for (int j = 0; j < nchunks && !*abort_flag; ++j) {
+            const int sbb = j % NB;
+            bool ok = mbar_wait_bounded(&done_o[j & 1], (j >> 1) & 1) &&
+                      mbar_wait_bounded(&full_b[sbb], (j / NB) & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) { fail(); break; }
+            t5::fence_after_sync();
             float w[DVT];
-            t5::ld_cols<DVT>(tmem + lane_base + DVT, w);
+            t5::ld_cols<DVT>(tmem + lane_base + DVT + (j & 1) * DVT, w);
+            t5::fence_before_sync();
+            mbar_arrive(&do_free[j & 1]);
             const int t0 = seq_t0 + j * C;
             const int len = min(C, seq_len - j * C);
             if (lane < 16 && orow < len) {
-                const uint8_t *op0 = st + REC_SHARED + L::R_BYTES;
+                const uint8_t *op0 = sm + L::OFF_B + sbb * L::B_BYTES + L::B_O0;
                 __nv_bfloat16 *op = o + ((size_t)(t0 + orow) * H + h) * D + col0;
 #pragma unroll
                 for (int i = 0; i < DVT / 8; ++i) {
@@ -807,33 +849,53 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
                     *reinterpret_cast<uint4 *>(op + i * 8) = res;
                 }
             }
+            mbar_arrive(&b_free[sbb]);
         }
-        t5::fence_before_sync();
-        abort = __syncthreads_or(!ok) != 0;
-        if (abort) break;
-        t5::fence_after_sync();
-        if (warp == 1 && j + NSTG < nchunks && t5::elect_one()) {
-            fence_proxy_async_smem();   // order this chunk's generic reads before the refill
-            issue(j + NSTG);
+    } else {
+        // ---------------- producer warp: lane 0 feeds ring A, lane 1 ring B ----------------
+        if (lane == 0) {
+            for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+                const int s = c % NA;
+                if (c >= NA && !mbar_wait_bounded(&a_free[s], ((c - NA) / NA) & 1)) { fail(); break; }
+                fence_proxy_async_smem();
+                uint64_t *bar = &full_a[s];
+                uint8_t *dst = sm + s * L::A_BYTES;
+                const uint8_t *rec = rec_of(c);
+                mbar_arrive_expect_tx(bar, L::A_RAW);
+                cnt[0] = c + 1;
+                if (debug_drop_first_copy && c == 0) continue;   // test hook: the wait must run out
+                bulk_g2s(dst, rec + REC_M, D * D * 2, bar);
+                bulk_g2s(dst + L::A_GC, rec + REC_GC, D * 4, bar);
+                bulk_g2s(dst + L::A_R, rec + REC_R + core_off(D, 0, col0), L::R_BYTES, bar);
+            }
+        } else if (lane == 1) {
+            for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+                const int s = c % NB;
+                if (c >= NB && !mbar_wait_bounded(&b_free[s], ((c - NB) / NB) & 1)) { fail(); break; }
+                fence_proxy_async_smem();
+                uint64_t *bar = &full_b[s];
+                uint8_t *dst = sm + L::OFF_B + s * L::B_BYTES;
+                const uint8_t *rec = rec_of(c);
+                mbar_arrive_expect_tx(bar, L::B_BYTES);
+                cnt[1] = c + 1;
+                bulk_g2s(dst, rec + REC_QP, C * D * 2, bar);
+                bulk_g2s(dst + L::B_O0, rec + REC_O0 + core_off(C, 0, col0), L::O0_BYTES, bar);
+            }
         }
+        __syncwarp();
     }
 
-    if (abort) {
-        if (tid == 0) {
-            atomicOr(err_word, ERR_TIMEOUT_BIT);
-            // let what this CTA issued finish (bounded) before its shared memory goes
-            for (int jj = j + 1; jj < j + NSTG && jj < nchunks; ++jj)
-                mbar_wait_bounded(&full[jj % NSTG], (jj / NSTG) & 1);
-            mbar_wait_bounded(done_s, j & 1);
-            mbar_wait_bounded(done_o, j & 1);
-        }
-    } else if (hT) {
-        float *dst = hT + sbase;
-#pragma unroll
-        for (int i = 0; i < DVT; i += 4)
-            *reinterpret_cast<float4 *>(dst + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
-    }
     t5::fence_before_sync();
+    __syncthreads();
+    if (*abort_flag && tid == 0) {
+        // let what this CTA issued finish (bounded) before its shared memory goes
+        for (int c = max(0, cnt[0] - NA); c < cnt[0]; ++c)
+            mbar_wait_bounded(&full_a[c % NA], (c / NA) & 1);
+        for (int c = max(0, cnt[1] - NB); c < cnt[1]; ++c)
+            mbar_wait_bounded(&full_b[c % NB], (c / NB) & 1);
+        for (int c = max(0, cnt[2] - 2); c < cnt[2]; ++c)
+            mbar_wait_bounded(&done_o[c & 1], (c >> 1) & 1);
+    }
     __syncthreads();
     t5::fence_after_sync();
     if (warp == 0) t5::dealloc(tmem, L::TMEM_COLS);
