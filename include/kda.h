@@ -68,6 +68,10 @@ const char *kda_status_string(kda_status s);
  * tensor-core path stores, per 64-token chunk and head, the chunk's affine map
  * on the state (98,816 bytes: the state transition and offset, the output
  * read-out and offset, and the chunk's total decay) that the state pass consumes.
+ * When few (sequence, head) chains would leave most SMs idle, kda_fwd splits
+ * each chain in time (see kda_fwd_segmented); the size returned here includes
+ * room for the largest split the library would choose on a GPU of up to 192
+ * SMs, so it does not depend on the current device.
  * Returns 0 for an invalid or unsupported combination.
  *   B, T      : fixed-length batch (B sequences of T tokens), or with
  *               num_seqs > 0 and packed input: B = 1, T = total tokens.
@@ -101,6 +105,9 @@ size_t kda_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
  * The cu_seqlens preconditions are checked on the device; a violation makes
  * the call write no outputs and is reported by kda_get_last_device_error.
  * T = 0 (or B = 0) is a valid empty call that only copies h0 to hT.
+ * On the tensor-core path the call picks the number of time segments of the
+ * state pass itself (kda_fwd_segmented with a policy based on the SM count:
+ * split only when N * H chains are too few to fill the GPU).
  */
 kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                    const float *beta, const float *h0, const int32_t *cu_seqlens,
@@ -133,6 +140,35 @@ kda_status kda_fwd_inter(const float *h0, const int32_t *cu_seqlens, int num_seq
                          size_t ws_bytes, void *stream);
 
 /*
+ * Prefill with an explicit time split of the state pass.  Source: the "Kimi K3"
+ * field notes, panel "传固定状态片段" (pass fixed-size state fragments): each
+ * worker summarises its stretch of the sequence as a cumulative transform plus
+ * a state grown from zero, and the stretches are then combined in prefix order;
+ * the same page's "FlashKDA / FLA" panel names the within-device form of this
+ * context parallelism, which is what this entry point does.  It works because
+ * every chunk's map on the state is affine, S -> P S + R.
+ *
+ * Each chain's chunks are cut into num_segments consecutive segments of
+ * ceil(chunks / num_segments) chunks (trailing segments may be short or empty).
+ * Pass 1 computes every segment's map [R | P] from zero / identity, a combine
+ * kernel walks the segments in order in fp32 (S_{s+1} = P_s S_s + R_s) to get
+ * each segment's starting state, and pass 2 reruns the segments from those
+ * states, writing o and (from the last segment) hT.  num_segments = 1 is
+ * exactly kda_fwd without a split.  num_segments > 1 needs the tensor-core path
+ * (bf16, d_k = d_v = 128), else KDA_ERR_UNSUPPORTED_SHAPE; at most 4,096.
+ * The workspace must hold kda_fwd_segmented_workspace_size(..., num_segments)
+ * bytes: the records plus N * H * num_segments * 192 KiB.
+ * Other arguments and results as for kda_fwd.
+ */
+size_t kda_fwd_segmented_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
+                                        int dtype, int num_segments);
+kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *h0, const int32_t *cu_seqlens,
+                             int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
+                             int num_segments, void *o, float *hT, void *workspace,
+                             size_t ws_bytes, void *stream);
+
+/*
  * One decode step: every (sequence, head) consumes one token and updates its
  * state in place (the recurrence above with T = 1).
  *
@@ -163,8 +199,10 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
  * Only the tensor-core path is offered (bf16, d_k = d_v = 128); other dtypes or
  * head sizes return KDA_ERR_UNSUPPORTED_SHAPE.
  *
- *   - Size limit: kda_fwd_workspace_size(B, T, H, 128, 128, num_seqs,
- *     KDA_DTYPE_BF16) must not exceed KDA_NOALLOC_SCRATCH_BYTES, otherwise the
+ *   - Size limit: this variant never splits the state pass in time, so its
+ *     scratch need is kda_fwd_segmented_workspace_size(B, T, H, 128, 128,
+ *     num_seqs, KDA_DTYPE_BF16, 1); that must not exceed
+ *     KDA_NOALLOC_SCRATCH_BYTES, otherwise the
  *     call returns KDA_ERR_EXCEEDS_STATIC_SCRATCH and launches nothing.  32 MiB
  *     holds 339 (64-token chunk, head) records, e.g. B = 1, H = 8, T = 2,688.
  *   - Set-up: the first call on a device looks up the array's device address

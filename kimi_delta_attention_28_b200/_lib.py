@@ -41,6 +41,9 @@ SIGNATURES = {
     "kda_get_last_device_error": ([_VP], _I),
     "kda_fwd_noalloc": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP,
                          _VP], _I),
+    "kda_fwd_segmented_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I], _SZ),
+    "kda_fwd_segmented": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I,
+                           _VP, _VP, _VP, _SZ, _VP], _I),
 }
 
 
@@ -148,6 +151,45 @@ def kda_fwd(q, k, v, g, beta, h0=None, cu_seqlens=None, *, output_final_state: b
     _check(lib.kda_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
                        _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, dt, _ptr(o), _ptr(hT),
                        _ptr(workspace), workspace.numel(), _stream(dev)), "kda_fwd")
+    return o, hT
+
+
+def segmented_workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
+                             dtype: torch.dtype, num_segments: int) -> int:
+    return int(load_library().kda_fwd_segmented_workspace_size(
+        B, T, H, dk, dv, num_seqs, _dtype_code(dtype), num_segments))
+
+
+def kda_fwd_segmented(q, k, v, g, beta, h0=None, cu_seqlens=None, *, num_segments: int,
+                      o=None, hT=None, workspace=None):
+    """kda_fwd with the state pass split into ``num_segments`` time segments per
+    (sequence, head) chain (segment maps, a sequential combine, then the output
+    pass from each segment's starting state).  Arguments as for kda_fwd; always
+    returns (o, hT)."""
+    lib = load_library()
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(h0, "h0", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = B if cu_seqlens is None else num_seqs
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=q.dtype, device=dev)
+    if hT is None:
+        hT = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    need = segmented_workspace_size(B, T, H, dk, dv, num_seqs, q.dtype, num_segments)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.kda_fwd_segmented(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                 _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv,
+                                 _dtype_code(q.dtype), num_segments, _ptr(o), _ptr(hT),
+                                 _ptr(workspace), workspace.numel(), _stream(dev)),
+           "kda_fwd_segmented")
     return o, hT
 
 

@@ -34,14 +34,53 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 //   seq_off  : num_seqs + 1 ints
 //   chunks   : max_chunks ChunkLoc
 //   records  : max_chunks * H records of tc::REC_BYTES (tensor-core path only)
+//   s_in     : (T-split only) units * D * D fp32 segment starting states
+//   seg_map  : (T-split only) units * D * 2D fp32 segment maps [R | P]
+// where units = chains (N * H) * nseg.
 struct WsLayout {
-    size_t hdr, seq_off, chunks, recs, total;
+    size_t hdr, seq_off, chunks, recs, s_in, seg_map, total;
     long long max_chunks;
+    int nseg;
 };
 
 inline bool is_tc_path(int dtype, int dk) { return dtype == KDA_DTYPE_BF16 && dk == 128; }
 
-WsLayout ws_layout(int B, int T, int H, int dk, int num_seqs, int dtype) {
+// T-split policy.  Splitting a chain into nseg segments costs about three times
+// its state-pass work (the map pass carries 2D columns, the output pass D) but
+// runs nseg times as many CTAs, so it pays only when the unsplit pass leaves most
+// SMs idle.  nseg is chosen so the map pass (chains * nseg * 2D/32 CTAs) fills at
+// most one wave, with at least kMinSegChunks chunks per segment.
+constexpr int kMaxSegments = 32;
+constexpr int kMinSegChunks = 16;
+constexpr int kSplitSmBound = 192;   // workspace sizing assumes at most this many SMs
+constexpr int kMaxSegmentsExplicit = 4096;   // cap of kda_fwd_segmented's num_segments
+
+int split_segments(long long chains, long long chunks_per_chain, int sms) {
+    if (chains <= 0 || sms <= 0) return 1;
+    long long n = (long long)sms / (chains * (2 * kda::tc::D / 32));
+    n = n < chunks_per_chain / kMinSegChunks ? n : chunks_per_chain / kMinSegChunks;
+    n = n < kMaxSegments ? n : kMaxSegments;
+    return n >= 2 ? (int)n : 1;
+}
+
+long long chunks_per_chain(int B, int T, int num_seqs, long long max_chunks) {
+    if (num_seqs > 0) return max_chunks / num_seqs;   // packed: the mean
+    (void)B;
+    return ((long long)T + kda::tc::C - 1) / kda::tc::C;
+}
+
+// SM count of the current device, capped at kSplitSmBound (0 if unknown).
+int device_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n < kSplitSmBound ? n : kSplitSmBound;
+}
+
+// nseg > 0: that many segments (tensor-core path); nseg == 0: the policy with
+// `sms` multiprocessors.
+WsLayout ws_layout(int B, int T, int H, int dk, int num_seqs, int dtype, int nseg = 0,
+                   int sms = kSplitSmBound) {
     WsLayout L{};
     const bool varlen = num_seqs > 0;
     const int chunk = is_tc_path(dtype, dk) ? kda::tc::C : kda::simt::C;
@@ -55,7 +94,19 @@ WsLayout ws_layout(int B, int T, int H, int dk, int num_seqs, int dtype) {
     L.recs = round_up(L.chunks + (varlen ? sizeof(kda::tc::ChunkLoc) * (size_t)L.max_chunks : 0),
                       256);
     L.total = L.recs;
-    if (is_tc_path(dtype, dk)) L.total += (size_t)L.max_chunks * H * kda::tc::REC_BYTES;
+    L.nseg = 1;
+    if (is_tc_path(dtype, dk)) {
+        L.total += (size_t)L.max_chunks * H * kda::tc::REC_BYTES;
+        const long long N = num_seqs > 0 ? num_seqs : B;
+        L.nseg = nseg > 0 ? nseg
+                          : split_segments(N * H, chunks_per_chain(B, T, num_seqs, L.max_chunks), sms);
+        if (L.nseg > 1) {
+            const size_t units = (size_t)N * H * L.nseg, D = kda::tc::D;
+            L.s_in = round_up(L.total, 256);
+            L.seg_map = round_up(L.s_in + units * D * D * sizeof(float), 256);
+            L.total = L.seg_map + units * D * 2 * D * sizeof(float);
+        }
+    }
     return L;
 }
 
@@ -118,21 +169,22 @@ kda_status dispatch_simt(int D, const void *q, const void *k, const void *v, con
     }
 }
 
+// One state-pass launch over `units` units (chains * nseg); a.err_word and the
+// test hook are filled in here.
 template <int DVT>
-kda_status launch_state(const uint8_t *recs, const float *h0, float *hT, void *o, int T, int H,
-                        int cps, int nunits, const int *hdr, const int *seq_off, const int *cu,
-                        cudaStream_t s) {
+kda_status launch_state(kda::tc::StateArgs a, long long units, cudaStream_t s) {
     using namespace kda::tc;
     const size_t smem = T5Layout<DVT>::BYTES;
     auto kern = kda_tc_state_kernel<DVT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return KDA_ERR_CUDA;
-    int *err = device_error_word();
-    if (!err) return KDA_ERR_CUDA;
-    const unsigned grid = (unsigned)nunits * (D / DVT);
-    kern<<<grid, 320, smem, s>>>(recs, h0, hT, static_cast<__nv_bfloat16 *>(o), T, H, cps, hdr,
-                                 seq_off, cu, err, debug_drop_first_copy());
+    a.err_word = device_error_word();
+    if (!a.err_word) return KDA_ERR_CUDA;
+    a.debug_drop_first_copy = debug_drop_first_copy();
+    const long long grid = units * ((a.mode == kStateMap ? 2 * D : D) / DVT);
+    if (grid > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    kern<<<(unsigned)grid, 320, smem, s>>>(a);
     return launch_status();
 }
 
@@ -174,7 +226,7 @@ static kda_status validate_fwd(const void *q, const void *k, const void *v, cons
                                int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
                                const void *o, const float *hT, const void *workspace,
                                size_t ws_bytes, bool need_inputs, bool need_outputs, int *N,
-                               WsLayout *L) {
+                               WsLayout *L, int nseg_req = 0) {
     if (B < 0 || T < 0 || num_seqs < 0) return KDA_ERR_INVALID_ARG;
     kda_status st = check_shape(H, dk, dv, dtype);
     if (st != KDA_OK) return st;
@@ -193,7 +245,10 @@ static kda_status validate_fwd(const void *q, const void *k, const void *v, cons
         return KDA_ERR_MISALIGNED;
     // outputs must not alias inputs (hT == h0 is the one allowed overlap)
     if (o && (o == q || o == k || o == v || o == g || o == beta)) return KDA_ERR_INVALID_ARG;
-    *L = ws_layout(B, T, H, dk, varlen ? num_seqs : 0, dtype);
+    if (nseg_req < 0 || nseg_req > kMaxSegmentsExplicit) return KDA_ERR_INVALID_ARG;
+    if (nseg_req > 1 && !is_tc_path(dtype, dk)) return KDA_ERR_UNSUPPORTED_SHAPE;
+    *L = ws_layout(B, T, H, dk, varlen ? num_seqs : 0, dtype, nseg_req,
+                   nseg_req > 0 ? kSplitSmBound : device_sms());
     if (!workspace || ws_bytes < L->total) return KDA_ERR_WORKSPACE_TOO_SMALL;
     if ((long long)(*N) * H * 8 > 0x7fffffffLL || L->max_chunks > 0x7fffffffLL)
         return KDA_ERR_INVALID_ARG;
@@ -241,9 +296,36 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *hdr = reinterpret_cast<int *>(ws + L.hdr);
     int *seq_off = reinterpret_cast<int *>(ws + L.seq_off);
-    const int cps = cu ? 0 : (T + C - 1) / C;
-    const int nunits = N * H;
-    return launch_state<32>(ws + L.recs, h0, hT, o, T, H, cps, nunits, hdr, seq_off, cu, s);
+    StateArgs a{};
+    a.recs = ws + L.recs;
+    a.h0 = h0;
+    a.hT = hT;
+    a.o = static_cast<__nv_bfloat16 *>(o);
+    a.T = T;
+    a.H = H;
+    a.cps = cu ? 0 : (T + C - 1) / C;
+    a.hdr = hdr;
+    a.seq_off = seq_off;
+    a.cu = cu;
+    a.nseg = L.nseg;
+    a.mode = kStateOutput;
+    const long long chains = (long long)N * H;
+    if (L.nseg <= 1) return launch_state<32>(a, chains, s);
+    // T-split: segment maps, the sequential combine, then the output pass from
+    // each segment's true starting state.
+    float *s_in = reinterpret_cast<float *>(ws + L.s_in);
+    float *seg_map = reinterpret_cast<float *>(ws + L.seg_map);
+    StateArgs m = a;
+    m.mode = kStateMap;
+    m.seg_map = seg_map;
+    kda_status st = launch_state<32>(m, chains * L.nseg, s);
+    if (st != KDA_OK) return st;
+    if (chains > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    kda_tc_seg_combine_kernel<<<dim3((unsigned)chains, D / 32), 256, 0, s>>>(
+        h0, seg_map, s_in, L.nseg, hdr, cu ? 1 : 0);
+    if ((st = launch_status()) != KDA_OK) return st;
+    a.s_in = s_in;
+    return launch_state<32>(a, chains * L.nseg, s);
 }
 
 kda_status kda_fwd_intra(const void *q, const void *k, const void *v, const float *g,
@@ -309,6 +391,38 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                                     cu_seqlens, s);
     return dispatch_simt<__nv_bfloat16>(dk, q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr,
                                         cu_seqlens, s);
+}
+
+size_t kda_fwd_segmented_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
+                                        int dtype, int num_segments) {
+    if (B < 0 || T < 0 || num_seqs < 0) return 0;
+    if (num_segments < 1 || num_segments > kMaxSegmentsExplicit) return 0;
+    if (check_shape(H, dk, dv, dtype) != KDA_OK) return 0;
+    if (num_seqs > 0 && B != 1) return 0;
+    if (num_segments > 1 && !is_tc_path(dtype, dk)) return 0;
+    return ws_layout(B, T, H, dk, num_seqs, dtype, num_segments).total;
+}
+
+kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *h0, const int32_t *cu_seqlens,
+                             int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
+                             int num_segments, void *o, float *hT, void *workspace,
+                             size_t ws_bytes, void *stream) {
+    if (num_segments < 1) return KDA_ERR_INVALID_ARG;
+    int N;
+    WsLayout L;
+    kda_status st = validate_fwd(q, k, v, g, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv,
+                                 dtype, o, hT, workspace, ws_bytes, true, true, &N, &L,
+                                 num_segments);
+    if (st != KDA_OK) return st;
+    if (N == 0) return KDA_OK;
+    if (!is_tc_path(dtype, dk))   // num_segments == 1 here: the plain pass
+        return kda_fwd(q, k, v, g, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv, dtype, o, hT,
+                       workspace, ws_bytes, stream);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = tc_intra(q, k, v, g, beta, cu_seqlens, N, T, H, L, workspace, s)) != KDA_OK)
+        return st;
+    return tc_inter(h0, cu_seqlens, N, T, H, L, o, hT, workspace, s);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const float *g,
@@ -397,7 +511,8 @@ extern "C" kda_status kda_fwd_noalloc(const void *q, const void *k, const void *
     WsLayout L;
     void *placeholder = reinterpret_cast<void *>(uintptr_t(256));
     kda_status st = validate_fwd(q, k, v, g, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv,
-                                 dtype, o, hT, placeholder, SIZE_MAX, true, true, &N, &L);
+                                 dtype, o, hT, placeholder, SIZE_MAX, true, true, &N, &L,
+                                 /*nseg_req=*/1);   // never T-split: scratch holds records only
     if (st != KDA_OK) return st;
     if (!is_tc_path(dtype, dk)) return KDA_ERR_UNSUPPORTED_SHAPE;
     if (L.total > (size_t)KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_EXCEEDS_STATIC_SCRATCH;

@@ -591,7 +591,10 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 
 // ---------------------------------------------------------------------------
 // Kernel 2: inter-chunk state pass on tcgen05, warp-specialised.
-// grid = N * H * (D / DVT) CTAs of 320 threads (10 warps):
+// grid = units * tiles CTAs of 320 threads (10 warps).  A unit is one (sequence,
+// head) chain, or with a T-split one of its nseg consecutive segments (equal
+// numbers of chunks, the last may be shorter or empty); tiles = D / DVT column
+// slices of the state.  Roles:
 //   warps 0-3  state:    thread t owns key row t of the fp32 state tile
 //                        S[:, col0:col0+DVT] in registers; per chunk it applies
 //                        S <- exp(G_C) S + R + (M' S) and writes the bf16 copy of
@@ -609,7 +612,31 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 // M' S on the tensor core -> state update -> bf16 copy -> next M' S.  Every wait is
 // bounded; a wait that runs out sets the shared abort flag and the timeout bit, all
 // roles stop, the CTA drains what it issued, frees its tensor memory and returns.
+//
+// Modes.  kStateOutput: the pass proper -- outputs for every chunk, the unit's
+// starting state from h0 (or s_in, per unit, after a T-split), the final state to
+// hT (last segment only).  kStateMap: the first pass of the T-split -- the unit's
+// affine map S_out = P S_in + R over its segment, obtained by running the same
+// recurrence on a widened state [R | P] of 2D columns: the R half from zero with
+// the records' R added, the P half from the identity without it (the map is affine,
+// so these are its offset and its linear part).  No outputs; [R | P] goes to seg_map.
 // ---------------------------------------------------------------------------
+constexpr int kStateOutput = 0, kStateMap = 1;
+
+struct StateArgs {
+    const uint8_t *recs;      // chunk records
+    const float *h0;          // [N, H, D, D] or null (zeros)
+    float *hT;                // [N, H, D, D] or null
+    __nv_bfloat16 *o;         // [tokens, H, D]
+    int T, H, cps;            // dense layout: tokens per sequence, heads, chunks per sequence
+    const int *hdr, *seq_off, *cu;   // packed layout (cu != null): chunk offsets per sequence
+    int *err_word;
+    int debug_drop_first_copy;
+    int nseg;                 // segments per chain (1: no T-split)
+    int mode;                 // kStateOutput or kStateMap
+    const float *s_in;        // kStateOutput after a T-split: [units, D, D] starting states
+    float *seg_map;           // kStateMap: [units, D, 2D] = [R | P] per unit
+};
 template <int DVT>
 struct T5Layout {
     static_assert(DVT == 32 || DVT == 64, "column tile");
@@ -641,12 +668,12 @@ struct T5Layout {
 };
 
 template <int DVT>
-__global__ void __launch_bounds__(320, 1)
-kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT,
-                    __nv_bfloat16 *__restrict__ o, int T, int H, int cps,
-                    const int *__restrict__ hdr, const int *__restrict__ seq_off,
-                    const int *__restrict__ cu, int *err_word, int debug_drop_first_copy) {
+__global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a) {
     using L = T5Layout<DVT>;
+    const uint8_t *__restrict__ recs = a.recs;
+    __nv_bfloat16 *__restrict__ o = a.o;
+    const int H = a.H;
+    const bool map_mode = a.mode == kStateMap;
     constexpr int NA = L::NA, NB = L::NB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -662,25 +689,37 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 4);
     int *cnt = reinterpret_cast<int *>(sm + L::OFF_MISC + 8);   // [0] ring A issued, [1] ring B issued, [2] MMA issued
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // 1-D grid, column tile fastest so the tiles of one chain run side by side
+    // 1-D grid, column tile fastest so the tiles of one unit run side by side
     // and share the chunk records through L2.
-    const int tile = blockIdx.x % (D / DVT), col0 = tile * DVT;
-    const int chain = blockIdx.x / (D / DVT), n = chain / H, h = chain % H;
+    const int tiles = (map_mode ? 2 * D : D) / DVT;
+    const int tile = blockIdx.x % tiles, unit = blockIdx.x / tiles;
+    const int chain = unit / a.nseg, seg = unit % a.nseg, n = chain / H, h = chain % H;
+    const bool p_half = map_mode && tile >= D / DVT;   // linear part of the map: no R
+    const int col0 = (tile % (D / DVT)) * DVT;
 
     int c_begin, c_end, seq_t0, seq_len;
-    if (cu) {
-        if (!hdr[0]) return;
-        c_begin = seq_off[n];
-        c_end = seq_off[n + 1];
-        seq_t0 = cu[n];
-        seq_len = cu[n + 1] - cu[n];
+    if (a.cu) {
+        if (!a.hdr[0]) return;
+        c_begin = a.seq_off[n];
+        c_end = a.seq_off[n + 1];
+        seq_t0 = a.cu[n];
+        seq_len = a.cu[n + 1] - a.cu[n];
     } else {
-        c_begin = n * cps;
-        c_end = c_begin + cps;
-        seq_t0 = n * T;
-        seq_len = T;
+        c_begin = n * a.cps;
+        c_end = c_begin + a.cps;
+        seq_t0 = n * a.T;
+        seq_len = a.T;
+    }
+    {   // this unit's segment of the chain
+        const int nch = c_end - c_begin, per = (nch + a.nseg - 1) / a.nseg;
+        const int lo = min(nch, seg * per), hi = min(nch, lo + per);
+        c_begin += lo;
+        c_end = c_begin + (hi - lo);
+        seq_t0 += lo * C;
+        seq_len -= lo * C;
     }
     const int nchunks = c_end - c_begin;
+    int *err_word = a.err_word;
 
     if (tid == 0) {
         for (int s = 0; s < NA; ++s) { mbar_init(&full_a[s], 1); mbar_init(&a_free[s], 128); }
@@ -716,15 +755,23 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
         // ---------------- state warps ----------------
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         float S[DVT];
-        const size_t sbase = (size_t)chain * D * D + (size_t)tid * D + col0;
+        const size_t row_off = (size_t)tid * D + col0;
+        const float *init = nullptr;
+        if (!map_mode)
+            init = a.s_in ? a.s_in + (size_t)unit * D * D + row_off
+                          : (a.h0 ? a.h0 + (size_t)chain * D * D + row_off : nullptr);
 #pragma unroll
         for (int i = 0; i < DVT; i += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (h0) x = *reinterpret_cast<const float4 *>(h0 + sbase + i);
+            if (init) x = *reinterpret_cast<const float4 *>(init + i);
             S[i] = x.x;
             S[i + 1] = x.y;
             S[i + 2] = x.z;
             S[i + 3] = x.w;
+        }
+        if (p_half) {   // identity columns col0 .. col0 + DVT - 1
+#pragma unroll
+            for (int i = 0; i < DVT; ++i) S[i] = (tid == col0 + i) ? 1.f : 0.f;
         }
         auto write_sb = [&](int buf) {   // bf16 copy of row tid, then signal it
             uint8_t *sb = sm + L::OFF_SB + buf * L::SB_BYTES;
@@ -749,8 +796,9 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
             const float gam = reinterpret_cast<const float *>(st + L::A_GC)[tid];
             uint4 rv[DVT / 8];
 #pragma unroll
-            for (int i = 0; i < DVT / 8; ++i)   // row tid of the R slice
-                rv[i] = *reinterpret_cast<const uint4 *>(st + L::A_R + core_off(D, tid, 8 * i));
+            for (int i = 0; i < DVT / 8; ++i)   // row tid of the R slice (zero for P)
+                rv[i] = p_half ? make_uint4(0u, 0u, 0u, 0u)
+                               : *reinterpret_cast<const uint4 *>(st + L::A_R + core_off(D, tid, 8 * i));
             // the tensor-memory load below is warp-collective: decide as a warp
             ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(done_s, j & 1));
             if (!ok) { fail(); break; }
@@ -772,8 +820,12 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
             }
             if (j + 1 < nchunks) write_sb((j + 1) & 1);
         }
-        if (!*abort_flag && hT && j == nchunks) {
-            float *dst = hT + sbase;
+        float *dst = nullptr;
+        if (map_mode)
+            dst = a.seg_map + ((size_t)unit * D + tid) * (2 * D) + tile * DVT;
+        else if (a.hT && seg == a.nseg - 1)
+            dst = a.hT + (size_t)chain * D * D + row_off;
+        if (!*abort_flag && dst && j == nchunks) {
 #pragma unroll
             for (int i = 0; i < DVT; i += 4)
                 *reinterpret_cast<float4 *>(dst + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
@@ -785,9 +837,10 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
         for (int j = 0; j < nchunks && !*abort_flag; ++j) {
             const int sa = j % NA, sbb = j % NB;
             bool ok = mbar_wait_bounded(&full_a[sa], (j / NA) & 1) &&
-                      mbar_wait_bounded(&full_b[sbb], (j / NB) & 1) &&
+                      (map_mode || mbar_wait_bounded(&full_b[sbb], (j / NB) & 1)) &&
                       mbar_wait_bounded(sb_full, j & 1) &&
-                      (j < 2 || mbar_wait_bounded(&do_free[j & 1], ((j - 2) >> 1) & 1));
+                      (map_mode || j < 2 ||
+                       mbar_wait_bounded(&do_free[j & 1], ((j - 2) >> 1) & 1));
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) { fail(); break; }
             if (t5::elect_one()) {
@@ -804,22 +857,24 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
                     t5::mma_bf16(tmem, am0 + (uint64_t)((ks * 2 * D * 16) >> 4),
                                  bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idS, ks > 0);
                 t5::commit(done_s);
-                const uint32_t dO = tmem + DVT + (j & 1) * DVT;
+                if (!map_mode) {
+                    const uint32_t dO = tmem + DVT + (j & 1) * DVT;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    t5::mma_bf16(dO, aq0 + (uint64_t)((ks * 2 * C * 16) >> 4),
-                                 bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idO, ks > 0);
-                t5::commit(&done_o[j & 1]);
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        t5::mma_bf16(dO, aq0 + (uint64_t)((ks * 2 * C * 16) >> 4),
+                                     bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idO, ks > 0);
+                    t5::commit(&done_o[j & 1]);
+                }
                 cnt[2] = j + 1;
             }
             __syncwarp();
         }
     } else if (warp < 9) {
-        // ---------------- output warps ----------------
+        // ---------------- output warps (none in the map pass) ----------------
         const int q = warp & 3;                          // tensor-memory lane quarter
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const int orow = q * 16 + lane;                  // output row of lanes 0..15
-        for (int j = 0; j < nchunks && !*abort_flag; ++j) {
+        for (int j = 0; j < (map_mode ? 0 : nchunks) && !*abort_flag; ++j) {
             const int sbb = j % NB;
             bool ok = mbar_wait_bounded(&done_o[j & 1], (j >> 1) & 1) &&
                       mbar_wait_bounded(&full_b[sbb], (j / NB) & 1);
@@ -861,15 +916,16 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
                 uint64_t *bar = &full_a[s];
                 uint8_t *dst = sm + s * L::A_BYTES;
                 const uint8_t *rec = rec_of(c);
-                mbar_arrive_expect_tx(bar, L::A_RAW);
+                mbar_arrive_expect_tx(bar, p_half ? L::A_RAW - L::R_BYTES : L::A_RAW);
                 cnt[0] = c + 1;
-                if (debug_drop_first_copy && c == 0) continue;   // test hook: the wait must run out
+                if (a.debug_drop_first_copy && c == 0) continue;   // test hook: the wait must run out
                 bulk_g2s(dst, rec + REC_M, D * D * 2, bar);
                 bulk_g2s(dst + L::A_GC, rec + REC_GC, D * 4, bar);
-                bulk_g2s(dst + L::A_R, rec + REC_R + core_off(D, 0, col0), L::R_BYTES, bar);
+                if (!p_half)
+                    bulk_g2s(dst + L::A_R, rec + REC_R + core_off(D, 0, col0), L::R_BYTES, bar);
             }
         } else if (lane == 1) {
-            for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+            for (int c = 0; c < (map_mode ? 0 : nchunks) && !*abort_flag; ++c) {
                 const int s = c % NB;
                 if (c >= NB && !mbar_wait_bounded(&b_free[s], ((c - NB) / NB) & 1)) { fail(); break; }
                 fence_proxy_async_smem();
@@ -893,12 +949,79 @@ kda_tc_state_kernel(const uint8_t *__restrict__ recs, const float *h0, float *hT
             mbar_wait_bounded(&full_a[c % NA], (c / NA) & 1);
         for (int c = max(0, cnt[1] - NB); c < cnt[1]; ++c)
             mbar_wait_bounded(&full_b[c % NB], (c / NB) & 1);
-        for (int c = max(0, cnt[2] - 2); c < cnt[2]; ++c)
-            mbar_wait_bounded(&done_o[c & 1], (c >> 1) & 1);
+        if (map_mode) {   // done_s is the last commit of each chunk
+            if (cnt[2] > 0) mbar_wait_bounded(done_s, (cnt[2] - 1) & 1);
+        } else {
+            for (int c = max(0, cnt[2] - 2); c < cnt[2]; ++c)
+                mbar_wait_bounded(&done_o[c & 1], (c >> 1) & 1);
+        }
     }
     __syncthreads();
     t5::fence_after_sync();
     if (warp == 0) t5::dealloc(tmem, L::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 3 (T-split only): the segment combine.  Walks each chain's segments in
+// order, S_{s+1} = P_s S_s + R_s in fp32, and stores every segment's starting state
+// S_s (S_0 = h0 or zero) for the output pass.  grid = (N * H, D / 32): one CTA per
+// chain and 32-column slice of the state (columns are independent); 256 threads,
+// thread t owns row t / 2, columns 16 (t & 1) .. +15 of the slice.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) kda_tc_seg_combine_kernel(
+    const float *__restrict__ h0, const float *__restrict__ seg_map, float *__restrict__ s_in,
+    int nseg, const int *__restrict__ hdr, int packed) {
+    __shared__ __align__(16) float Ssm[D][32];
+    if (packed && !hdr[0]) return;
+    const int chain = blockIdx.x, c0 = blockIdx.y * 32;
+    const int r = threadIdx.x >> 1, cl = (threadIdx.x & 1) * 16;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (h0) v = *reinterpret_cast<const float4 *>(h0 + ((size_t)chain * D + r) * D + c0 + cl + i);
+        x[i] = v.x;
+        x[i + 1] = v.y;
+        x[i + 2] = v.z;
+        x[i + 3] = v.w;
+    }
+    for (int s = 0; s < nseg; ++s) {
+        const size_t unit = (size_t)chain * nseg + s;
+        float *dst = s_in + (unit * D + r) * D + c0 + cl;
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4 *>(dst + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+        if (s == nseg - 1) break;
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4 *>(&Ssm[r][cl + i]) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+        __syncthreads();
+        const float *row = seg_map + (unit * D + r) * (2 * D);   // [R | P] row r
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(row + c0 + cl + i);
+            x[i] = v.x;
+            x[i + 1] = v.y;
+            x[i + 2] = v.z;
+            x[i + 3] = v.w;
+        }
+        for (int k4 = 0; k4 < D; k4 += 4) {
+            const float4 p = *reinterpret_cast<const float4 *>(row + D + k4);
+            const float pk[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                for (int i = 0; i < 16; i += 4) {
+                    const float4 sv = *reinterpret_cast<const float4 *>(&Ssm[k4 + u][cl + i]);
+                    x[i] = fmaf(pk[u], sv.x, x[i]);
+                    x[i + 1] = fmaf(pk[u], sv.y, x[i + 1]);
+                    x[i + 2] = fmaf(pk[u], sv.z, x[i + 2]);
+                    x[i + 3] = fmaf(pk[u], sv.w, x[i + 3]);
+                }
+            }
+        }
+        __syncthreads();
+    }
 }
 
 }  // namespace tc

@@ -68,6 +68,27 @@ def test_workspace_size(lib):
     assert 0 < ws(1, 64, 4, 32, 32, 0, F32) < 4096       # CUDA-core path: header only
 
 
+def test_segmented_workspace_size(lib):
+    seg = lib.kda_fwd_segmented_workspace_size
+    ws = lib.kda_fwd_workspace_size
+    unit = 128 * 128 * 4 * 3                               # s_in (D x D) + seg_map (D x 2D), fp32
+    # one segment: records only; the chain count (16) is too high for the split policy
+    assert seg(2, 4096, 8, 128, 128, 0, BF16, 1) == ws(2, 4096, 8, 128, 128, 0, BF16)
+    base = seg(1, 65536, 1, 128, 128, 0, BF16, 1)
+    for n in (2, 5, 32):
+        extra = seg(1, 65536, 1, 128, 128, 0, BF16, n) - base
+        assert unit * n <= extra < unit * n + 512
+    # the policy sizes for a 192-SM bound: 192 / (1 chain * 8 map tiles) = 24 segments
+    assert ws(1, 65536, 1, 128, 128, 0, BF16) == seg(1, 65536, 1, 128, 128, 0, BF16, 24)
+    # ... but never below 16 chunks per segment: 2048 tokens = 32 chunks -> 2 segments
+    assert ws(1, 2048, 1, 128, 128, 0, BF16) == seg(1, 2048, 1, 128, 128, 0, BF16, 2)
+    assert ws(1, 1024, 1, 128, 128, 0, BF16) == seg(1, 1024, 1, 128, 128, 0, BF16, 1)
+    assert seg(1, 100, 1, 128, 128, 0, BF16, 0) == 0      # bad counts
+    assert seg(1, 100, 1, 128, 128, 0, BF16, 4097) == 0
+    assert seg(1, 100, 1, 64, 64, 0, F32, 2) == 0         # split needs the tensor-core path
+    assert seg(1, 100, 1, 64, 64, 0, F32, 1) == ws(1, 100, 1, 64, 64, 0, F32)
+
+
 def _fwd(lib, ptr=0x10000, ws=1 << 40, **over):
     a = dict(q=ptr, k=ptr, v=ptr, g=ptr, beta=ptr, h0=None, cu=None, num_seqs=0, B=1, T=64,
              H=2, dk=128, dv=128, dtype=BF16, o=ptr + 0x100000, hT=None, work=ptr, ws=ws,
