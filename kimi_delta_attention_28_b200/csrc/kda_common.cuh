@@ -55,6 +55,20 @@ KDA_DEVINL void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                  : "r"(addr));
 }
 
+KDA_DEVINL void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(addr));
+}
+
+// 2^x by the PTX instruction ex2.approx.ftz.f32 (relative error about 2^-22;
+// results below the normal fp32 range flush to zero).
+KDA_DEVINL float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // 16-byte async global->shared copy; src_bytes < 16 zero-fills the remainder.
 KDA_DEVINL void cp_async16(void *smem, const void *gmem, int src_bytes = 16) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),

@@ -139,19 +139,21 @@ __global__ void __launch_bounds__(1024) kda_chunk_map_kernel(const int *__restri
 // Kernel 1: intra-chunk transform.  grid = (chunk slots, H), 256 threads.
 // ---------------------------------------------------------------------------
 constexpr int LDA = C + 8;      // padded bf16 row stride of the 64x64 blocks (144 B)
-constexpr int ZLD = 40;         // row stride of the per-warp substitution scratch
+constexpr int ZLD = 24;         // row stride of the per-warp 16x8 scratch (48 B: conflict-free)
 
 // The six sub-tile pairs (a, b), b < a, of a 64-token chunk.
 __constant__ int2 kPairs[6] = {{1, 0}, {2, 0}, {3, 0}, {2, 1}, {3, 1}, {3, 2}};
 
 struct PrepSmem {
-    // Five 16 KB tiles in swz128 layout, reused across phases:
-    //   r0: k -> k*exp(G_r - G_ref(a)) ; then, with r1, the [W|U] solution (swz256)
-    //   r1: q -> q*exp(G_r - G_ref(a))
-    //   r2: v
-    //   r3: k*exp(G_ref(b) - G_i) ; then per-warp scratch ; then Kt
-    //   r4: k*exp(G_r) ; then Qg
-    uint8_t r0[C * D * 2], r1[C * D * 2], r2[C * D * 2], r3[C * D * 2], r4[C * D * 2];
+    // Five 16 KB tiles, reused across phases:
+    //   ka: k*exp(G_r - G_ref(a)) (swz128); then T' = (I + A)^-1 Diag(b) (first 8 KB,
+    //       umma_k128) and the per-warp scratch of its substitution (last 8 KB)
+    //   qa: q*exp(G_r - G_ref(a)) (swz128); then, with kb, [W|U] (four umma_k128 planes)
+    //   kb: k*exp(G_ref(b) - G_i) (swz128)
+    //   xk: K*exp(G) (umma_k128 planes); then Kt (umma_k128 planes)
+    //   xv: V (umma_k128 planes); then Qg (swz128).  xk and xv are contiguous: together
+    //       they are the N = 256 right operand [K*exp G | V] of the [W|U] product.
+    uint8_t ka[C * D * 2], qa[C * D * 2], kb[C * D * 2], xk[C * D * 2], xv[C * D * 2];
     __nv_bfloat16 akkn[C * LDA];   // -b_r A_ri, sub-tile blocks b < a (bf16)
     uint8_t aqk[C * C * 2];        // masked query-key block, umma_k128 plane (bf16)
     __nv_bfloat16 taa[NST][ST * (ST + 8)];  // (I + A_aa)^-1, bf16
@@ -196,10 +198,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     uint8_t *rec = recs + ((size_t)cid * H + h) * REC_BYTES;
     const size_t rowstride = (size_t)H * D;  // elements between consecutive tokens
     const size_t base = ((size_t)t0 * H + h) * D;
-    const uint32_t s0 = smem_u32(sm.r0), s1 = smem_u32(sm.r1), s2 = smem_u32(sm.r2);
-    const uint32_t s3 = smem_u32(sm.r3), s4 = smem_u32(sm.r4);
+    const uint32_t s_ka = smem_u32(sm.ka), s_qa = smem_u32(sm.qa), s_kb = smem_u32(sm.kb);
 
-    if (warp == 0) {   // 256 tensor-memory columns for the P5 accumulators
+    if (warp == 0) {   // 256 tensor-memory columns, reused by the three products
         t5::alloc(tmem_slot, 2 * D);
         t5::relinquish();
     }
@@ -208,7 +209,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         fence_mbar_init();
     }
 
-    // ---- P0: stage k, q, v rows (zero-filled past len) and beta ----
+    // ---- P0: stage k, q (swz128), v (umma_k128 planes), zero-filled past len, and beta ----
 #pragma unroll
     for (int it = 0; it < 3 * C * (D / 8) / 256; ++it) {
         const int i = tid + it * 256;
@@ -216,7 +217,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         const int rem = i % (C * (D / 8));
         const int r = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
         const __nv_bfloat16 *src = (m == 0 ? k : (m == 1 ? q : v));
-        uint8_t *dst = (m == 0 ? sm.r0 : (m == 1 ? sm.r1 : sm.r2)) + swz128(r, c8);
+        uint8_t *dst = m == 0 ? sm.ka + swz128(r, c8)
+                              : (m == 1 ? sm.qa + swz128(r, c8) : sm.xv + umma_k128(C, r, c8));
         const bool ok = r < len;
         cp_async16(dst, ok ? (src + base + r * rowstride + c8) : src, ok ? 16 : 0);
     }
@@ -252,7 +254,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         const int pa = kPairs[p].x, pb = kPairs[p].y;
         float d = sm.u.p1.ref[pa][c] - sm.u.p1.ref[pb][c];
         for (int a = pb; a < pa; ++a) d += sm.u.p1.tot[a][c];
-        sm.mfac[p][c] = exp2f(d);
+        sm.mfac[p][c] = fast_exp2(d);
     }
     {
         float2 Ba = make_float2(0.f, 0.f), GC = make_float2(0.f, 0.f);
@@ -267,26 +269,26 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             GC.y += x.y;
         }
         const float2 Gref = gam[ST / 2 - 1], Gend = gam[ST - 1];   // local to the sub-tile
-        const float2 f1 = make_float2(exp2f(-Gref.x), exp2f(-Gref.y));                   // >= 1
-        const float2 f2 = make_float2(exp2f(Gref.x - Gend.x), exp2f(Gref.y - Gend.y));   // >= 1
-        const float2 eB = make_float2(exp2f(Ba.x), exp2f(Ba.y));                         // <= 1
-        const float2 fC = make_float2(exp2f(GC.x - Ba.x - Gend.x), exp2f(GC.y - Ba.y - Gend.y));
+        const float2 f1 = make_float2(fast_exp2(-Gref.x), fast_exp2(-Gref.y));                   // >= 1
+        const float2 f2 = make_float2(fast_exp2(Gref.x - Gend.x), fast_exp2(Gref.y - Gend.y));   // >= 1
+        const float2 eB = make_float2(fast_exp2(Ba.x), fast_exp2(Ba.y));                         // <= 1
+        const float2 fC = make_float2(fast_exp2(GC.x - Ba.x - Gend.x), fast_exp2(GC.y - Ba.y - Gend.y));
 #pragma unroll
         for (int j = 0; j < ST; ++j) {
             const int r = a1 * ST + j;
             const int off = swz128(r, c0);
             // every factor below lies in [e^-80, e^40] for g in (-5, 0]
-            const float2 E1 = make_float2(exp2f(gam[j].x), exp2f(gam[j].y));
-            const float2 E2 = make_float2(exp2f(Gend.x - gam[j].x), exp2f(Gend.y - gam[j].y));
-            const float2 kf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.r0 + off));
-            const float2 qf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.r1 + off));
-            *reinterpret_cast<uint32_t *>(sm.r0 + off) =
+            const float2 E1 = make_float2(fast_exp2(gam[j].x), fast_exp2(gam[j].y));
+            const float2 E2 = make_float2(fast_exp2(Gend.x - gam[j].x), fast_exp2(Gend.y - gam[j].y));
+            const float2 kf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.ka + off));
+            const float2 qf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.qa + off));
+            *reinterpret_cast<uint32_t *>(sm.ka + off) =
                 pack_bf16x2(kf.x * E1.x * f1.x, kf.y * E1.y * f1.y);
-            *reinterpret_cast<uint32_t *>(sm.r1 + off) =
+            *reinterpret_cast<uint32_t *>(sm.qa + off) =
                 pack_bf16x2(qf.x * E1.x * f1.x, qf.y * E1.y * f1.y);
-            *reinterpret_cast<uint32_t *>(sm.r3 + off) =
+            *reinterpret_cast<uint32_t *>(sm.kb + off) =
                 pack_bf16x2(kf.x * E2.x * f2.x, kf.y * E2.y * f2.y);
-            *reinterpret_cast<uint32_t *>(sm.r4 + off) =
+            *reinterpret_cast<uint32_t *>(sm.xk + umma_k128(C, r, c0)) =
                 pack_bf16x2(kf.x * E1.x * eB.x, kf.y * E1.y * eB.y);
             *reinterpret_cast<uint32_t *>(rec + REC_QG_SCRATCH + off) =
                 pack_bf16x2(qf.x * E1.x * eB.x, qf.y * E1.y * eB.y);
@@ -295,7 +297,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         if (a1 == NST - 1)
             *reinterpret_cast<float2 *>(rec + REC_GC + c0 * 4) =
-                make_float2(exp2f(GC.x), exp2f(GC.y));
+                make_float2(fast_exp2(GC.x), fast_exp2(GC.y));
     }
     __syncthreads();
 
@@ -317,9 +319,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             uint32_t lk[4], lq[4], bfr[4];
-            ldsm_x4(lk, s0 + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-            ldsm_x4(lq, s1 + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-            ldsm_x4(bfr, s3 + swz128(b * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
+            ldsm_x4(lk, s_ka + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+            ldsm_x4(lq, s_qa + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+            ldsm_x4(bfr, s_kb + swz128(b * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
             // right rows of sub-tile b move their reference from G_ref(b) to G_ref(a)
             const int cc = ks * 16 + 2 * tig;
             const float2 m01 = *reinterpret_cast<const float2 *>(&sm.mfac[warp][cc]);
@@ -356,9 +358,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
                 uint32_t lk[4], lq[4], bfr[4];
-                ldsm_x4(lk, s0 + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-                ldsm_x4(lq, s1 + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-                ldsm_x4(bfr, s3 + swz128(a * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
+                ldsm_x4(lk, s_ka + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+                ldsm_x4(lq, s_qa + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+                ldsm_x4(bfr, s_kb + swz128(a * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
                 mma_bf16_16816(ak[0], lk, bfr[0], bfr[1]);
                 mma_bf16_16816(ak[1], lk, bfr[2], bfr[3]);
                 mma_bf16_16816(aq[d][0], lq, bfr[0], bfr[1]);
@@ -406,99 +408,121 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     __syncthreads();
 
-    // ---- P3: [W|U] = (I + A)^-1 Diag(b) [K*exp G | V] by blocked forward substitution ----
-    // warp w owns 32 columns of the solution Y (over r0..r1, four 64-column planes in
-    // the umma_k128 layout, the tensor core's N-contiguous B operand): W[:, 32w..] for
-    // w < 4, U[:, 32(w-4)..] for w >= 4.  Only warp-level syncs are needed.
+    // ---- P3: T' = (I + A)^-1 Diag(b) by blocked forward substitution ----
+    // (I + A) T' = Diag(b), solved per 16-row block a:
+    //   T'_a = (I + A_aa)^-1 (Diag(b)_a - sum_{c<a} A_ac T'_c).
+    // Warp w owns columns 8w..8w+7 (inside column block w/2, above which T' is zero);
+    // each step is two m16n8k16 products and a 16x8 hop through shared memory.
     {
-        const uint32_t sY = s0;
-        uint8_t *Yb = sm.r0;
-        __nv_bfloat16 *Z = reinterpret_cast<__nv_bfloat16 *>(sm.r3) + warp * (ST * ZLD);
-        const uint8_t *X = warp < 4 ? sm.r4 : sm.r2;
-        const int xc = (warp & 3) * 32;   // column base inside X
-        const int yc = warp * 32;         // column base inside Y
-        for (int a = 0; a < NST; ++a) {
-            float acc[4][4];
+        uint8_t *Tp = sm.ka;
+        const uint32_t s_tp = s_ka;
+        __nv_bfloat16 *Z = reinterpret_cast<__nv_bfloat16 *>(sm.ka + C * C * 2) + warp * (ST * ZLD);
+        const int b = warp >> 1, i0 = warp * 8;
+        for (int a = 0; a < b; ++a)
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int r = a * ST + gid + 8 * hh;
-                    const float2 x = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
-                        X + swz128(r, xc + nt * 8 + 2 * tig)));
-                    acc[nt][2 * hh] = sm.beta[r] * x.x;
-                    acc[nt][2 * hh + 1] = sm.beta[r] * x.y;
-                }
-            for (int b = 0; b < a; ++b) {   // acc -= A_ab Y_b  (akkn holds -A)
-                uint32_t af[4];
-                ldsm_x4(af, smem_u32(sm.akkn + (a * ST + frag_a_row(lane)) * LDA + b * ST +
-                                     frag_a_col(lane)));
-#pragma unroll
-                for (int np = 0; np < 2; ++np) {
-                    uint32_t bb[4];
-                    ldsm_x4_t(bb, sY + umma_k128(C, b * ST + frag_bk_row(lane),
-                                                 yc + np * 16 + frag_bk_col(lane)));
-                    mma_bf16_16816(acc[2 * np], af, bb[0], bb[1]);
-                    mma_bf16_16816(acc[2 * np + 1], af, bb[2], bb[3]);
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int hh = 0; hh < 2; ++hh)
+                *reinterpret_cast<uint32_t *>(Tp + umma_k128(C, a * ST + gid + 8 * hh, i0 + 2 * tig)) = 0u;
+        for (int a = b; a < NST; ++a) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (a == b) {
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh)
-                    *reinterpret_cast<uint32_t *>(Z + (gid + 8 * hh) * ZLD + nt * 8 + 2 * tig) =
-                        pack_bf16x2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
-            __syncwarp();
-            float y[4][4] = {};
-            uint32_t at[4];
-            ldsm_x4(at, smem_u32(sm.taa[a] + frag_a_row(lane) * (ST + 8) + frag_a_col(lane)));
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                uint32_t bz[4];
-                ldsm_x4_t(bz, smem_u32(Z + frag_bk_row(lane) * ZLD + np * 16 + frag_bk_col(lane)));
-                mma_bf16_16816(y[2 * np], at, bz[0], bz[1]);
-                mma_bf16_16816(y[2 * np + 1], at, bz[2], bz[3]);
+                    for (int e = 0; e < 2; ++e) {
+                        const int r = a * ST + gid + 8 * hh, i = i0 + 2 * tig + e;
+                        acc[2 * hh + e] = (r == i) ? sm.beta[i] : 0.f;
+                    }
+            } else {
+                for (int c = b; c < a; ++c) {   // acc += (-A_ac) T'_c   (akkn holds -A)
+                    uint32_t af[4], bf[2];
+                    ldsm_x4(af, smem_u32(sm.akkn + (a * ST + frag_a_row(lane)) * LDA + c * ST +
+                                         frag_a_col(lane)));
+                    ldsm_x2_t(bf, s_tp + umma_k128(C, c * ST + (lane & 15), i0));
+                    mma_bf16_16816(acc, af, bf[0], bf[1]);
+                }
             }
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int hh = 0; hh < 2; ++hh)
+                *reinterpret_cast<uint32_t *>(Z + (gid + 8 * hh) * ZLD + 2 * tig) =
+                    pack_bf16x2(acc[2 * hh], acc[2 * hh + 1]);
+            __syncwarp();
+            uint32_t at[4], bz[2];
+            ldsm_x4(at, smem_u32(sm.taa[a] + frag_a_row(lane) * (ST + 8) + frag_a_col(lane)));
+            ldsm_x2_t(bz, smem_u32(Z + (lane & 15) * ZLD));
+            float y[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16_16816(y, at, bz[0], bz[1]);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int r = a * ST + gid + 8 * hh;
-                    *reinterpret_cast<uint32_t *>(Yb + umma_k128(C, r, yc + nt * 8 + 2 * tig)) =
-                        pack_bf16x2(y[nt][2 * hh], y[nt][2 * hh + 1]);
-                }
+            for (int hh = 0; hh < 2; ++hh)
+                *reinterpret_cast<uint32_t *>(Tp + umma_k128(C, a * ST + gid + 8 * hh, i0 + 2 * tig)) =
+                    pack_bf16x2(y[2 * hh], y[2 * hh + 1]);
             __syncwarp();
         }
     }
-    __syncthreads();
 
-    // ---- P4: Kt and Qg back from the record's scratch area into r3 / r4 ----
-#pragma unroll
-    for (int it = 0; it < 2 * C * D * 2 / 16 / 256; ++it) {
-        const int i = tid + it * 256;                  // 16-byte chunk index
-        const int m = i / (C * D * 2 / 16), off = (i % (C * D * 2 / 16)) * 16;
-        cp_async16((m == 0 ? sm.r3 : sm.r4) + off,
-                   rec + (m == 0 ? REC_KT_SCRATCH : REC_QG_SCRATCH) + off);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-
-    // ---- P5: the chunk's affine map, on tcgen05 (accumulators in tensor memory) ----
-    //   D1 = Kt^T [W|U]  (M = 128 key rows, N = 256, K = 64): M' = -D1[:, :128], R = D1[:, 128:]
-    //   D2 = Aqk  [W|U]  (M = 64 chunk rows):                 Q' = Qg - D2[:, :128], O0 = D2[:, 128:]
-    // Both reuse the same 256 tensor-memory columns, one after the other.
+    // ---- P4: three tcgen05 products, accumulators in tensor memory (256 columns) ----
+    //   Y  = T' [K*exp G | V]  (M = 64, N = 256, K = 64):  [W|U], to shared memory as bf16
+    //   D1 = Kt^T [W|U]        (M = 128 key rows):         M' = -D1[:, :128], R = D1[:, 128:]
+    //   D2 = Aqk  [W|U]        (M = 64 chunk rows):        Q' = Qg - D2[:, :128], O0 = D2[:, 128:]
     {
-        fence_proxy_async_smem();   // Y and aqk (generic stores), Kt (cp.async) -> tensor core
+        fence_proxy_async_smem();   // T' (generic stores) -> tensor core
         t5::fence_before_sync();
         __syncthreads();
         const uint32_t tmem = *tmem_slot;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint64_t ydesc = t5::smem_desc(s0, C * 128, 1024, t5::kSwz128);   // [W|U], N-major
         if (warp == 0) {
             if (t5::elect_one()) {
                 t5::fence_after_sync();
-                const uint64_t kdesc = t5::smem_desc(s3, C * 128, 1024, t5::kSwz128);  // Kt^T, M-major
+                const uint64_t tdesc = t5::smem_desc(s_ka, 16, 1024, t5::kSwz128);                  // T', K-major
+                const uint64_t xdesc = t5::smem_desc(smem_u32(sm.xk), C * 128, 1024, t5::kSwz128);  // X, N-major
+                constexpr uint32_t id = t5::idesc_bf16(64, 2 * D, 0, 1);
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    t5::mma_bf16(tmem, tdesc + (uint64_t)((ks * 32) >> 4),
+                                 xdesc + (uint64_t)((ks * 2048) >> 4), id, ks > 0);
+                t5::commit(&sm.mma_bar);
+            }
+            __syncwarp();
+        }
+        bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 0));
+        t5::fence_after_sync();
+        // X is consumed: bring Kt (into xk) and Qg (into xv) back from the record's scratch
+        // area while [W|U] leaves tensor memory
+#pragma unroll
+        for (int it = 0; it < 2 * C * D * 2 / 16 / 256; ++it) {
+            const int i = tid + it * 256;                  // 16-byte chunk index
+            const int m = i / (C * D * 2 / 16), off = (i % (C * D * 2 / 16)) * 16;
+            cp_async16((m == 0 ? sm.xk : sm.xv) + off,
+                       rec + (m == 0 ? REC_KT_SCRATCH : REC_QG_SCRATCH) + off);
+        }
+        cp_async_commit();
+        if (ok) {   // rows r = 16(w&3) + lane (lanes 0..15); warps 0-3 -> W, warps 4-7 -> U
+            const int r = (warp & 3) * 16 + lane, cb = (warp >> 2) * D;
+#pragma unroll
+            for (int qq = 0; qq < D / 32; ++qq) {
+                float vv[32];
+                t5::ld32(tmem + lane_base + cb + qq * 32, vv);
+                if (lane < 16) {
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(vv[c8 * 8 + 0], vv[c8 * 8 + 1]);
+                        pk.y = pack_bf16x2(vv[c8 * 8 + 2], vv[c8 * 8 + 3]);
+                        pk.z = pack_bf16x2(vv[c8 * 8 + 4], vv[c8 * 8 + 5]);
+                        pk.w = pack_bf16x2(vv[c8 * 8 + 6], vv[c8 * 8 + 7]);
+                        *reinterpret_cast<uint4 *>(sm.qa + umma_k128(C, r, cb + qq * 32 + c8 * 8)) = pk;
+                    }
+                }
+            }
+        }
+        cp_async_wait<0>();
+        fence_proxy_async_smem();   // [W|U] (generic stores), Kt (cp.async) -> tensor core
+        t5::fence_before_sync();
+        ok = __syncthreads_and(ok) != 0;
+        const uint64_t ydesc = t5::smem_desc(s_qa, C * 128, 1024, t5::kSwz128);   // [W|U], N-major
+        if (ok && warp == 0) {
+            if (t5::elect_one()) {
+                t5::fence_after_sync();
+                const uint64_t kdesc = t5::smem_desc(smem_u32(sm.xk), C * 128, 1024, t5::kSwz128);  // Kt^T, M-major
                 constexpr uint32_t id = t5::idesc_bf16(128, 2 * D, 1, 1);
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
@@ -508,23 +532,23 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
             __syncwarp();
         }
-        bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 0));
+        ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 1));
         t5::fence_after_sync();
         if (ok) {   // lane = key row; warps 0-3 -> M' (columns 0..127), warps 4-7 -> R
             const int m = (warp & 3) * 32 + lane, cb = (warp >> 2) * D;
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-                float v[32];
-                t5::ld32(tmem + lane_base + cb + q * 32, v);
+            for (int qq = 0; qq < D / 32; ++qq) {
+                float vv[32];
+                t5::ld32(tmem + lane_base + cb + qq * 32, vv);
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
-                    const int c = q * 32 + c8 * 8;
+                    const int c = qq * 32 + c8 * 8;
                     const float sg = warp < 4 ? -1.f : 1.f;
                     uint4 pk;
-                    pk.x = pack_bf16x2(sg * v[c8 * 8 + 0], sg * v[c8 * 8 + 1]);
-                    pk.y = pack_bf16x2(sg * v[c8 * 8 + 2], sg * v[c8 * 8 + 3]);
-                    pk.z = pack_bf16x2(sg * v[c8 * 8 + 4], sg * v[c8 * 8 + 5]);
-                    pk.w = pack_bf16x2(sg * v[c8 * 8 + 6], sg * v[c8 * 8 + 7]);
+                    pk.x = pack_bf16x2(sg * vv[c8 * 8 + 0], sg * vv[c8 * 8 + 1]);
+                    pk.y = pack_bf16x2(sg * vv[c8 * 8 + 2], sg * vv[c8 * 8 + 3]);
+                    pk.z = pack_bf16x2(sg * vv[c8 * 8 + 4], sg * vv[c8 * 8 + 5]);
+                    pk.w = pack_bf16x2(sg * vv[c8 * 8 + 6], sg * vv[c8 * 8 + 7]);
                     uint8_t *dst = rec + (warp < 4 ? REC_M : REC_R) + core_off(D, m, c);
                     *reinterpret_cast<uint4 *>(dst) = pk;
                 }
@@ -545,23 +569,23 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
             __syncwarp();
         }
-        ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 1));
+        ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 0));
         t5::fence_after_sync();
         if (ok) {   // rows r = 16(w&3) + lane (lanes 0..15); warps 0-3 -> Q', warps 4-7 -> O0
             const int r = (warp & 3) * 16 + lane, cb = (warp >> 2) * D;
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-                float v[32];
-                t5::ld32(tmem + lane_base + cb + q * 32, v);
+            for (int qq = 0; qq < D / 32; ++qq) {
+                float vv[32];
+                t5::ld32(tmem + lane_base + cb + qq * 32, vv);
                 if (lane < 16) {
 #pragma unroll
                     for (int c8 = 0; c8 < 4; ++c8) {
-                        const int c = q * 32 + c8 * 8;
+                        const int c = qq * 32 + c8 * 8;
                         float x[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = v[c8 * 8 + e];
+                        for (int e = 0; e < 8; ++e) x[e] = vv[c8 * 8 + e];
                         if (warp < 4) {   // Q' = Qg - Aqk W
-                            const uint4 qg = *reinterpret_cast<const uint4 *>(sm.r4 + swz128(r, c));
+                            const uint4 qg = *reinterpret_cast<const uint4 *>(sm.xv + swz128(r, c));
                             const uint32_t u[4] = {qg.x, qg.y, qg.z, qg.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
