@@ -283,10 +283,7 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype.itemsize == 2 else "f32",
         "data": "synthetic (seeded; q,k L2-normalised, g=-5*sigmoid(N(-3,1)), beta=sigmoid(N(0,1)))",
-        "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
-                   "h0": "N(0, 0.1^2)" if inp["h0"] is not None else "zeros",
-                   "varlen_seqs": nseq, "l2": "flushed between steps (256 MiB write)",
-                   "parallelism": f"replicas x{world} (independent batches)"},
+        "config": prefill_config(w, inp, world),
         "roofline": {"bound": "hbm", "kernel": "kda_tc_prep_kernel" if dom == "intra"
                      else "kda_tc_state_kernel", "achieved": achieved, "peak": hbm_peak,
                      "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
@@ -440,6 +437,16 @@ def cpu_baseline(w, inp, budget_s=10.0, chains_per_step=None):
                       f"{elapsed:.1f} s; fp64 token-by-token C, OpenMP over (sequence, head)"}
 
 
+def prefill_config(w, inp, world):
+    """The `config` object of a prefill workload (shared by both arms)."""
+    B, T, H, dk = inp["q"].shape
+    nseq = 0 if inp["cu_seqlens"] is None else inp["cu_seqlens"].numel() - 1
+    return {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": inp["v"].shape[-1],
+            "h0": "N(0, 0.1^2)" if inp["h0"] is not None else "zeros",
+            "varlen_seqs": nseq, "l2": "flushed between steps (256 MiB write)",
+            "parallelism": f"replicas x{world} (independent batches)"}
+
+
 def run_reference(args, world, rank):
     """The oracle on a bounded sample of the workload, timed per step."""
     import numpy as np
@@ -484,7 +491,7 @@ def run_reference(args, world, rank):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded), same generator as the GPU arm",
-            "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv},
+            "config": prefill_config(w, inp, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": int(used),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -508,13 +515,13 @@ def main():
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference" and args.workload == "decode":
+        ap.error("the reference arm covers the prefill workloads")
     if args.impl == "reference":
         if rank != 0:
             return 0
         print(json.dumps(run_reference(args, world, rank)), flush=True)
         return 0
-    if args.impl == "reference" and args.workload == "decode":
-        ap.error("the reference arm covers the prefill workloads")
     world, rank, local = dist_setup(args)
     try:
         if args.workload == "decode":

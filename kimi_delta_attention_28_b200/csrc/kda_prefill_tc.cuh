@@ -674,9 +674,9 @@ struct T5Layout {
     static constexpr int SB_BYTES = D * DVT * 2;                         // one bf16 state copy
     static constexpr int OFF_B = NA * A_BYTES;
     static constexpr int OFF_SB = OFF_B + NB * B_BYTES;
-    // barriers: full_a[NA] full_b[NB] a_free[NA] b_free[NB] done_s done_o[2] sb_full do_free[2]
+    // barriers: full_a[NA] full_b[NB] a_free[NA] b_free[NB] done_s done_o[2] sb_full[4] do_free[2]
     static constexpr int OFF_BAR = OFF_SB + 2 * SB_BYTES;
-    static constexpr int NBAR = 2 * (NA + NB) + 6;
+    static constexpr int NBAR = 2 * (NA + NB) + 9;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;   // tmem slot, abort flag, counters
     static constexpr int BYTES = OFF_MISC + 32 + 1024;    // + slack for 1024-byte alignment
     static constexpr uint32_t TMEM_COLS = DVT == 32 ? 128 : 256;   // D_S | D_O[0] | D_O[1]
@@ -707,8 +707,8 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
     uint64_t *b_free = a_free + NA;
     uint64_t *done_s = b_free + NB;
     uint64_t *done_o = done_s + 1;     // [2] by chunk parity
-    uint64_t *sb_full = done_o + 2;
-    uint64_t *do_free = sb_full + 1;   // [2] by chunk parity
+    uint64_t *sb_full = done_o + 2;    // [4]: key rows 32w..32w+31 of the state copy written
+    uint64_t *do_free = sb_full + 4;   // [2] by chunk parity
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 4);
     int *cnt = reinterpret_cast<int *>(sm + L::OFF_MISC + 8);   // [0] ring A issued, [1] ring B issued, [2] MMA issued
@@ -751,7 +751,7 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
         mbar_init(done_s, 1);
         mbar_init(&done_o[0], 1);
         mbar_init(&done_o[1], 1);
-        mbar_init(sb_full, 128);
+        for (int w = 0; w < 4; ++w) mbar_init(&sb_full[w], 32);
         mbar_init(&do_free[0], 128);
         mbar_init(&do_free[1], 128);
         *abort_flag = 0;
@@ -809,7 +809,7 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
                 *reinterpret_cast<uint4 *>(sb + L::sb_off(tid, c8)) = pk;
             }
             fence_proxy_async_smem();   // generic writes -> tensor-core reads
-            mbar_arrive(sb_full);
+            mbar_arrive(&sb_full[warp]);   // this warp's K slab of the next products
         };
         write_sb(0);
         int j = 0;
@@ -862,13 +862,12 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
             const int sa = j % NA, sbb = j % NB;
             bool ok = mbar_wait_bounded(&full_a[sa], (j / NA) & 1) &&
                       (map_mode || mbar_wait_bounded(&full_b[sbb], (j / NB) & 1)) &&
-                      mbar_wait_bounded(sb_full, j & 1) &&
                       (map_mode || j < 2 ||
                        mbar_wait_bounded(&do_free[j & 1], ((j - 2) >> 1) & 1));
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) { fail(); break; }
+            bool slab_ok = true;
             if (t5::elect_one()) {
-                t5::fence_after_sync();
                 const uint32_t sb_addr = sm_addr + L::OFF_SB + (j & 1) * L::SB_BYTES;
                 const uint64_t bd0 = t5::smem_desc(sb_addr, 4096, 8 * L::SB_ROW, L::SB_SWZ);
                 // A operands in the core-matrix layout: 8-row groups 128 B apart (SBO),
@@ -876,22 +875,36 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
                 const uint64_t am0 = t5::smem_desc(sm_addr + sa * L::A_BYTES, D * 16, 128, 0);
                 const uint64_t aq0 = t5::smem_desc(sm_addr + L::OFF_B + sbb * L::B_BYTES,
                                                    C * 16, 128, 0);
+                // M'.S by K slabs: slab w (key rows 32w..32w+31, two K=16 steps) goes as
+                // soon as state warp w has written its rows of the copy
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    t5::mma_bf16(tmem, am0 + (uint64_t)((ks * 2 * D * 16) >> 4),
-                                 bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idS, ks > 0);
+                for (int w = 0; w < 4; ++w) {
+                    if (!mbar_wait_bounded(&sb_full[w], j & 1)) {
+                        slab_ok = false;
+                        break;
+                    }
+                    t5::fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const int ks = 2 * w + kk;
+                        t5::mma_bf16(tmem, am0 + (uint64_t)((ks * 2 * D * 16) >> 4),
+                                     bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idS, ks > 0);
+                    }
+                }
                 t5::commit(done_s);
-                if (!map_mode) {
+                if (!map_mode && slab_ok) {
                     const uint32_t dO = tmem + DVT + (j & 1) * DVT;
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks)
                         t5::mma_bf16(dO, aq0 + (uint64_t)((ks * 2 * C * 16) >> 4),
                                      bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idO, ks > 0);
                     t5::commit(&done_o[j & 1]);
+                } else if (!map_mode) {
+                    t5::commit(&done_o[j & 1]);   // so the drain below can wait on it
                 }
                 cnt[2] = j + 1;
             }
-            __syncwarp();
+            if (__any_sync(0xffffffffu, !slab_ok)) { fail(); break; }
         }
     } else if (warp < 9) {
         // ---------------- output warps (none in the map pass) ----------------
