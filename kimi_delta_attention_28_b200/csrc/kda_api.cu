@@ -280,11 +280,17 @@ static kda_status tc_intra(const void *q, const void *k, const void *v, const fl
     if (cudaFuncSetAttribute(kda_tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return KDA_ERR_CUDA;
-    dim3 grid((unsigned)L.max_chunks, H);
+    // persistent: two CTAs per SM (the kernel's shared memory allows no more), each
+    // walking the (chunk, head) items with a stride of the grid
+    const long long items = L.max_chunks * H;
+    if (items > 0x7fffffffLL - 4096) return KDA_ERR_INVALID_ARG;   // int item indices
+    const int sms = device_sms();
+    const long long cap = 2LL * (sms > 0 ? sms : 148);
+    const unsigned grid = (unsigned)(items < cap ? items : cap);
     kda_tc_prep_kernel<<<grid, 256, smem, s>>>(
         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-        static_cast<const __nv_bfloat16 *>(v), g, beta, T, H, cps, hdr, cu ? chunks : nullptr,
-        ws + L.recs, device_error_word());
+        static_cast<const __nv_bfloat16 *>(v), g, beta, T, H, cps, (int)L.max_chunks, hdr,
+        cu ? chunks : nullptr, ws + L.recs, device_error_word());
     return launch_status();
 }
 

@@ -74,6 +74,11 @@ KDA_DEVINL void cp_async16(void *smem, const void *gmem, int src_bytes = 16) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
                  "l"(gmem), "r"(src_bytes));
 }
+// 4-byte async global->shared copy (cp.async.ca); src_bytes = 0 writes zero.
+KDA_DEVINL void cp_async4(void *smem, const void *gmem, int src_bytes = 4) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_u32(smem)),
+                 "l"(gmem), "r"(src_bytes));
+}
 KDA_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
 KDA_DEVINL void cp_async_wait() {

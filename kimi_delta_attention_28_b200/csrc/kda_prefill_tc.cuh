@@ -136,7 +136,10 @@ __global__ void __launch_bounds__(1024) kda_chunk_map_kernel(const int *__restri
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 1: intra-chunk transform.  grid = (chunk slots, H), 256 threads.
+// Kernel 1: intra-chunk transform.  Persistent: grid = min(items, 2 per SM) CTAs of
+// 256 threads; CTA b takes the (chunk, head) items b, b + gridDim.x, ... and loads
+// each item's inputs while the previous item's last products and epilogues run, into
+// the tiles those phases have just released.
 // ---------------------------------------------------------------------------
 constexpr int LDA = C + 8;      // padded bf16 row stride of the 64x64 blocks (144 B)
 constexpr int ZLD = 24;         // row stride of the per-warp 16x8 scratch (48 B: conflict-free)
@@ -145,12 +148,14 @@ constexpr int ZLD = 24;         // row stride of the per-warp 16x8 scratch (48 B
 __constant__ int2 kPairs[6] = {{1, 0}, {2, 0}, {3, 0}, {2, 1}, {3, 1}, {3, 2}};
 
 struct PrepSmem {
-    // Five 16 KB tiles, reused across phases:
-    //   ka: k*exp(G_r - G_ref(a)) (swz128); then T' = (I + A)^-1 Diag(b) (first 8 KB,
-    //       umma_k128) and the per-warp scratch of its substitution (last 8 KB)
-    //   qa: q*exp(G_r - G_ref(a)) (swz128); then, with kb, [W|U] (four umma_k128 planes)
-    //   kb: k*exp(G_ref(b) - G_i) (swz128)
-    //   xk: K*exp(G) (umma_k128 planes); then Kt (umma_k128 planes)
+    // Five 16 KB tiles, reused across phases (an item's inputs arrive as: g rows 0-31
+    // in ka and rows 32-63 in xk, 512-byte rows; k in qa, q in kb (swz128); V in xv):
+    //   ka: g (rows 0-31); k*exp(G_r - G_ref(a)) (swz128); then T' = (I + A)^-1 Diag(b)
+    //       (first 8 KB, umma_k128) and the per-warp scratch of its substitution
+    //   qa: raw k; q*exp(G_r - G_ref(a)) (swz128); then, with kb, [W|U] (four umma_k128
+    //       planes)
+    //   kb: raw q; k*exp(G_ref(b) - G_i) (swz128)
+    //   xk: g (rows 32-63); K*exp(G) (umma_k128 planes); then Kt (umma_k128 planes)
     //   xv: V (umma_k128 planes); then Qg (swz128).  xk and xv are contiguous: together
     //       they are the N = 256 right operand [K*exp G | V] of the [W|U] product.
     uint8_t ka[C * D * 2], qa[C * D * 2], kb[C * D * 2], xk[C * D * 2], xv[C * D * 2];
@@ -173,7 +178,7 @@ struct PrepSmem {
 __global__ void __launch_bounds__(256, 2)
 kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
-                   const float *__restrict__ beta, int T, int H, int cps,
+                   const float *__restrict__ beta, int T, int H, int cps, int slots,
                    const int *__restrict__ hdr, const ChunkLoc *__restrict__ chunks,
                    uint8_t *__restrict__ recs, int *err_word) {
     extern __shared__ uint8_t smem_raw[];
@@ -183,22 +188,71 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     uint32_t *tmem_slot = &sm.tmem_slot;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
-    const int cid = blockIdx.x, h = blockIdx.y;
-
-    int t0, len;
-    if (chunks) {
-        if (!hdr[0] || cid >= hdr[1]) return;
-        t0 = chunks[cid].t0;
-        len = chunks[cid].len;
-    } else {
-        const int n = cid / cps, j = cid % cps;
-        t0 = n * T + j * C;
-        len = min(C, T - j * C);
-    }
-    uint8_t *rec = recs + ((size_t)cid * H + h) * REC_BYTES;
+    if (chunks && !hdr[0]) return;
+    const int items = (chunks ? min(hdr[1], slots) : slots) * H;
+    if ((int)blockIdx.x >= items) return;
     const size_t rowstride = (size_t)H * D;  // elements between consecutive tokens
-    const size_t base = ((size_t)t0 * H + h) * D;
     const uint32_t s_ka = smem_u32(sm.ka), s_qa = smem_u32(sm.qa), s_kb = smem_u32(sm.kb);
+
+    struct Item {
+        int t0, len, h;
+        size_t base;       // element offset of (token t0, head h, channel 0)
+        uint8_t *rec;
+    };
+    auto locate = [&](int item) {
+        Item it;
+        const int cid = item / H;
+        it.h = item % H;
+        if (chunks) {
+            it.t0 = chunks[cid].t0;
+            it.len = chunks[cid].len;
+        } else {
+            const int n = cid / cps, j = cid % cps;
+            it.t0 = n * T + j * C;
+            it.len = min(C, T - j * C);
+        }
+        it.base = ((size_t)it.t0 * H + it.h) * D;
+        it.rec = recs + ((size_t)cid * H + it.h) * REC_BYTES;
+        return it;
+    };
+    // input loads (16-byte cp.async, zero-filled past len), in the pieces the tail of
+    // the previous item releases them
+    auto load_g_half = [&](const Item &it, int half) {   // g rows 32 half .. +31
+        uint8_t *dst0 = half ? sm.xk : sm.ka;
+#pragma unroll
+        for (int m = 0; m < 32 * (D / 4) / 256; ++m) {
+            const int i = tid + m * 256, rr = i / (D / 4), c4 = (i % (D / 4)) * 4;
+            const int r = 32 * half + rr;
+            const bool ok = r < it.len;
+            cp_async16(dst0 + rr * (D * 4) + c4 * 4, ok ? g + it.base + r * rowstride + c4 : g,
+                       ok ? 16 : 0);
+        }
+    };
+    auto load_kq = [&](const Item &it) {                 // k -> qa, q -> kb (swz128)
+#pragma unroll
+        for (int m = 0; m < 2 * C * (D / 8) / 256; ++m) {
+            const int i = tid + m * 256, w = i / (C * (D / 8)), rem = i % (C * (D / 8));
+            const int r = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
+            const bool ok = r < it.len;
+            const __nv_bfloat16 *src = w ? q : k;
+            cp_async16((w ? sm.kb : sm.qa) + swz128(r, c8),
+                       ok ? src + it.base + r * rowstride + c8 : src, ok ? 16 : 0);
+        }
+    };
+    auto load_v_beta = [&](const Item &it) {             // V -> xv (umma_k128), beta
+#pragma unroll
+        for (int m = 0; m < C * (D / 8) / 256; ++m) {
+            const int i = tid + m * 256, r = i / (D / 8), c8 = (i % (D / 8)) * 8;
+            const bool ok = r < it.len;
+            cp_async16(sm.xv + umma_k128(C, r, c8), ok ? v + it.base + r * rowstride + c8 : v,
+                       ok ? 16 : 0);
+        }
+        if (tid < C) {
+            const bool ok = tid < it.len;
+            cp_async4(&sm.beta[tid], ok ? beta + (size_t)(it.t0 + tid) * H + it.h : beta,
+                      ok ? 4 : 0);
+        }
+    };
 
     if (warp == 0) {   // 256 tensor-memory columns, reused by the three products
         t5::alloc(tmem_slot, 2 * D);
@@ -208,36 +262,42 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         mbar_init(&sm.mma_bar, 1);
         fence_mbar_init();
     }
-
-    // ---- P0: stage k, q (swz128), v (umma_k128 planes), zero-filled past len, and beta ----
-#pragma unroll
-    for (int it = 0; it < 3 * C * (D / 8) / 256; ++it) {
-        const int i = tid + it * 256;
-        const int m = i / (C * (D / 8));
-        const int rem = i % (C * (D / 8));
-        const int r = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
-        const __nv_bfloat16 *src = (m == 0 ? k : (m == 1 ? q : v));
-        uint8_t *dst = m == 0 ? sm.ka + swz128(r, c8)
-                              : (m == 1 ? sm.qa + swz128(r, c8) : sm.xv + umma_k128(C, r, c8));
-        const bool ok = r < len;
-        cp_async16(dst, ok ? (src + base + r * rowstride + c8) : src, ok ? 16 : 0);
+    // the query-key block is read whole by the tensor core: its upper blocks stay zero
+    if (tid < 6 * ST * 2) {
+        const int p = tid / (ST * 2), rr = (tid / 2) % ST, half = tid & 1;
+        const int ba = kPairs[p].y, bb = kPairs[p].x;   // block (row ba, column bb), bb > ba
+        *reinterpret_cast<uint4 *>(sm.aqk + umma_k128(C, ba * ST + rr, bb * ST + half * 8)) =
+            make_uint4(0u, 0u, 0u, 0u);
     }
+    uint32_t mma_phase = 0;   // completions of mma_bar so far
+    bool ok = true;
+
+    Item cur = locate(blockIdx.x);
+    load_g_half(cur, 0);
+    load_g_half(cur, 1);
+    load_kq(cur);
+    load_v_beta(cur);
     cp_async_commit();
-    if (tid < C) sm.beta[tid] = tid < len ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+    const int nxt_item = item + gridDim.x;
+    const bool has_next = nxt_item < items;
+    const Item nxt = locate(has_next ? nxt_item : item);
+    uint8_t *rec = cur.rec;
+    cp_async_wait<0>();
+    __syncthreads();
 
     // ---- P1: cumulative decay and the scaled operands ----
     // thread -> channel pair (c0, c0+1) x sub-tile a1 (rows 16a1..16a1+15).  gam holds
-    // the cumsum local to the sub-tile, in log2 units.
+    // the cumsum local to the sub-tile, in log2 units (g rows past len arrive as zero).
     const int c0 = 2 * (tid & 63), a1 = tid >> 6;
     float2 gam[ST];
     {
         float2 run = make_float2(0.f, 0.f);
-        const float *gp = g + base + c0;
+        const uint8_t *gsrc = (a1 < 2 ? sm.ka : sm.xk) + (a1 & 1) * ST * (D * 4) + c0 * 4;
 #pragma unroll
         for (int j = 0; j < ST; ++j) {
-            const int r = a1 * ST + j;
-            const float2 gv = r < len ? *reinterpret_cast<const float2 *>(gp + r * rowstride)
-                                      : make_float2(0.f, 0.f);
+            const float2 gv = *reinterpret_cast<const float2 *>(gsrc + j * (D * 4));
             run.x += gv.x * kLog2e;
             run.y += gv.y * kLog2e;
             gam[j] = run;
@@ -245,8 +305,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         *reinterpret_cast<float2 *>(&sm.u.p1.tot[a1][c0]) = run;
         *reinterpret_cast<float2 *>(&sm.u.p1.ref[a1][c0]) = gam[ST / 2 - 1];
     }
-    cp_async_wait<0>();
-    __syncthreads();
+    __syncthreads();   // every g value is in registers; ka and xk may be overwritten
     // pair factors exp(G_ref(a) - G_ref(b)) <= 1 for the off-diagonal sub-tile blocks
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
@@ -280,8 +339,10 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             // every factor below lies in [e^-80, e^40] for g in (-5, 0]
             const float2 E1 = make_float2(fast_exp2(gam[j].x), fast_exp2(gam[j].y));
             const float2 E2 = make_float2(fast_exp2(Gend.x - gam[j].x), fast_exp2(Gend.y - gam[j].y));
-            const float2 kf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.ka + off));
-            const float2 qf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.qa + off));
+            // raw k sits in qa and raw q in kb at the same offset; this thread reads
+            // both before it overwrites them
+            const float2 kf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.qa + off));
+            const float2 qf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.kb + off));
             *reinterpret_cast<uint32_t *>(sm.ka + off) =
                 pack_bf16x2(kf.x * E1.x * f1.x, kf.y * E1.y * f1.y);
             *reinterpret_cast<uint32_t *>(sm.qa + off) =
@@ -300,14 +361,6 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 make_float2(fast_exp2(GC.x), fast_exp2(GC.y));
     }
     __syncthreads();
-
-    // the query-key block is read whole by the tensor core: zero its upper blocks
-    if (tid < 6 * ST * 2) {
-        const int p = tid / (ST * 2), rr = (tid / 2) % ST, half = tid & 1;
-        const int ba = kPairs[p].y, bb = kPairs[p].x;   // block (row ba, column bb), bb > ba
-        *reinterpret_cast<uint4 *>(sm.aqk + umma_k128(C, ba * ST + rr, bb * ST + half * 8)) =
-            make_uint4(0u, 0u, 0u, 0u);
-    }
 
     // ---- P2: key-key and query-key blocks ----
     // warps 0-5: one off-diagonal sub-tile pair each (both products share the
@@ -377,19 +430,16 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 }
         }
         __syncwarp();
-        {   // lane -> (block a0 + lane/16, column j): solve (I + A_aa) x = e_j in fp32
+        {   // lane -> (block a0 + lane/16, column j): solve (I + A_aa) x = e_j in fp32,
+            // column by column (x_i is final when row i is reached; depth 16, not 120)
             const int a = a0 + (lane >> 4), j = lane & 15;
             float x[ST];
 #pragma unroll
-            for (int r = 0; r < ST; ++r) {
-                float sacc = (r == j) ? 1.f : 0.f;
-                if (r > j) {
+            for (int r = 0; r < ST; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-                    for (int i = 0; i < r; ++i)
-                        if (i >= j) sacc -= sm.u.akd[a][r][i] * x[i];
-                }
-                x[r] = sacc;
-            }
+            for (int i = 0; i < ST - 1; ++i)
+#pragma unroll
+                for (int r = i + 1; r < ST; ++r) x[r] = fmaf(-sm.u.akd[a][r][i], x[i], x[r]);
 #pragma unroll
             for (int r = 0; r < ST; ++r) sm.taa[a][r * (ST + 8) + j] = f2bf(x[r]);
         }
@@ -483,10 +533,11 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
             __syncwarp();
         }
-        bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 0));
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, mma_phase++ & 1));
         t5::fence_after_sync();
         // X is consumed: bring Kt (into xk) and Qg (into xv) back from the record's scratch
-        // area while [W|U] leaves tensor memory
+        // area while [W|U] leaves tensor memory; T' is consumed too: the next item's g
+        // rows 0-31 go to ka
 #pragma unroll
         for (int it = 0; it < 2 * C * D * 2 / 16 / 256; ++it) {
             const int i = tid + it * 256;                  // 16-byte chunk index
@@ -494,6 +545,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             cp_async16((m == 0 ? sm.xk : sm.xv) + off,
                        rec + (m == 0 ? REC_KT_SCRATCH : REC_QG_SCRATCH) + off);
         }
+        cp_async_commit();
+        if (has_next) load_g_half(nxt, 0);
         cp_async_commit();
         if (ok) {   // rows r = 16(w&3) + lane (lanes 0..15); warps 0-3 -> W, warps 4-7 -> U
             const int r = (warp & 3) * 16 + lane, cb = (warp >> 2) * D;
@@ -514,7 +567,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 }
             }
         }
-        cp_async_wait<0>();
+        cp_async_wait<1>();         // Kt and Qg (the next item's g may still be in flight)
         fence_proxy_async_smem();   // [W|U] (generic stores), Kt (cp.async) -> tensor core
         t5::fence_before_sync();
         ok = __syncthreads_and(ok) != 0;
@@ -532,8 +585,10 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
             __syncwarp();
         }
-        ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 1));
+        ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, mma_phase++ & 1));
         t5::fence_after_sync();
+        if (has_next) load_g_half(nxt, 1);   // Kt is consumed: g rows 32-63 to xk
+        cp_async_commit();
         if (ok) {   // lane = key row; warps 0-3 -> M' (columns 0..127), warps 4-7 -> R
             const int m = (warp & 3) * 32 + lane, cb = (warp >> 2) * D;
 #pragma unroll
@@ -569,8 +624,10 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
             __syncwarp();
         }
-        ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, 0));
+        ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, mma_phase++ & 1));
         t5::fence_after_sync();
+        if (has_next) load_kq(nxt);   // [W|U] is consumed: the next k and q to qa and kb
+        cp_async_commit();
         if (ok) {   // rows r = 16(w&3) + lane (lanes 0..15); warps 0-3 -> Q', warps 4-7 -> O0
             const int r = (warp & 3) * 16 + lane, cb = (warp >> 2) * D;
 #pragma unroll
@@ -605,12 +662,21 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 }
             }
         }
-        if (!ok && tid == 0) atomicOr(err_word, ERR_TIMEOUT_BIT);
         t5::fence_before_sync();
-        __syncthreads();
+        ok = __syncthreads_and(ok) != 0;   // Qg in xv is consumed
         t5::fence_after_sync();
-        if (warp == 0) t5::dealloc(tmem, 2 * D);
+        if (has_next) load_v_beta(nxt);
+        cp_async_commit();
     }
+    cur = nxt;
+    }   // item loop
+
+    if (!ok && tid == 0) atomicOr(err_word, ERR_TIMEOUT_BIT);
+    cp_async_wait<0>();   // nothing may land in shared memory after the CTA ends
+    t5::fence_before_sync();
+    __syncthreads();
+    t5::fence_after_sync();
+    if (warp == 0) t5::dealloc(*tmem_slot, 2 * D);
 }
 
 // ---------------------------------------------------------------------------
