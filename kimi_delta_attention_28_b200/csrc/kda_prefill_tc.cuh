@@ -228,7 +228,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                        ok ? 16 : 0);
         }
     };
-    auto load_kq = [&](const Item &it) {                 // k -> qa, q -> kb (swz128)
+    auto load_kq = [&](const Item &it) {                 // k -> qa, q -> kb (swz128), beta
 #pragma unroll
         for (int m = 0; m < 2 * C * (D / 8) / 256; ++m) {
             const int i = tid + m * 256, w = i / (C * (D / 8)), rem = i % (C * (D / 8));
@@ -238,19 +238,21 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             cp_async16((w ? sm.kb : sm.qa) + swz128(r, c8),
                        ok ? src + it.base + r * rowstride + c8 : src, ok ? 16 : 0);
         }
+        if (tid < C) {
+            const bool ok = tid < it.len;
+            cp_async4(&sm.beta[tid], ok ? beta + (size_t)(it.t0 + tid) * H + it.h : beta,
+                      ok ? 4 : 0);
+        }
     };
-    auto load_v_beta = [&](const Item &it) {             // V -> xv (umma_k128), beta
+    // V -> xv (umma_k128), in a cp.async group of its own: it is needed only by the
+    // [W|U] product, so an item starts without waiting for it
+    auto load_v = [&](const Item &it) {
 #pragma unroll
         for (int m = 0; m < C * (D / 8) / 256; ++m) {
             const int i = tid + m * 256, r = i / (D / 8), c8 = (i % (D / 8)) * 8;
             const bool ok = r < it.len;
             cp_async16(sm.xv + umma_k128(C, r, c8), ok ? v + it.base + r * rowstride + c8 : v,
                        ok ? 16 : 0);
-        }
-        if (tid < C) {
-            const bool ok = tid < it.len;
-            cp_async4(&sm.beta[tid], ok ? beta + (size_t)(it.t0 + tid) * H + it.h : beta,
-                      ok ? 4 : 0);
         }
     };
 
@@ -276,7 +278,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     load_g_half(cur, 0);
     load_g_half(cur, 1);
     load_kq(cur);
-    load_v_beta(cur);
+    cp_async_commit();
+    load_v(cur);
     cp_async_commit();
 
     for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
@@ -284,7 +287,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     const bool has_next = nxt_item < items;
     const Item nxt = locate(has_next ? nxt_item : item);
     uint8_t *rec = cur.rec;
-    cp_async_wait<0>();
+    cp_async_wait<1>();   // g, k, q, beta (V, the newest group, may still be in flight)
     __syncthreads();
 
     // ---- P1: cumulative decay and the scaled operands ----
@@ -514,7 +517,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     //   D1 = Kt^T [W|U]        (M = 128 key rows):         M' = -D1[:, :128], R = D1[:, 128:]
     //   D2 = Aqk  [W|U]        (M = 64 chunk rows):        Q' = Qg - D2[:, :128], O0 = D2[:, 128:]
     {
-        fence_proxy_async_smem();   // T' (generic stores) -> tensor core
+        cp_async_wait<0>();         // V
+        fence_proxy_async_smem();   // T' (generic stores), V -> tensor core
         t5::fence_before_sync();
         __syncthreads();
         const uint32_t tmem = *tmem_slot;
@@ -665,7 +669,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         t5::fence_before_sync();
         ok = __syncthreads_and(ok) != 0;   // Qg in xv is consumed
         t5::fence_after_sync();
-        if (has_next) load_v_beta(nxt);
+        if (has_next) load_v(nxt);
         cp_async_commit();
     }
     cur = nxt;
