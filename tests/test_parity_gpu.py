@@ -92,6 +92,13 @@ def test_varlen_small_with_empty_sequences(dtype, d):
     run_and_check(inp, dtype, "varlen small")
 
 
+@pytest.mark.parametrize("T", [64, 130])
+def test_many_chains_several_waves(T):
+    """512 (sequence, head) chains: the state pass runs in several waves of CTAs."""
+    inp = W.make_prefill_inputs(64, T, 8, 128, 128, torch.bfloat16, True, seed=T + 17, device=DEV)
+    run_and_check(inp, torch.bfloat16, f"512 chains T={T}")
+
+
 def test_varlen_workload_sampled_heads():
     """Packed varlen workload (16 sequences, H=32) on the GPU; the oracle checks
     every sequence on a sample of heads (heads are independent chains)."""
