@@ -261,6 +261,25 @@ KDA_DEVINL void ld64(uint32_t taddr, float (&v)[64]) {
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 16x256b shape, x4: lanes L..L+15 of this warp's quarter (L from taddr) and 32
+// columns.  Thread t (g = t/4, c = t%4) receives, for each 8-column group j (0..3),
+// v[4j], v[4j+1] = (lane L+g, columns 8j+2c, 8j+2c+1) and v[4j+2], v[4j+3] = the same
+// columns of lane L+g+8 -- the mma.sync accumulator layout; for an M = 64 accumulator
+// (rows 16w..16w+15 in lanes 32w..32w+15) every thread of the warp gets data.
+KDA_DEVINL void ld16x256b_x4(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15}, [%16];\n"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 template <int N>
 KDA_DEVINL void ld_cols(uint32_t taddr, float (&v)[N]) {
     if constexpr (N == 32) ld32(taddr, v);

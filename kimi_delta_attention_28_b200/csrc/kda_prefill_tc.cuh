@@ -552,22 +552,19 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         cp_async_commit();
         if (has_next) load_g_half(nxt, 0);
         cp_async_commit();
-        if (ok) {   // rows r = 16(w&3) + lane (lanes 0..15); warps 0-3 -> W, warps 4-7 -> U
-            const int r = (warp & 3) * 16 + lane, cb = (warp >> 2) * D;
+        if (ok) {   // M = 64 accumulator: rows 16(w&3)..+15; warps 0-3 -> W, warps 4-7 -> U
+            const int r0 = (warp & 3) * 16 + gid, cb = (warp >> 2) * D;
 #pragma unroll
             for (int qq = 0; qq < D / 32; ++qq) {
-                float vv[32];
-                t5::ld32(tmem + lane_base + cb + qq * 32, vv);
-                if (lane < 16) {
+                float vv[16];
+                t5::ld16x256b_x4(tmem + lane_base + cb + qq * 32, vv);
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint4 pk;
-                        pk.x = pack_bf16x2(vv[c8 * 8 + 0], vv[c8 * 8 + 1]);
-                        pk.y = pack_bf16x2(vv[c8 * 8 + 2], vv[c8 * 8 + 3]);
-                        pk.z = pack_bf16x2(vv[c8 * 8 + 4], vv[c8 * 8 + 5]);
-                        pk.w = pack_bf16x2(vv[c8 * 8 + 6], vv[c8 * 8 + 7]);
-                        *reinterpret_cast<uint4 *>(sm.qa + umma_k128(C, r, cb + qq * 32 + c8 * 8)) = pk;
-                    }
+                for (int j8 = 0; j8 < 4; ++j8) {
+                    const int c = cb + qq * 32 + j8 * 8 + 2 * tig;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        *reinterpret_cast<uint32_t *>(sm.qa + umma_k128(C, r0 + 8 * hh, c)) =
+                            pack_bf16x2(vv[4 * j8 + 2 * hh], vv[4 * j8 + 2 * hh + 1]);
                 }
             }
         }
@@ -632,36 +629,27 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         t5::fence_after_sync();
         if (has_next) load_kq(nxt);   // [W|U] is consumed: the next k and q to qa and kb
         cp_async_commit();
-        if (ok) {   // rows r = 16(w&3) + lane (lanes 0..15); warps 0-3 -> Q', warps 4-7 -> O0
-            const int r = (warp & 3) * 16 + lane, cb = (warp >> 2) * D;
+        if (ok) {   // M = 64 accumulator: rows 16(w&3)..+15; warps 0-3 -> Q', warps 4-7 -> O0
+            const int r0 = (warp & 3) * 16 + gid, cb = (warp >> 2) * D;
+            uint8_t *dst0 = rec + (warp < 4 ? REC_QP : REC_O0);
 #pragma unroll
             for (int qq = 0; qq < D / 32; ++qq) {
-                float vv[32];
-                t5::ld32(tmem + lane_base + cb + qq * 32, vv);
-                if (lane < 16) {
+                float vv[16];
+                t5::ld16x256b_x4(tmem + lane_base + cb + qq * 32, vv);
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        const int c = qq * 32 + c8 * 8;
-                        float x[8];
+                for (int j8 = 0; j8 < 4; ++j8) {
+                    const int c = qq * 32 + j8 * 8 + 2 * tig;   // column within Q' / O0
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) x[e] = vv[c8 * 8 + e];
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int r = r0 + 8 * hh;
+                        float x0 = vv[4 * j8 + 2 * hh], x1 = vv[4 * j8 + 2 * hh + 1];
                         if (warp < 4) {   // Q' = Qg - Aqk W
-                            const uint4 qg = *reinterpret_cast<const uint4 *>(sm.xv + swz128(r, c));
-                            const uint32_t u[4] = {qg.x, qg.y, qg.z, qg.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 f = unpack_bf16x2(u[e]);
-                                x[2 * e] = f.x - x[2 * e];
-                                x[2 * e + 1] = f.y - x[2 * e + 1];
-                            }
+                            const float2 f = unpack_bf16x2(
+                                *reinterpret_cast<const uint32_t *>(sm.xv + swz128(r, c)));
+                            x0 = f.x - x0;
+                            x1 = f.y - x1;
                         }
-                        uint4 pk;
-                        pk.x = pack_bf16x2(x[0], x[1]);
-                        pk.y = pack_bf16x2(x[2], x[3]);
-                        pk.z = pack_bf16x2(x[4], x[5]);
-                        pk.w = pack_bf16x2(x[6], x[7]);
-                        uint8_t *dst = rec + (warp < 4 ? REC_QP : REC_O0) + core_off(C, r, c);
-                        *reinterpret_cast<uint4 *>(dst) = pk;
+                        *reinterpret_cast<uint32_t *>(dst0 + core_off(C, r, c)) = pack_bf16x2(x0, x1);
                     }
                 }
             }
