@@ -118,6 +118,17 @@ def dist_setup(args):
     return world, rank, local
 
 
+def max_over_ranks(x, world, device):
+    """The maximum of a per-rank float over all ranks (the job's time is its slowest
+    rank's); a no-op for one rank."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def workload_inputs(name, device, seed_offset=0):
     from kimi_delta_attention_28_b200 import workloads as W
     w = {"prefill": W.PREFILL, "long": W.LONG, "varlen": W.VARLEN}[name]
@@ -221,10 +232,7 @@ def run_ours(args, world, rank, local):
     intra = [e[0].elapsed_time(e[1]) for e in split]
     inter = [e[1].elapsed_time(e[2]) for e in split]
     launches_per_step = (2 if cu is not None else 1) + 1
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
     A = algorithmic(w, inp)
 
@@ -263,10 +271,7 @@ def run_ours(args, world, rank, local):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, world, dev)
         e2e = {"value": world * A["ntok"] / (e2e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms}
@@ -355,10 +360,7 @@ def run_ours_decode(args, world, rank, local):
         torch.distributed.barrier()
     clocks.stop()
     total_ms = ev[0].elapsed_time(ev[-1])
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     if rank != 0:
         return None
     ms = total_ms / args.steps
