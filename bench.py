@@ -131,7 +131,8 @@ def max_over_ranks(x, world, device):
 
 def workload_inputs(name, device, seed_offset=0):
     from kimi_delta_attention_28_b200 import workloads as W
-    w = {"prefill": W.PREFILL, "long": W.LONG, "varlen": W.VARLEN}[name]
+    w = {"prefill": W.PREFILL, "long": W.LONG, "varlen": W.VARLEN,
+         "few_chains": W.FEW_CHAINS}[name]
     import dataclasses
     w = dataclasses.replace(w, seed=w.seed + seed_offset)
     return w, W.make_workload(w, device)
@@ -231,7 +232,8 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     intra = [e[0].elapsed_time(e[1]) for e in split]
     inter = [e[1].elapsed_time(e[2]) for e in split]
-    launches_per_step = (2 if cu is not None else 1) + 1
+    nseg = kda.plan_segments(B, T, H, dk, dv, nseq, w.dtype)
+    launches_per_step = (2 if cu is not None else 1) + (1 if nseg <= 1 else 3)
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
     A = algorithmic(w, inp)
@@ -308,7 +310,9 @@ def run_ours(args, world, rank, local):
                  "hbm_frac": path_gbs / hbm_peak,
                  "tflops_recurrence": A["flops"] / (ms_per_step * 1e-3) / 1e12,
                  "tensor_frac": A["flops"] / (ms_per_step * 1e-3) / 1e12 / tf_peak},
-        "kernels_ms": {"kda_tc_prep_kernel": intra_ms, "kda_tc_state_kernel": inter_ms},
+        "kernels_ms": {"kda_tc_prep_kernel": intra_ms,
+                       ("kda_tc_state_kernel" if nseg <= 1 else
+                        f"state pass split in {nseg} segments (map, combine, output)"): inter_ms},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(t_wall0, t_wall1),
         "e2e": e2e,
@@ -465,7 +469,8 @@ def run_reference(args, world, rank):
     import torch
     import oracle
     from kimi_delta_attention_28_b200 import workloads as W
-    w = {"prefill": W.PREFILL, "long": W.LONG, "varlen": W.VARLEN}[args.workload]
+    w = {"prefill": W.PREFILL, "long": W.LONG, "varlen": W.VARLEN,
+         "few_chains": W.FEW_CHAINS}[args.workload]
     inp = W.make_workload(w, "cpu")
     h = host_f64(inp)
     B, T, H, dk = h["q"].shape
@@ -516,7 +521,7 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "long", "varlen", "decode"],
+    ap.add_argument("--workload", choices=["prefill", "long", "varlen", "decode", "few_chains"],
                     default="prefill")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

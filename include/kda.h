@@ -162,6 +162,9 @@ kda_status kda_fwd_inter(const float *h0, const int32_t *cu_seqlens, int num_seq
  */
 size_t kda_fwd_segmented_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
                                         int dtype, int num_segments);
+/* The number of time segments kda_fwd chooses for these sizes on the current
+ * device (1: no split; 0: invalid or unsupported sizes, or no device). */
+int kda_fwd_plan_segments(int B, int T, int H, int dk, int dv, int num_seqs, int dtype);
 kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const float *g,
                              const float *beta, const float *h0, const int32_t *cu_seqlens,
                              int num_seqs, int B, int T, int H, int dk, int dv, int dtype,

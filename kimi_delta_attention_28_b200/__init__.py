@@ -15,8 +15,9 @@ This package is the thin Python binding; ``include/kda.h`` is the interface.
 """
 from ._lib import (KDAError, device_error, kda_decode_step, kda_fwd,  # noqa: F401
                    kda_fwd_inter, kda_fwd_intra, kda_fwd_noalloc, kda_fwd_segmented,
-                   load_library, segmented_workspace_size, workspace_size)
+                   load_library, plan_segments, segmented_workspace_size, workspace_size)
 
 __all__ = ["kda_fwd", "kda_fwd_intra", "kda_fwd_inter", "kda_fwd_noalloc", "kda_fwd_segmented",
-           "kda_decode_step", "workspace_size", "segmented_workspace_size", "device_error",
+           "kda_decode_step", "workspace_size", "segmented_workspace_size", "plan_segments",
+           "device_error",
            "load_library", "KDAError"]

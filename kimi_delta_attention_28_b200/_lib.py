@@ -42,6 +42,7 @@ SIGNATURES = {
     "kda_fwd_noalloc": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP,
                          _VP], _I),
     "kda_fwd_segmented_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I], _SZ),
+    "kda_fwd_plan_segments": ([_I, _I, _I, _I, _I, _I, _I], _I),
     "kda_fwd_segmented": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I,
                            _VP, _VP, _VP, _SZ, _VP], _I),
 }
@@ -158,6 +159,13 @@ def segmented_workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_seqs:
                              dtype: torch.dtype, num_segments: int) -> int:
     return int(load_library().kda_fwd_segmented_workspace_size(
         B, T, H, dk, dv, num_seqs, _dtype_code(dtype), num_segments))
+
+
+def plan_segments(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
+                  dtype: torch.dtype) -> int:
+    """Time segments kda_fwd uses for these sizes on the current device (1: none)."""
+    return int(load_library().kda_fwd_plan_segments(B, T, H, dk, dv, num_seqs,
+                                                    _dtype_code(dtype)))
 
 
 def kda_fwd_segmented(q, k, v, g, beta, h0=None, cu_seqlens=None, *, num_segments: int,

@@ -399,6 +399,13 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                                         cu_seqlens, s);
 }
 
+int kda_fwd_plan_segments(int B, int T, int H, int dk, int dv, int num_seqs, int dtype) {
+    if (B < 0 || T < 0 || num_seqs < 0) return 0;
+    if (check_shape(H, dk, dv, dtype) != KDA_OK) return 0;
+    if (num_seqs > 0 && B != 1) return 0;
+    return ws_layout(B, T, H, dk, num_seqs, dtype, 0, device_sms()).nseg;
+}
+
 size_t kda_fwd_segmented_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
                                         int dtype, int num_segments) {
     if (B < 0 || T < 0 || num_seqs < 0) return 0;

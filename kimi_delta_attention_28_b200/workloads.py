@@ -58,7 +58,12 @@ DECODE = Workload("decode_bf16_N256_H96_d128", B=256, H=96, T=1, dk=128, dv=128,
                   dtype=torch.bfloat16, h0=True, decode_steps=1000, seed=1004,
                   note="one token per sequence per step, fp32 state updated in place")
 
-ALL = (TINY, PREFILL, LONG, VARLEN, DECODE)
+FEW_CHAINS = Workload("few_chains_bf16_B1_H2_T262144_d128", B=1, H=2, T=1 << 18, dk=128,
+                      dv=128, dtype=torch.bfloat16, h0=True, seed=1005,
+                      note="two (sequence, head) chains of 4,096 chunks: too few to fill "
+                           "the GPU, so the state pass is split in time")
+
+ALL = (TINY, PREFILL, LONG, VARLEN, DECODE, FEW_CHAINS)
 BY_NAME = {w.name: w for w in ALL}
 
 

@@ -68,6 +68,14 @@ def test_workspace_size(lib):
     assert 0 < ws(1, 64, 4, 32, 32, 0, F32) < 4096       # CUDA-core path: header only
 
 
+def test_plan_segments_validates(lib):
+    plan = lib.kda_fwd_plan_segments
+    assert plan(1, 65536, 1, 128, 128, 0, BF16) >= 1     # 1 without a device
+    assert plan(2, 4096, 8, 64, 64, 0, F32) == 1           # CUDA-core path never splits
+    assert plan(2, 100, 4, 128, 64, 0, BF16) == 0          # d_k != d_v
+    assert plan(2, 100, 4, 128, 128, 3, BF16) == 0         # packed needs B == 1
+
+
 def test_segmented_workspace_size(lib):
     seg = lib.kda_fwd_segmented_workspace_size
     ws = lib.kda_fwd_workspace_size

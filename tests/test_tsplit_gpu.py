@@ -103,6 +103,8 @@ def test_auto_policy_splits_few_long_chains():
     CTAs; kda_fwd splits it by itself.  The workspace it asks for includes the
     split's buffers, and the result matches the oracle and the explicit split."""
     B, T, H = 1, 16384, 1
+    assert kda.plan_segments(B, T, H, 128, 128, 0, BF16) > 1
+    assert kda.plan_segments(2, 4096, 8, 128, 128, 0, BF16) == 1   # 16 chains fill the GPU
     plain = kda.segmented_workspace_size(B, T, H, 128, 128, 0, BF16, 1)
     auto = kda.workspace_size(B, T, H, 128, 128, 0, BF16)
     assert auto > plain   # room for the split
