@@ -266,3 +266,23 @@ def test_extreme_decay_at_the_bound():
     inp["g"] = -5.0 + 1e-3 * torch.rand_like(inp["g"])
     o, hT = run_and_check(inp, torch.bfloat16, "g at bound")
     assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
+
+
+@pytest.mark.parametrize("case", ["no_decay", "no_write", "full_write", "mixed_decay"])
+def test_special_inputs_tensor_core_path(case):
+    """Corner values of the gates over 4,096 tokens (64 chunks, several record
+    rings' worth): g = 0 (nothing forgets, the state carries everything), beta = 0
+    (pure decay of h0, no writes), beta = 1 (full delta-rule overwrite), and
+    channels that never decay next to channels at the decay bound."""
+    inp = W.make_prefill_inputs(1, 4096, 2, 128, 128, torch.bfloat16, True, seed=12, device=DEV)
+    if case == "no_decay":
+        inp["g"].zero_()
+    elif case == "no_write":
+        inp["beta"].zero_()
+    elif case == "full_write":
+        inp["beta"].fill_(1.0)
+    else:
+        inp["g"][..., 0::2] = 0.0
+        inp["g"][..., 1::2] = -5.0
+    o, hT = run_and_check(inp, torch.bfloat16, case)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
