@@ -55,10 +55,15 @@ KDA_DEVINL void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                  : "r"(addr));
 }
 
-KDA_DEVINL void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
-                 : "=r"(r[0]), "=r"(r[1])
-                 : "r"(addr));
+
+// Four 8x8 bf16 tiles from registers to shared memory, each stored transposed:
+// lanes 8m..8m+7 give the row addresses of tile m (register m), and thread t's pair
+// (row t/4, columns 2(t%4), 2(t%4)+1) of the tile lands in rows 2(t%4), 2(t%4)+1,
+// column t/4.
+KDA_DEVINL void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};\n"
+                 ::"r"(addr), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
 }
 
 // 2^x by the PTX instruction ex2.approx.ftz.f32 (relative error about 2^-22;

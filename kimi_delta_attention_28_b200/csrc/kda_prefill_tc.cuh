@@ -142,7 +142,6 @@ __global__ void __launch_bounds__(1024) kda_chunk_map_kernel(const int *__restri
 // the tiles those phases have just released.
 // ---------------------------------------------------------------------------
 constexpr int LDA = C + 8;      // padded bf16 row stride of the 64x64 blocks (144 B)
-constexpr int ZLD = 24;         // row stride of the per-warp 16x8 scratch (48 B: conflict-free)
 
 // The six sub-tile pairs (a, b), b < a, of a 64-token chunk.
 __constant__ int2 kPairs[6] = {{1, 0}, {2, 0}, {3, 0}, {2, 1}, {3, 1}, {3, 2}};
@@ -151,7 +150,7 @@ struct PrepSmem {
     // Five 16 KB tiles, reused across phases (an item's inputs arrive as: g rows 0-31
     // in ka and rows 32-63 in xk, 512-byte rows; k in qa, q in kb (swz128); V in xv):
     //   ka: g (rows 0-31); k*exp(G_r - G_ref(a)) (swz128); then T' = (I + A)^-1 Diag(b)
-    //       (first 8 KB, umma_k128) and the per-warp scratch of its substitution
+    //       (first 8 KB, umma_k128)
     //   qa: raw k; q*exp(G_r - G_ref(a)) (swz128); then, with kb, [W|U] (four umma_k128
     //       planes)
     //   kb: raw q; k*exp(G_ref(b) - G_i) (swz128)
@@ -461,54 +460,61 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     __syncthreads();
 
-    // ---- P3: T' = (I + A)^-1 Diag(b) by blocked forward substitution ----
+    // ---- P3: T' = (I + A)^-1 Diag(b) by blocked forward substitution, transposed ----
     // (I + A) T' = Diag(b), solved per 16-row block a:
     //   T'_a = (I + A_aa)^-1 (Diag(b)_a - sum_{c<a} A_ac T'_c).
-    // Warp w owns columns 8w..8w+7 (inside column block w/2, above which T' is zero);
-    // each step is two m16n8k16 products and a 16x8 hop through shared memory.
-    {
-        uint8_t *Tp = sm.ka;
-        const uint32_t s_tp = s_ka;
-        __nv_bfloat16 *Z = reinterpret_cast<__nv_bfloat16 *>(sm.ka + C * C * 2) + warp * (ST * ZLD);
-        const int b = warp >> 1, i0 = warp * 8;
-        for (int a = 0; a < b; ++a)
+    // Warp b (b < 4) owns columns 16b..16b+15 (above row block b, T' is zero) and works
+    // with the transposes X_a = (T'_a restricted to them)^T: X_a = Z^T (I + A_aa)^-T with
+    // Z^T = sum_c X_c (-A_ac)^T.  Every product's accumulator is, repacked to bf16, the
+    // A operand of the next one, so the whole chain stays in registers; each X_a is
+    // written to T' with transposing matrix stores.
+    if (warp < NST) {
+        const int b = warp;
+        const uint32_t s_tp = s_ka;   // T' (umma_k128 plane, 64 x 64 bf16)
+        for (int a = 0; a < b; ++a)   // row blocks above b: zero
+            *reinterpret_cast<uint4 *>(sm.ka + umma_k128(C, a * ST + (lane >> 1), b * ST + 8 * (lane & 1))) =
+                make_uint4(0u, 0u, 0u, 0u);
+        uint32_t X[NST][4];           // bf16 A fragments of X_c, c = b .. a-1
+        const int brow = (lane & 7) + 8 * (lane >> 4), bcol = 8 * ((lane >> 3) & 1);   // x4 B tiles
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint32_t *>(Tp + umma_k128(C, a * ST + gid + 8 * hh, i0 + 2 * tig)) = 0u;
-        for (int a = b; a < NST; ++a) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            if (a == b) {
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int r = a * ST + gid + 8 * hh, i = i0 + 2 * tig + e;
-                        acc[2 * hh + e] = (r == i) ? sm.beta[i] : 0.f;
-                    }
+        for (int a = 0; a < NST; ++a) {
+            if (a < b) continue;
+            uint32_t za[4];
+            if (a == b) {   // Z^T = Diag(b) on the block: diagonal entries only
+                const float* bt = sm.beta + b * ST + 2 * tig;
+                za[0] = pack_bf16x2(gid == 2 * tig ? bt[0] : 0.f, gid == 2 * tig + 1 ? bt[1] : 0.f);
+                za[1] = 0u;
+                za[2] = 0u;
+                za[3] = pack_bf16x2(gid == 2 * tig ? bt[8] : 0.f, gid == 2 * tig + 1 ? bt[9] : 0.f);
             } else {
-                for (int c = b; c < a; ++c) {   // acc += (-A_ac) T'_c   (akkn holds -A)
-                    uint32_t af[4], bf[2];
-                    ldsm_x4(af, smem_u32(sm.akkn + (a * ST + frag_a_row(lane)) * LDA + c * ST +
-                                         frag_a_col(lane)));
-                    ldsm_x2_t(bf, s_tp + umma_k128(C, c * ST + (lane & 15), i0));
-                    mma_bf16_16816(acc, af, bf[0], bf[1]);
+                float z[2][4] = {};
+#pragma unroll
+                for (int c = 0; c < NST; ++c) {
+                    if (c < b || c >= a) continue;
+                    uint32_t bf[4];   // (-A_ac)^T: akkn rows of block a, columns of block c
+                    ldsm_x4(bf, smem_u32(sm.akkn + (a * ST + brow) * LDA + c * ST + bcol));
+                    mma_bf16_16816(z[0], X[c], bf[0], bf[1]);
+                    mma_bf16_16816(z[1], X[c], bf[2], bf[3]);
                 }
+                za[0] = pack_bf16x2(z[0][0], z[0][1]);
+                za[1] = pack_bf16x2(z[0][2], z[0][3]);
+                za[2] = pack_bf16x2(z[1][0], z[1][1]);
+                za[3] = pack_bf16x2(z[1][2], z[1][3]);
             }
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint32_t *>(Z + (gid + 8 * hh) * ZLD + 2 * tig) =
-                    pack_bf16x2(acc[2 * hh], acc[2 * hh + 1]);
-            __syncwarp();
-            uint32_t at[4], bz[2];
-            ldsm_x4(at, smem_u32(sm.taa[a] + frag_a_row(lane) * (ST + 8) + frag_a_col(lane)));
-            ldsm_x2_t(bz, smem_u32(Z + (lane & 15) * ZLD));
-            float y[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_bf16_16816(y, at, bz[0], bz[1]);
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                *reinterpret_cast<uint32_t *>(Tp + umma_k128(C, a * ST + gid + 8 * hh, i0 + 2 * tig)) =
-                    pack_bf16x2(y[2 * hh], y[2 * hh + 1]);
-            __syncwarp();
+            uint32_t tb[4];   // (I + A_aa)^-T
+            ldsm_x4(tb, smem_u32(sm.taa[a] + brow * (ST + 8) + bcol));
+            float x[2][4] = {};
+            mma_bf16_16816(x[0], za, tb[0], tb[1]);
+            mma_bf16_16816(x[1], za, tb[2], tb[3]);
+            X[a][0] = pack_bf16x2(x[0][0], x[0][1]);
+            X[a][1] = pack_bf16x2(x[0][2], x[0][3]);
+            X[a][2] = pack_bf16x2(x[1][0], x[1][1]);
+            X[a][3] = pack_bf16x2(x[1][2], x[1][3]);
+            // T' rows 16a..16a+15, columns 16b..16b+15 = X_a^T; tile m = (column half m&1,
+            // row half m>>1)
+            const int m = lane >> 3;
+            stsm_x4_t(s_tp + umma_k128(C, a * ST + 8 * (m >> 1) + (lane & 7), b * ST + 8 * (m & 1)),
+                      X[a][0], X[a][1], X[a][2], X[a][3]);
         }
     }
 
