@@ -184,7 +184,7 @@ kda_status launch_state(kda::tc::StateArgs a, long long units, cudaStream_t s) {
     a.debug_drop_first_copy = debug_drop_first_copy();
     const long long grid = units * ((a.mode == kStateMap ? 2 * D : D) / DVT);
     if (grid > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
-    kern<<<(unsigned)grid, 320, smem, s>>>(a);
+    kern<<<(unsigned)grid, StateRoles<DVT>::THREADS, smem, s>>>(a);
     return launch_status();
 }
 
@@ -316,7 +316,14 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
     a.nseg = L.nseg;
     a.mode = kStateOutput;
     const long long chains = (long long)N * H;
-    if (L.nseg <= 1) return launch_state<32>(a, chains, s);
+    if (L.nseg <= 1) {
+        // 32-column slices give the shortest per-chunk latency (they suit few chains);
+        // with more than two waves of them the pass is throughput-bound and 64-column
+        // slices (half the CTAs, each chunk's map read once per two slices) are faster
+        const int sms = device_sms();
+        if (chains * (D / 32) > 2LL * (sms > 0 ? sms : 148)) return launch_state<64>(a, chains, s);
+        return launch_state<32>(a, chains, s);
+    }
     // T-split: segment maps, the sequential combine, then the output pass from
     // each segment's true starting state.
     float *s_in = reinterpret_cast<float *>(ws + L.s_in);

@@ -679,7 +679,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 
 // ---------------------------------------------------------------------------
 // Kernel 2: inter-chunk state pass on tcgen05, warp-specialised.
-// grid = units * tiles CTAs of 320 threads (10 warps).  A unit is one (sequence,
+// grid = units * tiles CTAs of 32 (NSW + 6) threads.  A unit is one (sequence,
 // head) chain, or with a T-split one of its nseg consecutive segments (equal
 // numbers of chunks, the last may be shorter or empty); tiles = D / DVT column
 // slices of the state.  Roles:
@@ -755,9 +755,20 @@ struct T5Layout {
     static_assert(BYTES <= 232448, "shared memory budget");
 };
 
+// Warp roles of the state pass: NSW = 4 DVT/32 state warps (warp w: key row
+// 32 (w % 4) + lane, columns 32 (w / 4) .. + 31 of the slice), then the MMA warp, four
+// output warps and the producer warp.
 template <int DVT>
-__global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a) {
+struct StateRoles {
+    static constexpr int NSW = 4 * (DVT / 32);
+    static constexpr int MMA_WARP = NSW, OUT_WARP0 = NSW + 1, PROD_WARP = NSW + 5;
+    static constexpr int THREADS = 32 * (NSW + 6);
+};
+
+template <int DVT>
+__global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kernel(const StateArgs a) {
     using L = T5Layout<DVT>;
+    using RL = StateRoles<DVT>;
     const uint8_t *__restrict__ recs = a.recs;
     __nv_bfloat16 *__restrict__ o = a.o;
     const int H = a.H;
@@ -810,12 +821,12 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
     int *err_word = a.err_word;
 
     if (tid == 0) {
-        for (int s = 0; s < NA; ++s) { mbar_init(&full_a[s], 1); mbar_init(&a_free[s], 128); }
+        for (int s = 0; s < NA; ++s) { mbar_init(&full_a[s], 1); mbar_init(&a_free[s], 32 * RL::NSW); }
         for (int s = 0; s < NB; ++s) { mbar_init(&full_b[s], 1); mbar_init(&b_free[s], 128); }
         mbar_init(done_s, 1);
         mbar_init(&done_o[0], 1);
         mbar_init(&done_o[1], 1);
-        for (int w = 0; w < 4; ++w) mbar_init(&sb_full[w], 32);
+        for (int w = 0; w < 4; ++w) mbar_init(&sb_full[w], 32 * (DVT / 32));
         mbar_init(&do_free[0], 128);
         mbar_init(&do_free[1], 128);
         *abort_flag = 0;
@@ -839,17 +850,18 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
     };
     auto rec_of = [&](int j) { return recs + ((size_t)(c_begin + j) * H + h) * REC_BYTES; };
 
-    if (warp < 4) {
+    if (warp < RL::NSW) {
         // ---------------- state warps ----------------
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        float S[DVT];
-        const size_t row_off = (size_t)tid * D + col0;
+        const int row = (warp & 3) * 32 + lane, cb = (warp >> 2) * 32;   // key row, columns cb..cb+31
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        float S[32];
+        const size_t row_off = (size_t)row * D + col0 + cb;
         const float *init = nullptr;
         if (!map_mode)
             init = a.s_in ? a.s_in + (size_t)unit * D * D + row_off
                           : (a.h0 ? a.h0 + (size_t)chain * D * D + row_off : nullptr);
 #pragma unroll
-        for (int i = 0; i < DVT; i += 4) {
+        for (int i = 0; i < 32; i += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (init) x = *reinterpret_cast<const float4 *>(init + i);
             S[i] = x.x;
@@ -857,23 +869,23 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
             S[i + 2] = x.z;
             S[i + 3] = x.w;
         }
-        if (p_half) {   // identity columns col0 .. col0 + DVT - 1
+        if (p_half) {   // identity columns col0 + cb ..
 #pragma unroll
-            for (int i = 0; i < DVT; ++i) S[i] = (tid == col0 + i) ? 1.f : 0.f;
+            for (int i = 0; i < 32; ++i) S[i] = (row == col0 + cb + i) ? 1.f : 0.f;
         }
-        auto write_sb = [&](int buf) {   // bf16 copy of row tid, then signal it
+        auto write_sb = [&](int buf) {   // bf16 copy of this thread's part of its row, then signal
             uint8_t *sb = sm + L::OFF_SB + buf * L::SB_BYTES;
 #pragma unroll
-            for (int c8 = 0; c8 < DVT; c8 += 8) {
+            for (int c8 = 0; c8 < 32; c8 += 8) {
                 uint4 pk;
                 pk.x = pack_bf16x2(S[c8], S[c8 + 1]);
                 pk.y = pack_bf16x2(S[c8 + 2], S[c8 + 3]);
                 pk.z = pack_bf16x2(S[c8 + 4], S[c8 + 5]);
                 pk.w = pack_bf16x2(S[c8 + 6], S[c8 + 7]);
-                *reinterpret_cast<uint4 *>(sb + L::sb_off(tid, c8)) = pk;
+                *reinterpret_cast<uint4 *>(sb + L::sb_off(row, cb + c8)) = pk;
             }
             fence_proxy_async_smem();   // generic writes -> tensor-core reads
-            mbar_arrive(&sb_full[warp]);   // this warp's K slab of the next products
+            mbar_arrive(&sb_full[warp & 3]);   // key rows 32(w%4).. : K slab w%4 of the next products
         };
         write_sb(0);
         int j = 0;
@@ -881,22 +893,22 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
             const int sa = j % NA;
             const uint8_t *st = sm + sa * L::A_BYTES;
             bool ok = mbar_wait_bounded(&full_a[sa], (j / NA) & 1);
-            const float gam = reinterpret_cast<const float *>(st + L::A_GC)[tid];
-            uint4 rv[DVT / 8];
+            const float gam = reinterpret_cast<const float *>(st + L::A_GC)[row];
+            uint4 rv[4];
 #pragma unroll
-            for (int i = 0; i < DVT / 8; ++i)   // row tid of the R slice (zero for P)
+            for (int i = 0; i < 4; ++i)   // this thread's part of R row `row` (zero for P)
                 rv[i] = p_half ? make_uint4(0u, 0u, 0u, 0u)
-                               : *reinterpret_cast<const uint4 *>(st + L::A_R + core_off(D, tid, 8 * i));
+                               : *reinterpret_cast<const uint4 *>(st + L::A_R + core_off(D, row, cb + 8 * i));
             // the tensor-memory load below is warp-collective: decide as a warp
             ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(done_s, j & 1));
             if (!ok) { fail(); break; }
             t5::fence_after_sync();
-            float v[DVT];
-            t5::ld_cols<DVT>(tmem + lane_base, v);
+            float v[32];
+            t5::ld32(tmem + lane_base + cb, v);
             t5::fence_before_sync();
             mbar_arrive(&a_free[sa]);   // this thread is done with the slot and with D_S
 #pragma unroll
-            for (int i = 0; i < DVT / 8; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 const uint32_t u[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -910,15 +922,15 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
         }
         float *dst = nullptr;
         if (map_mode)
-            dst = a.seg_map + ((size_t)unit * D + tid) * (2 * D) + tile * DVT;
+            dst = a.seg_map + ((size_t)unit * D + row) * (2 * D) + tile * DVT + cb;
         else if (a.hT && seg == a.nseg - 1)
             dst = a.hT + (size_t)chain * D * D + row_off;
         if (!*abort_flag && dst && j == nchunks) {
 #pragma unroll
-            for (int i = 0; i < DVT; i += 4)
+            for (int i = 0; i < 32; i += 4)
                 *reinterpret_cast<float4 *>(dst + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
         }
-    } else if (warp == 4) {
+    } else if (warp == RL::MMA_WARP) {
         // ---------------- MMA warp ----------------
         constexpr uint32_t idS = t5::idesc_bf16(128, DVT, 0, 1);
         constexpr uint32_t idO = t5::idesc_bf16(64, DVT, 0, 1);
@@ -970,7 +982,7 @@ __global__ void __launch_bounds__(320, 1) kda_tc_state_kernel(const StateArgs a)
             }
             if (__any_sync(0xffffffffu, !slab_ok)) { fail(); break; }
         }
-    } else if (warp < 9) {
+    } else if (warp < RL::PROD_WARP) {
         // ---------------- output warps (none in the map pass) ----------------
         const int q = warp & 3;                          // tensor-memory lane quarter
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;

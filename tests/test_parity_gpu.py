@@ -94,7 +94,8 @@ def test_varlen_small_with_empty_sequences(dtype, d):
 
 @pytest.mark.parametrize("T", [64, 130])
 def test_many_chains_several_waves(T):
-    """512 (sequence, head) chains: the state pass runs in several waves of CTAs."""
+    """512 (sequence, head) chains: more than two waves of 32-column state slices,
+    so the state pass runs on 64-column slices (eight state warps per CTA)."""
     inp = W.make_prefill_inputs(64, T, 8, 128, 128, torch.bfloat16, True, seed=T + 17, device=DEV)
     run_and_check(inp, torch.bfloat16, f"512 chains T={T}")
 
