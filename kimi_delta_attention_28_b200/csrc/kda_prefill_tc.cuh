@@ -11,16 +11,18 @@
 //   O     = (Q * exp G) S_in + [i <= r](sum_c q_rc k_ic exp(G_rc - G_ic)) Delta
 //   S_out = Diag(exp G_C) S_in + (K * exp(G_C - G))^T Delta
 //
-// Kernel 1 (kda_tc_prep_kernel) computes every chunk-local quantity, fully in
-// parallel over (chunk, head): the log-decay cumsum; the key-key and query-key
-// blocks with the pairwise decays factored through 16-token sub-tile reference
-// rows so no factor overflows (the same page's panel "g ∈ (-5, 0)" bounds a
-// 16-token decay by e^-80); [W|U] by blocked forward substitution (fp32 inverses
-// of the 16x16 diagonal blocks, tensor-core products elsewhere); and from them
-// the chunk's affine map on the state (below), one record per (chunk, head).
+// Kernel 1 (kda_tc_prep_kernel) computes every chunk-local quantity, in parallel
+// over (chunk, head) items (persistent CTAs that load the next item while finishing
+// the current one): the log-decay cumsum; the key-key and query-key blocks with the
+// pairwise decays factored through 16-token sub-tile reference rows so no factor
+// overflows (the same page's panel "g ∈ (-5, 0)" bounds a 16-token decay by e^-80);
+// T' = (I + A)^-1 Diag(b) by blocked forward substitution (fp32 inverses of the
+// 16x16 diagonal blocks, warp-level tensor-core products elsewhere); [W|U] = T' [K *
+// exp G | V] and from it the chunk's affine map on the state (below) on tcgen05,
+// one record per (chunk, head).
 // Kernel 2 (kda_tc_state_kernel) walks the chunks of each (sequence, head) in
-// order with the fp32 state on chip, split over 32-column slices of the state
-// (state columns evolve independently).  Its warps are specialised (state
+// order with the fp32 state on chip, split over 32- or 64-column slices of the
+// state (state columns evolve independently).  Its warps are specialised (state
 // update, tcgen05 issue, output, bulk-copy producer) and hand off through
 // mbarriers, so the loop-carried path per chunk is one tcgen05 product plus the
 // register update of the state; the outputs and copies run beside it.
@@ -683,17 +685,18 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 // head) chain, or with a T-split one of its nseg consecutive segments (equal
 // numbers of chunks, the last may be shorter or empty); tiles = D / DVT column
 // slices of the state.  Roles:
-//   warps 0-3  state:    thread t owns key row t of the fp32 state tile
-//                        S[:, col0:col0+DVT] in registers; per chunk it applies
+//   NSW = 4 DVT/32 state warps: warp w's thread owns key row 32 (w % 4) + lane,
+//                        columns 32 (w / 4) .. + 31 of the fp32 state tile
+//                        S[:, col0:col0+DVT], in registers; per chunk it applies
 //                        S <- exp(G_C) S + R + (M' S) and writes the bf16 copy of
 //                        the new state that the next products read;
-//   warp 4     MMA:      one elected lane issues, per chunk,
+//   1 MMA warp:          one elected lane issues, per chunk,
 //                          D_S        = M'(j) S   (M = 128 key rows, N = DVT, K = 128)
 //                          D_O[j & 1] = Q'(j) S   (M = 64 chunk rows)
 //                        on tcgen05, accumulating in tensor memory;
-//   warps 5-8  output:   O = D_O + O0 for the chunk's rows (warp w reads tensor-memory
+//   4 output warps:      O = D_O + O0 for the chunk's rows (warp w reads tensor-memory
 //                        lane quarter w % 4), stored as bf16;
-//   warp 9     producer: bulk copies of the chunk records into two rings, the state
+//   1 producer warp:     bulk copies of the chunk records into two rings, the state
 //                        ring (M', exp(G_C), R slice) and the output ring (Q', O0 slice),
 //                        refilling a slot once its consumers release it.
 // The roles hand off through mbarriers only, so the loop-carried path per chunk is
