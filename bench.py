@@ -416,15 +416,24 @@ def run_ours_decode(args, world, rank, local):
     }
 
 
-def kernel_source_sha():
-    """sha256 over the CUDA sources of the library (identifies a kernel build)."""
+def _strip_comments(text):
+    """C/C++ source without comments and blank lines (string literals are kept)."""
+    import re
+    pat = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', re.S)
+    text = pat.sub(lambda m: m.group(0) if m.group(0).startswith('"') else "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
+def kernel_source_sha(src=None):
+    """sha256 over the CUDA sources of the library with comments removed (identifies
+    the kernel code; an edit of comments alone keeps it)."""
     import hashlib
-    src = os.path.join(ROOT, "kimi_delta_attention_28_b200", "csrc")
+    src = src or os.path.join(ROOT, "kimi_delta_attention_28_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(src)):
         if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(src, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+            with open(os.path.join(src, f), encoding="utf-8") as fh:
+                h.update(f.encode() + b"\0" + _strip_comments(fh.read()).encode())
     return h.hexdigest()
 
 
