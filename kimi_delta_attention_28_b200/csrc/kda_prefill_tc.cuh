@@ -746,7 +746,12 @@ struct T5Layout {
     static constexpr int NBAR = 2 * (NA + NB) + 9;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;   // tmem slot, abort flag, counters
     static constexpr int BYTES = OFF_MISC + 32 + 1024;    // + slack for 1024-byte alignment
-    static constexpr uint32_t TMEM_COLS = DVT == 32 ? 128 : 256;   // D_S | D_O[0] | D_O[1]
+    // Tensor memory: D_S[0] | D_O[0] | D_O[1] | D_S[1], DVT columns each.  D_S is
+    // double-buffered by chunk parity: the next chunk's M'.S starts as soon as the
+    // first state warp has handed over its K slab, while the other state warps may
+    // still be reading this chunk's D_S.
+    static constexpr uint32_t TMEM_COLS = DVT == 32 ? 128 : 256;
+    KDA_DEVINL static uint32_t ds_col(int parity) { return parity ? 3 * DVT : 0; }
     // B operand (the state copy), MN-major: row k (key) holds DVT bf16 values.
     // DVT = 64: 128-byte rows, 128-byte swizzle; DVT = 32: 64-byte rows, 64-byte swizzle.
     static constexpr uint32_t SB_ROW = DVT * 2;
@@ -907,7 +912,7 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
             if (!ok) { fail(); break; }
             t5::fence_after_sync();
             float v[32];
-            t5::ld32(tmem + lane_base + cb, v);
+            t5::ld32(tmem + lane_base + L::ds_col(j & 1) + cb, v);
             t5::fence_before_sync();
             mbar_arrive(&a_free[sa]);   // this thread is done with the slot and with D_S
 #pragma unroll
@@ -966,7 +971,7 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
                         const int ks = 2 * w + kk;
-                        t5::mma_bf16(tmem, am0 + (uint64_t)((ks * 2 * D * 16) >> 4),
+                        t5::mma_bf16(tmem + L::ds_col(j & 1), am0 + (uint64_t)((ks * 2 * D * 16) >> 4),
                                      bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idS, ks > 0);
                     }
                 }
