@@ -942,23 +942,23 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
         // ---------------- MMA warp ----------------
         constexpr uint32_t idS = t5::idesc_bf16(128, DVT, 0, 1);
         constexpr uint32_t idO = t5::idesc_bf16(64, DVT, 0, 1);
+        // One lane issues every product, so each commit also covers the products it
+        // issued before: done_s(j) implies the previous chunk's Q'.S is complete too.
+        const bool leader = t5::elect_one();
         for (int j = 0; j < nchunks && !*abort_flag; ++j) {
             const int sa = j % NA, sbb = j % NB;
-            bool ok = mbar_wait_bounded(&full_a[sa], (j / NA) & 1) &&
-                      (map_mode || mbar_wait_bounded(&full_b[sbb], (j / NB) & 1)) &&
-                      (map_mode || j < 2 ||
-                       mbar_wait_bounded(&do_free[j & 1], ((j - 2) >> 1) & 1));
+            // M'.S waits only for its ring slot and the state copy; the output product's
+            // ring slot and accumulator are waited for after it is on its way
+            bool ok = mbar_wait_bounded(&full_a[sa], (j / NA) & 1);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) { fail(); break; }
             bool slab_ok = true;
-            if (t5::elect_one()) {
-                const uint32_t sb_addr = sm_addr + L::OFF_SB + (j & 1) * L::SB_BYTES;
-                const uint64_t bd0 = t5::smem_desc(sb_addr, 4096, 8 * L::SB_ROW, L::SB_SWZ);
+            const uint32_t sb_addr = sm_addr + L::OFF_SB + (j & 1) * L::SB_BYTES;
+            const uint64_t bd0 = t5::smem_desc(sb_addr, 4096, 8 * L::SB_ROW, L::SB_SWZ);
+            if (leader) {
                 // A operands in the core-matrix layout: 8-row groups 128 B apart (SBO),
                 // 8-column chunks rows*16 B apart (LBO), no swizzle.
                 const uint64_t am0 = t5::smem_desc(sm_addr + sa * L::A_BYTES, D * 16, 128, 0);
-                const uint64_t aq0 = t5::smem_desc(sm_addr + L::OFF_B + sbb * L::B_BYTES,
-                                                   C * 16, 128, 0);
                 // M'.S by K slabs: slab w (key rows 32w..32w+31, two K=16 steps) goes as
                 // soon as state warp w has written its rows of the copy
 #pragma unroll
@@ -976,19 +976,28 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
                     }
                 }
                 t5::commit(done_s);
-                if (!map_mode && slab_ok) {
-                    const uint32_t dO = tmem + DVT + (j & 1) * DVT;
+            }
+            bool ok2 = !__any_sync(0xffffffffu, !slab_ok);
+            ok2 = ok2 && (map_mode || (mbar_wait_bounded(&full_b[sbb], (j / NB) & 1) &&
+                                       (j < 2 || mbar_wait_bounded(&do_free[j & 1], ((j - 2) >> 1) & 1))));
+            ok2 = __all_sync(0xffffffffu, ok2);
+            if (leader) {
+                if (!map_mode) {
+                    if (ok2) {
+                        const uint64_t aq0 = t5::smem_desc(sm_addr + L::OFF_B + sbb * L::B_BYTES,
+                                                           C * 16, 128, 0);
+                        const uint32_t dO = tmem + DVT + (j & 1) * DVT;
+                        t5::fence_after_sync();
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks)
-                        t5::mma_bf16(dO, aq0 + (uint64_t)((ks * 2 * C * 16) >> 4),
-                                     bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idO, ks > 0);
-                    t5::commit(&done_o[j & 1]);
-                } else if (!map_mode) {
-                    t5::commit(&done_o[j & 1]);   // so the drain below can wait on it
+                        for (int ks = 0; ks < D / 16; ++ks)
+                            t5::mma_bf16(dO, aq0 + (uint64_t)((ks * 2 * C * 16) >> 4),
+                                         bd0 + (uint64_t)((ks * 16 * L::SB_ROW) >> 4), idO, ks > 0);
+                    }
+                    t5::commit(&done_o[j & 1]);   // always: the drain below waits on it
                 }
                 cnt[2] = j + 1;
             }
-            if (__any_sync(0xffffffffu, !slab_ok)) { fail(); break; }
+            if (!ok2) { fail(); break; }
         }
     } else if (warp < RL::PROD_WARP) {
         // ---------------- output warps (none in the map pass) ----------------
