@@ -114,6 +114,41 @@ def _need(t, name, dtype=None, device=None):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
 
 
+def _shape(t, name, shape):
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _prefill_shapes(q, k, v, g, beta, h0=None, cu_seqlens=None, o=None, hT=None,
+                    workspace=None):
+    """Check the tensors' shapes against q's [B, T, H, d_k] (metadata only; the C ABI
+    sees raw pointers and would read past a short tensor).  Returns (B, T, H, dk, dv,
+    num_seqs, N)."""
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, T, H, d_k], got shape {tuple(q.shape)}")
+    B, T, H, dk = q.shape
+    if v.dim() != 4 or tuple(v.shape[:3]) != (B, T, H):
+        raise ValueError(f"v has shape {tuple(v.shape)}, expected ({B}, {T}, {H}, d_v)")
+    dv = v.shape[3]
+    _shape(k, "k", q.shape)
+    _shape(g, "g", q.shape)
+    _shape(beta, "beta", (B, T, H))
+    num_seqs = 0
+    if cu_seqlens is not None:
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must be a 1-D tensor of N + 1 offsets")
+        if B != 1:
+            raise ValueError("packed sequences (cu_seqlens) need B == 1")
+        num_seqs = cu_seqlens.numel() - 1
+    N = B if cu_seqlens is None else num_seqs
+    _shape(h0, "h0", (N, H, dk, dv))
+    _shape(o, "o", (B, T, H, dv))
+    _shape(hT, "hT", (N, H, dk, dv))
+    if workspace is not None and (workspace.dtype != torch.uint8 or workspace.dim() != 1):
+        raise ValueError("workspace must be a 1-D uint8 tensor (its numel is the byte count)")
+    return B, T, H, dk, dv, num_seqs, N
+
+
 def workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
                    dtype: torch.dtype) -> int:
     return int(load_library().kda_fwd_workspace_size(B, T, H, dk, dv, num_seqs,
@@ -131,17 +166,17 @@ def kda_fwd(q, k, v, g, beta, h0=None, cu_seqlens=None, *, output_final_state: b
     """
     lib = load_library()
     dev = q.device
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T, H, dk, dv, num_seqs, N = _prefill_shapes(q, k, v, g, beta, h0, cu_seqlens, o, hT,
+                                                   workspace)
     dt = _dtype_code(q.dtype)
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _need(t, n, q.dtype, dev)
     _need(g, "g", torch.float32, dev)
     _need(beta, "beta", torch.float32, dev)
     _need(h0, "h0", torch.float32, dev)
+    _need(hT, "hT", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    N = B if cu_seqlens is None else num_seqs
+    _need(workspace, "workspace", torch.uint8, dev)
     if o is None:
         o = torch.empty(B, T, H, dv, dtype=q.dtype, device=dev)
     if hT is None and output_final_state:
@@ -176,16 +211,16 @@ def kda_fwd_segmented(q, k, v, g, beta, h0=None, cu_seqlens=None, *, num_segment
     returns (o, hT)."""
     lib = load_library()
     dev = q.device
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+    B, T, H, dk, dv, num_seqs, N = _prefill_shapes(q, k, v, g, beta, h0, cu_seqlens, o, hT,
+                                                   workspace)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _need(t, n, q.dtype, dev)
     _need(g, "g", torch.float32, dev)
     _need(beta, "beta", torch.float32, dev)
     _need(h0, "h0", torch.float32, dev)
+    _need(hT, "hT", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    N = B if cu_seqlens is None else num_seqs
+    _need(workspace, "workspace", torch.uint8, dev)
     if o is None:
         o = torch.empty(B, T, H, dv, dtype=q.dtype, device=dev)
     if hT is None:
@@ -206,10 +241,14 @@ def kda_fwd_intra(q, k, v, g, beta, cu_seqlens=None, *, workspace):
     intra-chunk records into ``workspace``.  Same argument conventions as kda_fwd."""
     lib = load_library()
     dev = q.device
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T, H, dk, dv, num_seqs, _ = _prefill_shapes(q, k, v, g, beta, None, cu_seqlens,
+                                                   workspace=workspace)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _need(workspace, "workspace", torch.uint8, dev)
     _check(lib.kda_fwd_intra(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
                              num_seqs, B, T, H, dk, dv, _dtype_code(q.dtype), _ptr(workspace),
                              workspace.numel(), _stream(dev)), "kda_fwd_intra")
@@ -220,6 +259,15 @@ def kda_fwd_inter(h0, cu_seqlens, o, hT, *, B, T, H, dk, dv, dtype, workspace):
     lib = load_library()
     dev = o.device
     num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = B if cu_seqlens is None else num_seqs
+    _shape(o, "o", (B, T, H, dv))
+    _shape(h0, "h0", (N, H, dk, dv))
+    _shape(hT, "hT", (N, H, dk, dv))
+    _need(o, "o", dtype, dev)
+    _need(h0, "h0", torch.float32, dev)
+    _need(hT, "hT", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(workspace, "workspace", torch.uint8, dev)
     _check(lib.kda_fwd_inter(_ptr(h0), _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv,
                              _dtype_code(dtype), _ptr(o), _ptr(hT), _ptr(workspace),
                              workspace.numel(), _stream(dev)), "kda_fwd_inter")
@@ -230,10 +278,18 @@ def kda_decode_step(q, k, v, g, beta, S, o=None):
     in place.  q, k, g: [N, H, d_k]; v: [N, H, d_v]; beta: [N, H].  Returns o."""
     lib = load_library()
     dev = q.device
+    if q.dim() != 3 or v.dim() != 3 or tuple(v.shape[:2]) != tuple(q.shape[:2]):
+        raise ValueError(f"q must be [N, H, d_k] and v [N, H, d_v], got {tuple(q.shape)} "
+                         f"and {tuple(v.shape)}")
     N, H, dk = q.shape
     dv = v.shape[-1]
+    _shape(k, "k", q.shape)
+    _shape(g, "g", q.shape)
+    _shape(beta, "beta", (N, H))
+    _shape(S, "S", (N, H, dk, dv))
+    _shape(o, "o", (N, H, dv))
     dt = _dtype_code(q.dtype)
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _need(t, n, q.dtype, dev)
     _need(g, "g", torch.float32, dev)
     _need(beta, "beta", torch.float32, dev)
@@ -253,8 +309,7 @@ def kda_fwd_noalloc(q, k, v, g, beta, h0, cu_seqlens, o, hT):
     nothing.  bf16, d = 128 only; the problem must fit the 32 MiB scratch."""
     lib = load_library()
     dev = q.device
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    B, T, H, dk, dv, num_seqs, _ = _prefill_shapes(q, k, v, g, beta, h0, cu_seqlens, o, hT)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _need(t, n, q.dtype, dev)
     _need(g, "g", torch.float32, dev)
@@ -262,7 +317,6 @@ def kda_fwd_noalloc(q, k, v, g, beta, h0, cu_seqlens, o, hT):
     _need(h0, "h0", torch.float32, dev)
     _need(hT, "hT", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
     _check(lib.kda_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
                                _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, _dtype_code(q.dtype),
                                _ptr(o), _ptr(hT), _stream(dev)), "kda_fwd_noalloc")

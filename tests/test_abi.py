@@ -158,6 +158,37 @@ def test_python_binding_rejects_cpu_tensors():
         kda.kda_fwd(x, x, x, x.float(), torch.zeros(1, 4, 1), None)
 
 
+def test_python_binding_checks_shapes_before_launch():
+    """The C ABI sees raw pointers, so the binding checks every tensor's shape
+    against q's (metadata only: these CPU tensors never reach the library)."""
+    import torch
+    B, T, H, d = 1, 8, 2, 64
+    q = torch.zeros(B, T, H, d, dtype=torch.bfloat16)
+    g = torch.zeros(B, T, H, d)
+    beta = torch.zeros(B, T, H)
+    short = torch.zeros(B, T - 1, H, d, dtype=torch.bfloat16)
+    cases = [
+        dict(k=short), dict(v=short), dict(g=g[:, :-1]), dict(beta=beta[:, :-1]),
+        dict(h0=torch.zeros(B, H, d, d - 1)), dict(o=short),
+        dict(hT=torch.zeros(B + 1, H, d, d)),
+        dict(workspace=torch.zeros(16, dtype=torch.float32)),
+        dict(cu_seqlens=torch.tensor([0, 4, 8], dtype=torch.int32), h0=torch.zeros(1, H, d, d)),
+    ]
+    for over in cases:
+        a = dict(q=q, k=q, v=q, g=g, beta=beta, h0=None)
+        a.update(over)
+        kw = {n: a.pop(n) for n in ("o", "hT", "workspace", "cu_seqlens") if n in a}
+        cu = kw.pop("cu_seqlens", None)
+        with pytest.raises(ValueError, match="shape|workspace|cu_seqlens"):
+            kda.kda_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["h0"], cu, **kw)
+    with pytest.raises(ValueError, match="shape"):   # decode: state of the wrong size
+        kda.kda_decode_step(q[0], q[0], q[0], g[0], beta[0], torch.zeros(T, H, d, d + 1))
+    with pytest.raises(ValueError, match="B == 1"):
+        kda.kda_fwd(q.expand(2, T, H, d), q.expand(2, T, H, d), q.expand(2, T, H, d),
+                    g.expand(2, T, H, d), beta.expand(2, T, H), None,
+                    torch.tensor([0, 8], dtype=torch.int32))
+
+
 def test_library_is_built_for_sm100a():
     # the build recipe targets sm_100a only
     assert "arch=compute_100a,code=sm_100a" in " ".join(build.FLAGS)
