@@ -184,10 +184,22 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    # --ckpt-every N: every step also stores the state after each N tokens of every
+    # sequence (kda_fwd_checkpointed, prefix caching) into a preallocated buffer
+    ck = None
+    if args.ckpt_every > 0:
+        ck = torch.empty(kda.checkpoint_count(T, args.ckpt_every, B, cu), H, dk, dv,
+                         dtype=torch.float32, device=dev)
+
     def step():
-        # one kda_fwd call: the state pass may start while the prep kernel finishes
-        kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], cu, o=o,
-                    hT=hT, workspace=ws)
+        # one kda_fwd call: the prep kernel, then the state pass
+        if ck is not None:
+            kda.kda_fwd_checkpointed(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                     inp["h0"], cu, ckpt_every=args.ckpt_every, ckpts=ck, o=o,
+                                     hT=hT, workspace=ws)
+        else:
+            kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], cu, o=o,
+                        hT=hT, workspace=ws)
 
     def step_split(ev):
         # the two phases as separate calls, an event between them: per-kernel times
@@ -243,7 +255,7 @@ def run_ours(args, world, rank, local):
     # are pipelined on three streams with two buffer sets, so step i+1's inputs go
     # up while step i computes and step i-1's results come down.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and ck is None:
         host = {k_: (v_.cpu().pin_memory() if v_ is not None else None) for k_, v_ in inp.items()}
         o_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
         hT_h = [torch.empty(hT.shape, dtype=hT.dtype).pin_memory() for _ in range(2)]
@@ -343,6 +355,11 @@ def run_ours(args, world, rank, local):
         "clocks": clocks.summary(t_wall0, t_wall1),
         "e2e": e2e,
     }
+    if ck is not None:
+        out["config"]["ckpt_every"] = args.ckpt_every
+        out["config"]["checkpoints_per_head"] = int(ck.shape[0])
+        out["kernels_ms_note"] = ("per-kernel split measured through kda_fwd_intra / "
+                                  "kda_fwd_inter, which store no checkpoints")
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_seconds)
     return out
@@ -559,6 +576,8 @@ def main():
     ap.add_argument("--workload", choices=["prefill", "long", "varlen", "decode", "few_chains"],
                     default="prefill")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ckpt-every", type=int, default=0,
+                    help="prefill workloads: also store the state every N tokens (multiple of 64)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)

@@ -52,7 +52,8 @@ typedef enum {
     KDA_ERR_CUDA = 5,                 /* a CUDA launch or query failed             */
     KDA_ERR_DEVICE_TIMEOUT = 6,       /* a bounded device-side wait gave up        */
     KDA_ERR_BAD_SEQLENS = 7,          /* cu_seqlens not monotone / out of range    */
-    KDA_ERR_EXCEEDS_STATIC_SCRATCH = 8 /* kda_fwd_noalloc: problem too large       */
+    KDA_ERR_EXCEEDS_STATIC_SCRATCH = 8, /* kda_fwd_noalloc: problem too large      */
+    KDA_ERR_CHECKPOINT_CAPACITY = 9   /* kda_fwd_checkpointed: more checkpoints than slots */
 } kda_status;
 
 typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
@@ -172,6 +173,41 @@ kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const 
                              size_t ws_bytes, void *stream);
 
 /*
+ * kda_fwd that also stores the state at fixed token intervals, for prefix caching
+ * (a later call resumes from a stored state as its h0).  The state is the one
+ * after a whole number of tokens; checkpoints sit on the 64-token chunk
+ * boundaries, so ckpt_every must be a positive multiple of 64.
+ *
+ * For sequence n of length L_n and head h, checkpoint c = 0 .. L_n / ckpt_every - 1
+ * (integer division) is the state after the sequence's first (c + 1) * ckpt_every
+ * tokens, stored fp32 at
+ *     ckpts[((first_n + c) * H + h) * d_k * d_v ...],   [d_k][d_v] row-major,
+ *     first_n = sum over m < n of L_m / ckpt_every,
+ * i.e. ckpts is [num_checkpoints, H, d_k, d_v] with the checkpoints of each sequence
+ * together and in token order.  ckpt_capacity is the number of checkpoint slots
+ * (the first dimension of ckpts).  For fixed-length input it must be at least
+ * B * (T / ckpt_every), else KDA_ERR_INVALID_ARG; for packed input the lengths
+ * live on the device, so a checkpoint past the capacity is not written and the
+ * call's device error becomes KDA_ERR_CHECKPOINT_CAPACITY.
+ *
+ * Tensor-core path only (bf16, d_k = d_v = 128), else KDA_ERR_UNSUPPORTED_SHAPE.
+ * ckpts must be 16-byte aligned (KDA_ERR_MISALIGNED) and must not overlap any
+ * other argument.  Workspace, o, hT and the time-split policy as for kda_fwd; o
+ * and hT are bitwise those of kda_fwd.
+ *
+ * Source: the "Kimi K3" open-weights field notes, panel "目标模型太大，缓存和草稿都必须
+ * 理解 KDA" (a prefix cache must restore the KDA recurrent state at the same token
+ * boundary as the attention cache), and the API card's 256-token shortest cached
+ * prefix; the stored state is the recurrence's S_t (panel "KDA 单头递归").
+ */
+kda_status kda_fwd_checkpointed(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *h0, const int32_t *cu_seqlens,
+                                int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
+                                void *o, float *hT, int ckpt_every, float *ckpts,
+                                long long ckpt_capacity, void *workspace, size_t ws_bytes,
+                                void *stream);
+
+/*
  * One decode step: every (sequence, head) consumes one token and updates its
  * state in place (the recurrence above with T = 1).
  *
@@ -226,8 +262,9 @@ kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const fl
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error word
- * (cu_seqlens violations, bounded waits that gave up).  Returns KDA_OK,
- * KDA_ERR_BAD_SEQLENS, KDA_ERR_DEVICE_TIMEOUT or KDA_ERR_CUDA.
+ * (cu_seqlens violations, bounded waits that gave up, checkpoints past the
+ * capacity).  Returns KDA_OK, KDA_ERR_BAD_SEQLENS, KDA_ERR_DEVICE_TIMEOUT,
+ * KDA_ERR_CHECKPOINT_CAPACITY or KDA_ERR_CUDA.
  */
 kda_status kda_get_last_device_error(void *stream);
 

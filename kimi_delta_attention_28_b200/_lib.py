@@ -21,7 +21,7 @@ KDA_DTYPE_BF16 = 1
 STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED_SHAPE",
           3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_WORKSPACE_TOO_SMALL", 5: "KDA_ERR_CUDA",
           6: "KDA_ERR_DEVICE_TIMEOUT", 7: "KDA_ERR_BAD_SEQLENS",
-          8: "KDA_ERR_EXCEEDS_STATIC_SCRATCH"}
+          8: "KDA_ERR_EXCEEDS_STATIC_SCRATCH", 9: "KDA_ERR_CHECKPOINT_CAPACITY"}
 
 # Size of the static scratch array behind kda_fwd_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -45,6 +45,8 @@ SIGNATURES = {
     "kda_fwd_plan_segments": ([_I, _I, _I, _I, _I, _I, _I], _I),
     "kda_fwd_segmented": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I,
                            _VP, _VP, _VP, _SZ, _VP], _I),
+    "kda_fwd_checkpointed": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP,
+                              _VP, _I, _VP, ctypes.c_longlong, _VP, _SZ, _VP], _I),
 }
 
 
@@ -234,6 +236,59 @@ def kda_fwd_segmented(q, k, v, g, beta, h0=None, cu_seqlens=None, *, num_segment
                                  _ptr(workspace), workspace.numel(), _stream(dev)),
            "kda_fwd_segmented")
     return o, hT
+
+
+def checkpoint_count(T: int, ckpt_every: int, B: int = 1, cu_seqlens=None) -> int:
+    """Number of state checkpoints kda_fwd_checkpointed stores per head: sum over the
+    sequences of length // ckpt_every (reads packed lengths back from the device)."""
+    if cu_seqlens is None:
+        return B * (T // ckpt_every)
+    lens = (cu_seqlens[1:] - cu_seqlens[:-1]).to("cpu", torch.int64)
+    return int((lens // ckpt_every).sum())
+
+
+def kda_fwd_checkpointed(q, k, v, g, beta, h0=None, cu_seqlens=None, *, ckpt_every: int = 256,
+                         ckpts=None, o=None, hT=None, workspace=None):
+    """kda_fwd that also stores the state after every ``ckpt_every`` tokens of each
+    sequence (a multiple of 64), for prefix caching.  Returns (o, hT, ckpts) with
+    ckpts [num_checkpoints, H, d_k, d_v] fp32: each sequence's checkpoints together, in
+    token order; checkpoint c of a sequence is its state after (c + 1) * ckpt_every
+    tokens.  When ``ckpts`` is not given it is allocated here (packed input: the
+    lengths are read back from the device)."""
+    lib = load_library()
+    dev = q.device
+    B, T, H, dk, dv, num_seqs, N = _prefill_shapes(q, k, v, g, beta, h0, cu_seqlens, o, hT,
+                                                   workspace)
+    if ckpt_every <= 0 or ckpt_every % 64:
+        raise ValueError(f"ckpt_every must be a positive multiple of 64, got {ckpt_every}")
+    if ckpts is not None and (ckpts.dim() != 4 or tuple(ckpts.shape[1:]) != (H, dk, dv)):
+        raise ValueError(f"ckpts has shape {tuple(ckpts.shape)}, expected (n, {H}, {dk}, {dv})")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, n, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(h0, "h0", torch.float32, dev)
+    _need(hT, "hT", torch.float32, dev)
+    _need(ckpts, "ckpts", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    if ckpts is None:
+        ckpts = torch.empty(checkpoint_count(T, ckpt_every, B, cu_seqlens), H, dk, dv,
+                            dtype=torch.float32, device=dev)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=q.dtype, device=dev)
+    if hT is None:
+        hT = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    need = workspace_size(B, T, H, dk, dv, num_seqs, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.kda_fwd_checkpointed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                    _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv,
+                                    _dtype_code(q.dtype), _ptr(o), _ptr(hT), ckpt_every,
+                                    _ptr(ckpts) if ckpts.numel() else None, ckpts.shape[0],
+                                    _ptr(workspace), workspace.numel(), _stream(dev)),
+           "kda_fwd_checkpointed")
+    return o, hT, ckpts
 
 
 def kda_fwd_intra(q, k, v, g, beta, cu_seqlens=None, *, workspace):

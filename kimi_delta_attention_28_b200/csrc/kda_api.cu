@@ -23,6 +23,7 @@ namespace {
 
 constexpr int ERRBIT_SEQLENS = 1;
 constexpr int ERRBIT_TIMEOUT = 2;
+constexpr int ERRBIT_CKPT = 4;
 
 inline bool aligned_to(const void *p, size_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;  // NULL counts as aligned
@@ -208,6 +209,9 @@ const char *kda_status_string(kda_status s) {
         case KDA_ERR_EXCEEDS_STATIC_SCRATCH:
             return "KDA_ERR_EXCEEDS_STATIC_SCRATCH: problem needs more scratch than the 32 MiB "
                    "static array of kda_fwd_noalloc; use kda_fwd with a workspace";
+        case KDA_ERR_CHECKPOINT_CAPACITY:
+            return "KDA_ERR_CHECKPOINT_CAPACITY: the sequences have more state checkpoints than "
+                   "ckpt_capacity slots";
         default: return "KDA_ERR_UNKNOWN";
     }
 }
@@ -297,7 +301,8 @@ static kda_status tc_intra(const void *q, const void *k, const void *v, const fl
 // Tensor-core path, phase 2: the state pass over the records.
 static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int H,
                            const WsLayout &L, void *o, float *hT, void *workspace,
-                           cudaStream_t s) {
+                           cudaStream_t s, float *ckpt = nullptr, int ckpt_chunks = 0,
+                           long long ckpt_cap = 0) {
     using namespace kda::tc;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *hdr = reinterpret_cast<int *>(ws + L.hdr);
@@ -315,6 +320,9 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
     a.cu = cu;
     a.nseg = L.nseg;
     a.mode = kStateOutput;
+    a.ckpt = ckpt;
+    a.ckpt_chunks = ckpt_chunks;
+    a.ckpt_cap = ckpt_cap;
     const long long chains = (long long)N * H;
     if (L.nseg <= 1) {
         // 32-column slices give the shortest per-chunk latency (they suit few chains);
@@ -406,6 +414,31 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                                         cu_seqlens, s);
 }
 
+kda_status kda_fwd_checkpointed(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *h0, const int32_t *cu_seqlens,
+                                int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
+                                void *o, float *hT, int ckpt_every, float *ckpts,
+                                long long ckpt_capacity, void *workspace, size_t ws_bytes,
+                                void *stream) {
+    int N;
+    WsLayout L;
+    kda_status st = validate_fwd(q, k, v, g, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv,
+                                 dtype, o, hT, workspace, ws_bytes, true, true, &N, &L);
+    if (st != KDA_OK) return st;
+    if (!is_tc_path(dtype, dk)) return KDA_ERR_UNSUPPORTED_SHAPE;
+    if (ckpt_every <= 0 || ckpt_every % kda::tc::C != 0 || ckpt_capacity < 0)
+        return KDA_ERR_INVALID_ARG;
+    if (ckpt_capacity > 0 && !ckpts) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(ckpts, 16)) return KDA_ERR_MISALIGNED;
+    if (!cu_seqlens && (long long)B * (T / ckpt_every) > ckpt_capacity) return KDA_ERR_INVALID_ARG;
+    if (N == 0) return KDA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = tc_intra(q, k, v, g, beta, cu_seqlens, N, T, H, L, workspace, s)) != KDA_OK)
+        return st;
+    return tc_inter(h0, cu_seqlens, N, T, H, L, o, hT, workspace, s, ckpts,
+                    ckpt_every / kda::tc::C, ckpt_capacity);
+}
+
 int kda_fwd_plan_segments(int B, int T, int H, int dk, int dv, int num_seqs, int dtype) {
     if (B < 0 || T < 0 || num_seqs < 0) return 0;
     if (check_shape(H, dk, dv, dtype) != KDA_OK) return 0;
@@ -489,6 +522,7 @@ kda_status kda_get_last_device_error(void *stream) {
         return KDA_ERR_CUDA;
     if (word & ERRBIT_SEQLENS) return KDA_ERR_BAD_SEQLENS;
     if (word & ERRBIT_TIMEOUT) return KDA_ERR_DEVICE_TIMEOUT;
+    if (word & ERRBIT_CKPT) return KDA_ERR_CHECKPOINT_CAPACITY;
     return KDA_OK;
 }
 

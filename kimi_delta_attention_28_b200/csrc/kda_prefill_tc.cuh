@@ -82,6 +82,7 @@ struct ChunkLoc {
 };
 
 constexpr int ERR_TIMEOUT_BIT = 2;
+constexpr int ERR_CKPT_BIT = 4;   // a state checkpoint fell past the caller's capacity
 
 // ---------------------------------------------------------------------------
 // Varlen chunk map: validates cu_seqlens and lays out each sequence's chunks.
@@ -706,7 +707,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 //
 // Modes.  kStateOutput: the pass proper -- outputs for every chunk, the unit's
 // starting state from h0 (or s_in, per unit, after a T-split), the final state to
-// hT (last segment only).  kStateMap: the first pass of the T-split -- the unit's
+// hT (last segment only), and with ckpt_chunks > 0 the state after every ckpt_chunks
+// whole chunks of each sequence (prefix-cache checkpoints; the segment offset keeps
+// the count per sequence).  kStateMap: the first pass of the T-split -- the unit's
 // affine map S_out = P S_in + R over its segment, obtained by running the same
 // recurrence on a widened state [R | P] of 2D columns: the R half from zero with
 // the records' R added, the P half from the identity without it (the map is affine,
@@ -727,6 +730,11 @@ struct StateArgs {
     int mode;                 // kStateOutput or kStateMap
     const float *s_in;        // kStateOutput after a T-split: [units, D, D] starting states
     float *seg_map;           // kStateMap: [units, D, 2D] = [R | P] per unit
+    // kStateOutput: state checkpoints every ckpt_chunks chunks of each sequence (0: none)
+    // into ckpt[slot][H][D][D], ckpt_cap slots, each sequence's slots in token order
+    float *ckpt;
+    int ckpt_chunks;
+    long long ckpt_cap;
 };
 template <int DVT>
 struct T5Layout {
@@ -817,9 +825,12 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
         seq_t0 = n * a.T;
         seq_len = a.T;
     }
+    const int seq_tokens = seq_len;   // the whole sequence
+    int seg_lo;                       // chunks of the sequence before this unit's segment
     {   // this unit's segment of the chain
         const int nch = c_end - c_begin, per = (nch + a.nseg - 1) / a.nseg;
         const int lo = min(nch, seg * per), hi = min(nch, lo + per);
+        seg_lo = lo;
         c_begin += lo;
         c_end = c_begin + (hi - lo);
         seq_t0 += lo * C;
@@ -881,6 +892,22 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] = (row == col0 + cb + i) ? 1.f : 0.f;
         }
+        // state checkpoints: the first slot of this sequence (its earlier sequences'
+        // checkpoint counts, summed by the warp for packed input)
+        const bool ckpt_on = !map_mode && a.ckpt_chunks > 0;
+        long long ck_first = 0;
+        if (ckpt_on) {
+            const int every = a.ckpt_chunks * C;
+            if (a.cu) {
+                long long part = 0;
+                for (int m = lane; m < n; m += 32) part += (a.cu[m + 1] - a.cu[m]) / every;
+#pragma unroll
+                for (int off = 16; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+                ck_first = part;
+            } else {
+                ck_first = (long long)n * (seq_tokens / every);
+            }
+        }
         auto write_sb = [&](int buf) {   // bf16 copy of this thread's part of its row, then signal
             uint8_t *sb = sm + L::OFF_SB + buf * L::SB_BYTES;
 #pragma unroll
@@ -924,6 +951,20 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
                     const int c = i * 8 + 2 * e;
                     S[c] = fmaf(gam, S[c], r2.x + v[c]);
                     S[c + 1] = fmaf(gam, S[c + 1], r2.y + v[c + 1]);
+                }
+            }
+            if (ckpt_on) {   // S now holds the state after `done` whole chunks of the sequence
+                const int done = seg_lo + j + 1;
+                if (done % a.ckpt_chunks == 0 && done * C <= seq_tokens) {
+                    const long long slot = ck_first + done / a.ckpt_chunks - 1;
+                    if (slot < a.ckpt_cap) {
+                        float *cp = a.ckpt + ((slot * H + h) * D + row) * D + col0 + cb;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4 *>(cp + i) = make_float4(S[i], S[i + 1], S[i + 2], S[i + 3]);
+                    } else if (lane == 0) {
+                        atomicOr(err_word, ERR_CKPT_BIT);
+                    }
                 }
             }
             if (j + 1 < nchunks) write_sb((j + 1) & 1);

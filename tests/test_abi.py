@@ -48,7 +48,7 @@ def test_binding_declares_nothing_extra():
 
 def test_version_and_status_strings(lib):
     assert lib.kda_version() >= 100
-    for code in range(8):
+    for code in range(10):
         s = lib.kda_status_string(code).decode()
         assert s.startswith("KDA_")
     assert lib.kda_status_string(99).decode() == "KDA_ERR_UNKNOWN"
@@ -127,6 +127,30 @@ def test_fwd_validation_before_launch(lib):
     assert _fwd(lib, cu=0x30002, num_seqs=2) == MISALIGNED
     # empty batch: valid, nothing to do, no launch
     assert _fwd(lib, B=0) == OK
+
+
+def test_checkpointed_validation_before_launch(lib):
+    """kda_fwd_checkpointed checks its checkpoint arguments on the host, before any
+    launch: interval a positive multiple of 64, enough slots for fixed-length input,
+    a 16-byte aligned buffer, the tensor-core path only."""
+    p = 0x10000
+
+    def ck(every=256, ckpts=0x40000, cap=2, B=1, T=512, H=2, dk=128, dtype=BF16, cu=None,
+           num_seqs=0):
+        return lib.kda_fwd_checkpointed(p, p, p, p, p, None, cu, num_seqs, B, T, H, dk, dk, dtype,
+                                        p + 0x100000, None, every, ckpts, cap, p, 1 << 40, None)
+    assert ck(every=100) == INVALID                     # not a chunk boundary
+    assert ck(every=0) == INVALID
+    assert ck(every=-64) == INVALID
+    assert ck(cap=1) == INVALID                         # 512 // 256 = 2 checkpoints needed
+    assert ck(B=3, cap=5) == INVALID                    # 3 sequences x 2
+    assert ck(ckpts=None, cap=2) == INVALID             # slots promised, no buffer
+    assert ck(cap=-1) == INVALID
+    assert ck(ckpts=0x40008) == MISALIGNED              # stored as float4
+    assert ck(dk=64) == UNSUPPORTED                     # tensor-core path only
+    assert ck(dtype=F32) == UNSUPPORTED
+    assert ck(B=0) == OK                                # nothing to do, no launch
+    assert lib.kda_status_string(9).decode().startswith("KDA_ERR_CHECKPOINT_CAPACITY")
 
 
 def test_phase_entry_points_validate(lib):
