@@ -153,6 +153,16 @@ def test_checkpointed_validation_before_launch(lib):
     assert lib.kda_status_string(9).decode().startswith("KDA_ERR_CHECKPOINT_CAPACITY")
 
 
+def test_checkpoint_count():
+    """Slots kda_fwd_checkpointed needs: the sum over sequences of length // interval."""
+    import torch
+    assert kda.checkpoint_count(1000, 128, B=2) == 2 * 7
+    assert kda.checkpoint_count(63, 64, B=4) == 0
+    cu = torch.tensor([0, 300, 300, 1000, 1064, 1193], dtype=torch.int32)   # 300, 0, 700, 64, 129
+    assert kda.checkpoint_count(1193, 64, cu_seqlens=cu) == 4 + 0 + 10 + 1 + 2
+    assert kda.checkpoint_count(1193, 256, cu_seqlens=cu) == 1 + 0 + 2 + 0 + 0
+
+
 def test_phase_entry_points_validate(lib):
     p = 0x10000
     assert lib.kda_fwd_intra(p, p, p, p, p, None, 0, 1, 64, 2, 32, 32, F32, p, 1 << 40,
