@@ -570,7 +570,9 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 1000 for the bench workload, whose step is "
+                         "~0.1 ms, so the timed region spans many clock samples; 300 otherwise)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["prefill", "long", "varlen", "decode", "few_chains"],
@@ -582,6 +584,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 1000 if (args.impl == "ours" and args.workload == "prefill") else 300
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))
