@@ -694,7 +694,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 //   1 MMA warp:          one elected lane issues, per chunk,
 //                          D_S        = M'(j) S   (M = 128 key rows, N = DVT, K = 128)
 //                          D_O[j & 1] = Q'(j) S   (M = 64 chunk rows)
-//                        on tcgen05, accumulating in tensor memory;
+//                        on tcgen05, accumulating in tensor memory; D_S by 32-row K
+//                        slabs as the state warps hand them over, and only then the
+//                        waits for D_O's ring slot and accumulator;
 //   4 output warps:      O = D_O + O0 for the chunk's rows (warp w reads tensor-memory
 //                        lane quarter w % 4), stored as bf16;
 //   1 producer warp:     bulk copies of the chunk records into two rings, the state
