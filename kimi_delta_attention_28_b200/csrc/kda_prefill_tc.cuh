@@ -955,7 +955,10 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
                     S[c + 1] = fmaf(gam, S[c + 1], r2.y + v[c + 1]);
                 }
             }
-            if (ckpt_on) {   // S now holds the state after `done` whole chunks of the sequence
+            if (j + 1 < nchunks) write_sb((j + 1) & 1);
+            // after the hand-off: its arrive releases this thread's earlier stores too, so
+            // checkpoint stores issued before it would hold up the next chunk's product
+            if (ckpt_on) {   // S holds the state after `done` whole chunks of the sequence
                 const int done = seg_lo + j + 1;
                 if (done % a.ckpt_chunks == 0 && done * C <= seq_tokens) {
                     const long long slot = ck_first + done / a.ckpt_chunks - 1;
@@ -969,7 +972,6 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
                     }
                 }
             }
-            if (j + 1 < nchunks) write_sb((j + 1) & 1);
         }
         float *dst = nullptr;
         if (map_mode)
