@@ -1,12 +1,18 @@
 #!/usr/bin/env python
 """KDA prefill throughput on B200 through the library's C ABI.
 
-Default workload: bf16 q/k/v, fp32 g/beta/state, B=2, H=8, T=4096,
-d_k = d_v = 128, nonzero initial state (seeded synthetic inputs).  A step is one
-full prefill (both kernels of the tensor-core path: the intra-chunk transform and
-the state pass) over one batch.  With --gpus N > 1 (launched by torchrun) every
-rank runs its own independent batch (weak scaling, no collective on the data
-path); the reported time is the max over ranks.
+Default (headline) workload: the 1M-token prefill -- bf16 q/k/v, fp32 g/beta/state,
+B=1, H=16, T=1,048,576, d_k = d_v = 128, zero initial state, seeded synthetic
+inputs (about 26 GB of inputs and outputs, far larger than L2).  A step is one
+full ``kda_fwd`` call (the intra-chunk kernel, then the state pass) over the whole
+batch.  On one GPU the same JSON line also carries, under ``workloads``, the other
+measured workloads with their own roofline and sampled parity: the B=2, H=8,
+T=4,096 prefill, the packed varlen prefill (16 sequences, H=32) and the decode
+step (256 sequences x 96 heads, fp32 state in place).
+
+With --gpus N > 1 (launched by torchrun) every rank runs its own independent batch
+of the headline workload (weak scaling, no collective on the data path); the
+reported time is the max over ranks.
 
 Prints ONE JSON line (rank 0).  --impl reference times the fp64 CPU oracle on a
 bounded sample of the same workload instead.
@@ -15,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import gc
 import json
 import math
 import os
@@ -29,8 +36,11 @@ if ROOT not in sys.path:
 
 METRIC = "KDA prefill tokens/s at d=128; achieved TFLOP/s and HBM GB/s vs B200 peak"
 L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
+L2_BYTES = 126 << 20
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+HEADLINE = "long"
+WORKLOAD_KEYS = ("prefill", "long", "varlen", "few_chains", "decode")
 
 
 def load_peaks():
@@ -129,12 +139,16 @@ def max_over_ranks(x, world, device):
     return float(t.item())
 
 
+def workload_of(name):
+    from kimi_delta_attention_28_b200 import workloads as W
+    return {"prefill": W.PREFILL, "long": W.LONG, "varlen": W.VARLEN,
+            "few_chains": W.FEW_CHAINS, "decode": W.DECODE}[name]
+
+
 def workload_inputs(name, device, seed_offset=0):
     from kimi_delta_attention_28_b200 import workloads as W
-    w = {"prefill": W.PREFILL, "long": W.LONG, "varlen": W.VARLEN,
-         "few_chains": W.FEW_CHAINS}[name]
     import dataclasses
-    w = dataclasses.replace(w, seed=w.seed + seed_offset)
+    w = dataclasses.replace(workload_of(name), seed=workload_of(name).seed + seed_offset)
     return w, W.make_workload(w, device)
 
 
@@ -145,294 +159,37 @@ def record_bytes():
 
 
 def algorithmic(w, inp):
-    """Units and algorithmic byte / flop counts of one prefill step."""
-    ntok = inp["q"].shape[0] * inp["q"].shape[1]          # tokens (each with H heads)
-    units = ntok * w.H                                       # token-heads
-    nseq = inp["h0"].shape[0] if inp["h0"] is not None else inp["q"].shape[0]
-    chains = nseq * w.H
-    state_bytes = w.dk * w.dv * 4
-    io = 2 if w.dtype.itemsize == 2 else 4
-    per_unit_in = 3 * w.dk * io + w.dk * 4 + 4               # q, k, v, g, beta
-    per_unit_out = w.dv * io                                 # o
-    compulsory = units * (per_unit_in + per_unit_out) + chains * state_bytes * (
-        2 if inp["h0"] is not None else 1)
-    rec_per_unit = record_bytes() / 64                       # intra-chunk record bytes per token-head
-    intra_bytes = units * (per_unit_in + rec_per_unit)
-    inter_bytes = units * (rec_per_unit + per_unit_out) + chains * state_bytes * (
-        2 if inp["h0"] is not None else 1)
-    flops_recurrence = units * 7 * w.dk * w.dv
-    return dict(ntok=ntok, units=units, chains=chains, compulsory=compulsory,
-                intra_bytes=intra_bytes, inter_bytes=inter_bytes, flops=flops_recurrence)
+    """Units and the compulsory byte / flop counts of one prefill step.
 
-
-def run_ours(args, world, rank, local):
-    import torch
-    import kimi_delta_attention_28_b200 as kda
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    kda.load_library()
-    w, inp = workload_inputs(args.workload, dev, seed_offset=rank)
+    Compulsory bytes are the method's own traffic: per token-head q, k, v
+    (3 d_k elements), g (fp32 d_k), beta (fp32) in and o out -- 1,540 B at
+    d = 128 in bf16 -- plus each (sequence, head) state read once (if given)
+    and written once.  The records the tensor-core path writes and reads back
+    are this implementation's intermediate and are reported separately."""
     B, T, H, dk = inp["q"].shape
     dv = inp["v"].shape[-1]
-    cu = inp["cu_seqlens"]
-    nseq = 0 if cu is None else cu.numel() - 1
-    N = B if cu is None else nseq
-    ws = torch.empty(kda.workspace_size(B, T, H, dk, dv, nseq, w.dtype), dtype=torch.uint8,
-                     device=dev)
-    o = torch.empty(B, T, H, dv, dtype=w.dtype, device=dev)
-    hT = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    # --ckpt-every N: every step also stores the state after each N tokens of every
-    # sequence (kda_fwd_checkpointed, prefix caching) into a preallocated buffer
-    ck = None
-    if args.ckpt_every > 0:
-        ck = torch.empty(kda.checkpoint_count(T, args.ckpt_every, B, cu), H, dk, dv,
-                         dtype=torch.float32, device=dev)
-
-    def step():
-        # one kda_fwd call: the prep kernel, then the state pass
-        if ck is not None:
-            kda.kda_fwd_checkpointed(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
-                                     inp["h0"], cu, ckpt_every=args.ckpt_every, ckpts=ck, o=o,
-                                     hT=hT, workspace=ws)
-        else:
-            kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], cu, o=o,
-                        hT=hT, workspace=ws)
-
-    def step_split(ev):
-        # the two phases as separate calls, an event between them: per-kernel times
-        ev[0].record(stream)
-        kda.kda_fwd_intra(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], cu, workspace=ws)
-        ev[1].record(stream)
-        kda.kda_fwd_inter(inp["h0"], cu, o, hT, B=B, T=T, H=H, dk=dk, dv=dv, dtype=w.dtype,
-                          workspace=ws)
-        ev[2].record(stream)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize(dev)
-
-    clocks = ClockSampler(dev)
-    clocks.start()
-    time.sleep(0.02)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    t_wall0 = time.perf_counter()
-    for i in range(args.steps):
-        flush.zero_()
-        ev = events[i]
-        ev[0].record(stream)
-        step()
-        ev[2].record(stream)
-    torch.cuda.synchronize(dev)
-    t_wall1 = time.perf_counter()
-    if world > 1:
-        torch.distributed.barrier()
-    clocks.stop()
-    total_ms = sum(e[0].elapsed_time(e[2]) for e in events)
-    # per-kernel split, outside the timed region
-    split = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
-             for _ in range(min(args.steps, 20))]
-    for ev in split:
-        flush.zero_()
-        step_split(ev)
-    torch.cuda.synchronize(dev)
-    intra = [e[0].elapsed_time(e[1]) for e in split]
-    inter = [e[1].elapsed_time(e[2]) for e in split]
-    nseg = kda.plan_segments(B, T, H, dk, dv, nseq, w.dtype)
-    launches_per_step = (2 if cu is not None else 1) + (1 if nseg <= 1 else 3)
-    total_ms = max_over_ranks(total_ms, world, dev)
-    ms_per_step = total_ms / args.steps
-    A = algorithmic(w, inp)
-
-    # end to end: pinned host inputs -> device, kda_fwd through the C ABI, results -> host.
-    # Every step copies its inputs in and its outputs (o, hT) out; consecutive steps
-    # are pipelined on three streams with two buffer sets, so step i+1's inputs go
-    # up while step i computes and step i-1's results come down.
-    e2e = None
-    if not args.no_e2e and ck is None:
-        host = {k_: (v_.cpu().pin_memory() if v_ is not None else None) for k_, v_ in inp.items()}
-        o_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
-        hT_h = [torch.empty(hT.shape, dtype=hT.dtype).pin_memory() for _ in range(2)]
-        dev_in = [{k_: (torch.empty_like(v_, device=dev) if v_ is not None else None)
-                   for k_, v_ in host.items()} for _ in range(2)]
-        o_d = [o, torch.empty_like(o)]
-        hT_d = [hT, torch.empty_like(hT)]
-        h2d = sum(v_.numel() * v_.element_size() for v_ in host.values() if v_ is not None)
-        d2h = o_h[0].numel() * o_h[0].element_size() + hT_h[0].numel() * hT_h[0].element_size()
-        s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        ev_up = [torch.cuda.Event() for _ in range(2)]
-        ev_comp = [torch.cuda.Event() for _ in range(2)]
-        ev_down = [torch.cuda.Event() for _ in range(2)]
-        for b_ in range(2):   # all buffers free at the start
-            ev_comp[b_].record(stream)
-            ev_down[b_].record(stream)
-
-        def e2e_step(i):
-            b_ = i & 1
-            with torch.cuda.stream(s_up):
-                s_up.wait_event(ev_comp[b_])           # step i-2 has read these inputs
-                for k_, v_ in host.items():
-                    if v_ is not None:
-                        dev_in[b_][k_].copy_(v_, non_blocking=True)
-                ev_up[b_].record(s_up)
-            stream.wait_event(ev_up[b_])
-            stream.wait_event(ev_down[b_])            # step i-2's results are down
-            d = dev_in[b_]
-            kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu_seqlens"],
-                        o=o_d[b_], hT=hT_d[b_], workspace=ws)
-            ev_comp[b_].record(stream)
-            with torch.cuda.stream(s_down):
-                s_down.wait_event(ev_comp[b_])
-                o_h[b_].copy_(o_d[b_], non_blocking=True)
-                hT_h[b_].copy_(hT_d[b_], non_blocking=True)
-                ev_down[b_].record(s_down)
-
-        for i in range(max(3, args.warmup // 4)):
-            e2e_step(i)
-        torch.cuda.synchronize(dev)
-        n_e2e = max(3, min(args.steps, 50))
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize(dev)
-        e0.record(s_up)
-        for i in range(n_e2e):
-            e2e_step(i)
-        for b_ in range(2):                           # everything down before the stop
-            s_down.wait_event(ev_down[b_])
-        e1.record(s_down)
-        torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        e2e_ms = max_over_ranks(e2e_ms, world, dev)
-        e2e = {"value": world * A["ntok"] / (e2e_ms * 1e-3), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e2e_ms,
-               "note": "inputs up and outputs down every step; steps pipelined on 3 streams"}
-
-    if rank != 0:
-        return None
-    hbm_peak, tf_peak, peak_src = load_peaks()
-    intra_ms = statistics.mean(intra)
-    inter_ms = statistics.mean(inter)
-    dom = "intra" if intra_ms >= inter_ms else "inter"
-    dom_ms = max(intra_ms, inter_ms)
-    dom_bytes = A["intra_bytes"] if dom == "intra" else A["inter_bytes"]
-    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    traffic = load_traffic(dom)
-    path_gbs = A["compulsory"] / (ms_per_step * 1e-3) / 1e9
-    out = {
-        "metric": METRIC,
-        "value": world * A["ntok"] / (ms_per_step * 1e-3),
-        "unit": "tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_per_step,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16" if w.dtype.itemsize == 2 else "f32",
-        "data": "synthetic (seeded; q,k L2-normalised, g=-5*sigmoid(N(-3,1)), beta=sigmoid(N(0,1)))",
-        "config": prefill_config(w, inp, world),
-        "roofline": {"bound": "hbm", "kernel": "kda_tc_prep_kernel" if dom == "intra"
-                     else "kda_tc_state_kernel", "achieved": achieved, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
-                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
-                     "algorithmic_bytes_per_launch": dom_bytes},
-        "path": {"compulsory_bytes_per_step": A["compulsory"], "hbm_gbs": path_gbs,
-                 "hbm_frac": path_gbs / hbm_peak,
-                 "tflops_recurrence": A["flops"] / (ms_per_step * 1e-3) / 1e12,
-                 "tensor_frac": A["flops"] / (ms_per_step * 1e-3) / 1e12 / tf_peak},
-        "kernels_ms": {"kda_tc_prep_kernel": intra_ms,
-                       ("kda_tc_state_kernel" if nseg <= 1 else
-                        f"state pass split in {nseg} segments (map, combine, output)"): inter_ms},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks.summary(t_wall0, t_wall1),
-        "e2e": e2e,
-    }
-    if ck is not None:
-        out["config"]["ckpt_every"] = args.ckpt_every
-        out["config"]["checkpoints_per_head"] = int(ck.shape[0])
-        out["kernels_ms_note"] = ("per-kernel split measured through kda_fwd_intra / "
-                                  "kda_fwd_inter, which store no checkpoints")
-    if world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_seconds)
-    return out
+    ntok = B * T                                             # tokens (each with H heads)
+    units = ntok * H                                         # token-heads
+    nseq = inp["cu_seqlens"].numel() - 1 if inp["cu_seqlens"] is not None else B
+    chains = nseq * H
+    state_bytes = dk * dv * 4
+    io = inp["q"].element_size()
+    per_unit_in = 3 * dk * io + dk * 4 + 4                   # q, k, v, g, beta
+    per_unit_out = dv * io                                   # o
+    states = chains * state_bytes * (2 if inp["h0"] is not None else 1)
+    compulsory = units * (per_unit_in + per_unit_out) + states
+    rec_per_unit = record_bytes() / 64                       # records per token-head
+    flops_recurrence = units * 7 * dk * dv
+    return dict(ntok=ntok, units=units, chains=chains, compulsory=compulsory,
+                per_unit_compulsory=per_unit_in + per_unit_out,
+                prep_compulsory=units * per_unit_in,
+                state_compulsory=units * per_unit_out + states,
+                intermediate=2 * units * rec_per_unit, flops=flops_recurrence)
 
 
-def run_ours_decode(args, world, rank, local):
-    """Decode workload: 256 sequences x 96 heads x d=128, fp32 state updated in
-    place; each step consumes fresh pre-generated inputs (the state, 1.6 GB, is
-    larger than L2, so no flush is needed)."""
-    import torch
-    import kimi_delta_attention_28_b200 as kda
-    from kimi_delta_attention_28_b200 import workloads as W
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    kda.load_library()
-    w = W.DECODE
-    nsteps = args.warmup + args.steps
-    inp = W.make_decode_inputs(w.B, w.H, w.dk, w.dv, nsteps, w.dtype, w.seed + rank, dev)
-    S = inp["S"]
-    o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def step(t):
-        kda.kda_decode_step(inp["q"][t], inp["k"][t], inp["v"][t], inp["g"][t], inp["beta"][t],
-                            S, o)
-
-    for t in range(args.warmup):
-        step(t)
-    torch.cuda.synchronize(dev)
-    clocks = ClockSampler(dev)
-    clocks.start()
-    time.sleep(0.02)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    t_wall0 = time.perf_counter()
-    ev[0].record(stream)
-    for i in range(args.steps):
-        step(args.warmup + i)
-        ev[i + 1].record(stream)
-    torch.cuda.synchronize(dev)
-    t_wall1 = time.perf_counter()
-    if world > 1:
-        torch.distributed.barrier()
-    clocks.stop()
-    total_ms = ev[0].elapsed_time(ev[-1])
-    total_ms = max_over_ranks(total_ms, world, dev)
-    if rank != 0:
-        return None
-    ms = total_ms / args.steps
-    units = w.B * w.H
-    per_unit = 2 * w.dk * w.dv * 4 + 3 * w.dk * 2 + w.dk * 4 + 4 + w.dv * 2
-    bytes_step = units * per_unit
-    hbm_peak, _, peak_src = load_peaks()
-    gbs = bytes_step / (ms * 1e-3) / 1e9
-    return {
-        "metric": "KDA decode steps/s (256 sequences x 96 heads, d=128, fp32 state in place)",
-        "value": world * 1e3 / ms, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
-        "config": {"workload": w.name, "N": w.B, "H": w.H, "dk": w.dk, "dv": w.dv,
-                   "l2": "state (1.6 GB) larger than L2; no flush"},
-        "roofline": {"bound": "hbm", "kernel": "kda_decode_kernel", "achieved": gbs,
-                     "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
-                     "traffic": load_traffic("decode"),
-                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
-                     "algorithmic_bytes_per_launch": bytes_step},
-        "gpu_launches": args.steps,
-        "clocks": clocks.summary(t_wall0, t_wall1),
-    }
-
-
+# ---------------------------------------------------------------------------
+# committed DRAM traffic (ncu) per unit, valid only for the kernel sources it was taken on
+# ---------------------------------------------------------------------------
 def _strip_comments(text):
     """C/C++ source without comments and blank lines (string literals are kept)."""
     import re
@@ -454,19 +211,282 @@ def kernel_source_sha(src=None):
     return h.hexdigest()
 
 
-def load_traffic(which):
-    """DRAM bytes (read + write) per launch of kernel `which`, from the committed
-    ncu summary profiles/traffic.json -- only if it was taken on the current
-    kernel sources (same sha256), else None."""
+def load_traffic(kernel, units):
+    """DRAM bytes (read + write) of `kernel` for `units` units (token-heads for the
+    prefill kernels, (sequence, head) chains for decode): the per-unit figure of the
+    committed ncu summary profiles/traffic.json scaled by the units -- only if that
+    summary was taken on the current kernel sources (same sha256), else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
         if d.get("kernel_source_sha256") != kernel_source_sha():
             return None
-        return d["per_launch_dram_bytes"].get(which)
+        per = d["dram_bytes_per_unit"].get(kernel)
+        return None if per is None else float(per) * units
     except Exception:  # noqa: BLE001
         return None
+
+
+# ---------------------------------------------------------------------------
+# prefill
+# ---------------------------------------------------------------------------
+def prefill_config(w, inp, world):
+    """The `config` object of a prefill workload (shared by both arms)."""
+    B, T, H, dk = inp["q"].shape
+    nseq = 0 if inp["cu_seqlens"] is None else inp["cu_seqlens"].numel() - 1
+    big = _input_bytes(inp) > 4 * L2_BYTES
+    return {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": inp["v"].shape[-1],
+            "h0": "N(0, 0.1^2)" if inp["h0"] is not None else "zeros",
+            "varlen_seqs": nseq,
+            "l2": ("inputs (%.1f GB) far larger than L2; no flush" % (_input_bytes(inp) / 1e9))
+            if big else "flushed between steps (256 MiB write)",
+            "parallelism": f"replicas x{world} (independent batches)"}
+
+
+def _input_bytes(inp):
+    return sum(v.numel() * v.element_size() for v in inp.values() if v is not None)
+
+
+def measure_prefill(name, steps, warmup, world=1, rank=0, local=0, e2e=True, cpu=True,
+                    cpu_seconds=10.0, ckpt_every=0):
+    """Time `steps` kda_fwd calls on workload `name`; returns the JSON object (rank 0)."""
+    import torch
+    import kimi_delta_attention_28_b200 as kda
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    kda.load_library()
+    w, inp = workload_inputs(name, dev, seed_offset=rank)
+    B, T, H, dk = inp["q"].shape
+    dv = inp["v"].shape[-1]
+    cu = inp["cu_seqlens"]
+    nseq = 0 if cu is None else cu.numel() - 1
+    N = B if cu is None else nseq
+    ws = torch.empty(kda.workspace_size(B, T, H, dk, dv, nseq, w.dtype), dtype=torch.uint8,
+                     device=dev)
+    o = torch.empty(B, T, H, dv, dtype=w.dtype, device=dev)
+    hT = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    big = _input_bytes(inp) > 4 * L2_BYTES
+    flush = None if big else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # ckpt_every > 0: every step also stores the state after each ckpt_every tokens
+    # of every sequence (kda_fwd_checkpointed, prefix caching)
+    ck = None
+    if ckpt_every > 0:
+        ck = torch.empty(kda.checkpoint_count(T, ckpt_every, B, cu), H, dk, dv,
+                         dtype=torch.float32, device=dev)
+
+    def step():
+        if ck is not None:
+            kda.kda_fwd_checkpointed(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                     inp["h0"], cu, ckpt_every=ckpt_every, ckpts=ck, o=o,
+                                     hT=hT, workspace=ws)
+        else:
+            kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], cu, o=o,
+                        hT=hT, workspace=ws)
+
+    def step_split(ev):
+        # the two phases as separate calls, an event between them: per-kernel times
+        ev[0].record(stream)
+        kda.kda_fwd_intra(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], cu, workspace=ws)
+        ev[1].record(stream)
+        kda.kda_fwd_inter(inp["h0"], cu, o, hT, B=B, T=T, H=H, dk=dk, dv=dv, dtype=w.dtype,
+                          workspace=ws)
+        ev[2].record(stream)
+
+    def flush_l2():
+        if flush is not None:
+            flush.zero_()
+
+    for _ in range(warmup):
+        flush_l2()
+        step()
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.02)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.perf_counter()
+    for i in range(steps):
+        flush_l2()
+        events[i][0].record(stream)
+        step()
+        events[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.perf_counter()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.stop()
+    total_ms = sum(e[0].elapsed_time(e[1]) for e in events)
+    # per-kernel split, outside the timed region
+    nsplit = min(steps, 20 if not big else 5)
+    split = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nsplit)]
+    for ev in split:
+        flush_l2()
+        step_split(ev)
+    torch.cuda.synchronize(dev)
+    intra_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in split)
+    inter_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in split)
+    nseg = kda.plan_segments(B, T, H, dk, dv, nseq, w.dtype)
+    launches_per_step = (2 if cu is not None else 1) + (1 if nseg <= 1 else 3)
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_per_step = total_ms / steps
+    A = algorithmic(w, inp)
+    # the outputs of the timed steps, for the parity sample of the CPU leg
+    o_host = o.cpu() if rank == 0 and cpu and world == 1 else None
+    hT_host = hT.cpu() if o_host is not None else None
+
+    e2e_obj = None
+    if e2e and ck is None:
+        e2e_obj = measure_e2e(kda, w, inp, o, hT, ws, dev, stream, world, A["ntok"],
+                              n_steps=3 if big else max(3, min(steps, 50)))
+    if rank != 0:
+        return None
+
+    hbm_peak, tf_peak, peak_src = load_peaks()
+    call_gbs = A["compulsory"] / (ms_per_step * 1e-3) / 1e9
+    t_prep = load_traffic("kda_tc_prep_kernel", A["units"])
+    t_state = load_traffic("kda_tc_state_kernel", A["units"]) if nseg <= 1 else None
+    traffic = (t_prep + t_state) if (t_prep is not None and t_state is not None) else None
+    state_name = ("kda_tc_state_kernel" if nseg <= 1 else
+                  f"state pass split in {nseg} segments (map, combine, output)")
+    out = {
+        "metric": METRIC,
+        "value": world * A["ntok"] / (ms_per_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype.itemsize == 2 else "f32",
+        "data": "synthetic (seeded; q,k L2-normalised, g=-5*sigmoid(N(-3,1)), beta=sigmoid(N(0,1)))",
+        "config": prefill_config(w, inp, world),
+        # the whole kda_fwd call (its two kernels run back to back on one stream) against
+        # the method's compulsory bytes: 1,540 B per token-head plus the states
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "kda_fwd call (kda_tc_prep_kernel + %s)" % state_name,
+            "achieved": call_gbs, "peak": hbm_peak, "unit": "GB/s",
+            "frac": call_gbs / hbm_peak,
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": A["compulsory"],
+            "algorithmic_bytes_rule": "compulsory: %d B per token-head (q,k,v,g,beta in; o out) "
+                                      "x %d token-heads + states %d B" % (
+                                          A["per_unit_compulsory"], A["units"],
+                                          A["compulsory"] - A["units"] * A["per_unit_compulsory"]),
+            "intermediate_bytes": A["intermediate"],
+            "intermediate_rule": "records (%d B per 64-token chunk and head) written by the "
+                                 "prep kernel and read back by the state pass" % record_bytes(),
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+            "per_kernel": {
+                "kda_tc_prep_kernel": {
+                    "ms": intra_ms,
+                    "compulsory_bytes": A["prep_compulsory"],
+                    "frac": A["prep_compulsory"] / (intra_ms * 1e-3) / 1e9 / hbm_peak,
+                    "dram_bytes": t_prep},
+                state_name: {
+                    "ms": inter_ms,
+                    "compulsory_bytes": A["state_compulsory"],
+                    "frac": A["state_compulsory"] / (inter_ms * 1e-3) / 1e9 / hbm_peak,
+                    "dram_bytes": t_state},
+                "dominant": "kda_tc_prep_kernel" if intra_ms >= inter_ms else state_name,
+                "dominant_frac_all_compulsory_over_its_time":
+                    A["compulsory"] / (max(intra_ms, inter_ms) * 1e-3) / 1e9 / hbm_peak,
+            },
+        },
+        "path": {"compulsory_bytes_per_step": A["compulsory"], "hbm_gbs": call_gbs,
+                 "hbm_frac": call_gbs / hbm_peak,
+                 "tflops_recurrence": A["flops"] / (ms_per_step * 1e-3) / 1e12,
+                 "tensor_frac": A["flops"] / (ms_per_step * 1e-3) / 1e12 / tf_peak},
+        "kernels_ms": {"kda_tc_prep_kernel": intra_ms, state_name: inter_ms},
+        "gpu_launches": launches_per_step * steps,
+        "clocks": clocks.summary(t_wall0, t_wall1),
+        "e2e": e2e_obj,
+    }
+    if ck is not None:
+        out["config"]["ckpt_every"] = ckpt_every
+        out["config"]["checkpoints_per_head"] = int(ck.shape[0])
+        out["kernels_ms_note"] = ("per-kernel split measured through kda_fwd_intra / "
+                                  "kda_fwd_inter, which store no checkpoints")
+    if o_host is not None:
+        del o, hT, ws
+        out["cpu_baseline"] = cpu_baseline(w, inp, o_host, hT_host, budget_s=cpu_seconds)
+    return out
+
+
+def measure_e2e(kda, w, inp, o, hT, ws, dev, stream, world, ntok, n_steps):
+    """End to end through the C ABI with host buffers: every step copies its inputs up
+    from pinned host memory, runs kda_fwd and copies o and hT down.  Consecutive steps
+    are pipelined on three streams with two device buffer sets (step i+1's inputs go
+    up while step i computes and step i-1's results come down)."""
+    import torch
+    host = {k_: (torch.empty(v_.shape, dtype=v_.dtype, pin_memory=True).copy_(v_)
+                 if v_ is not None else None) for k_, v_ in inp.items()}
+    o_h = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for _ in range(2)]
+    hT_h = [torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True) for _ in range(2)]
+    dev_in = [inp, {k_: (torch.empty_like(v_) if v_ is not None else None)
+                    for k_, v_ in inp.items()}]
+    o_d = [o, torch.empty_like(o)]
+    hT_d = [hT, torch.empty_like(hT)]
+    h2d = sum(v_.numel() * v_.element_size() for v_ in host.values() if v_ is not None)
+    d2h = o_h[0].numel() * o_h[0].element_size() + hT_h[0].numel() * hT_h[0].element_size()
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
+    for b_ in range(2):   # all buffers free at the start
+        ev_comp[b_].record(stream)
+        ev_down[b_].record(stream)
+
+    def e2e_step(i):
+        b_ = i & 1
+        with torch.cuda.stream(s_up):
+            s_up.wait_event(ev_comp[b_])           # step i-2 has read these inputs
+            for k_, v_ in host.items():
+                if v_ is not None:
+                    dev_in[b_][k_].copy_(v_, non_blocking=True)
+            ev_up[b_].record(s_up)
+        stream.wait_event(ev_up[b_])
+        stream.wait_event(ev_down[b_])            # step i-2's results are down
+        d = dev_in[b_]
+        kda.kda_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], d["cu_seqlens"],
+                    o=o_d[b_], hT=hT_d[b_], workspace=ws)
+        ev_comp[b_].record(stream)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(ev_comp[b_])
+            o_h[b_].copy_(o_d[b_], non_blocking=True)
+            hT_h[b_].copy_(hT_d[b_], non_blocking=True)
+            ev_down[b_].record(s_down)
+
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(s_up)
+    for i in range(n_steps):
+        e2e_step(i)
+    for b_ in range(2):                           # everything down before the stop
+        s_down.wait_event(ev_down[b_])
+    e1.record(s_down)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / n_steps
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    del dev_in[1], o_d[1], hT_d[1]
+    return {"value": world * ntok / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": e2e_ms, "steps": n_steps,
+            "note": "inputs up from pinned host memory and o, hT down every step; steps "
+                    "pipelined on 3 streams with 2 device buffer sets"}
 
 
 def host_f64(inp):
@@ -482,51 +502,213 @@ def host_f64(inp):
     return out
 
 
-def cpu_baseline(w, inp, budget_s=10.0, chains_per_step=None):
-    """Time the fp64 oracle (as it stands) on the host cores on whole chains of
-    this workload: tokens/s in the same unit as the GPU number."""
+def _err(got, ref):
+    import numpy as np
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return {"rel_l2": float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)),
+            "max_abs": float(np.abs(got - ref).max()) if got.size else 0.0}
+
+
+PARITY_TOL = {"bf16": "rel-L2 <= 1e-2 and max-abs <= 5e-2", "f32": "rel-L2 <= 1e-4"}
+
+
+def cpu_baseline(w, inp, o_gpu, hT_gpu, budget_s=10.0):
+    """The fp64 oracle (as it stands) on the host cores, on whole (sequence, head) chains
+    of this workload from their true initial states: tokens/s in the GPU number's unit
+    (tokens that carry all H heads).  The oracle's outputs for the sample are also
+    compared with the GPU's outputs of the timed steps (o_gpu, hT_gpu, on the host)."""
+    import numpy as np
     import oracle
-    h = host_f64(inp)
+    h = {k_: v_ for k_, v_ in inp.items()}
     B, T, H, dk = h["q"].shape
-    q, k, v, g, beta = (h[n].reshape(B * T, H, -1) if n != "beta" else h[n].reshape(B * T, H)
-                        for n in ("q", "k", "v", "g", "beta"))
-    cu = h["cu_seqlens"] if h["cu_seqlens"] is not None else (
-        __import__("numpy").arange(B + 1) * T)
-    reps, elapsed, used = 0, 0.0, 1
-    while elapsed < budget_s and reps < 50:
+    cu = h["cu_seqlens"]
+    o_g = o_gpu.double().numpy()
+    hT_g = hT_gpu.double().numpy()
+    parity = {"tolerance": PARITY_TOL["bf16" if w.dtype.itemsize == 2 else "f32"]}
+    if cu is not None:
+        # packed: one head (0) of every sequence, whole sequences
+        hh = 0
+        sl = lambda x: np.ascontiguousarray(x[0, :, hh:hh + 1].detach().cpu().double().numpy())  # noqa: E731
+        args_ = (sl(h["q"]), sl(h["k"]), sl(h["v"]), sl(h["g"]),
+                 np.ascontiguousarray(h["beta"][0, :, hh:hh + 1].cpu().double().numpy()),
+                 None if h["h0"] is None else
+                 np.ascontiguousarray(h["h0"][:, hh:hh + 1].cpu().double().numpy()),
+                 cu.cpu().numpy().astype(np.int64))
         t0 = time.perf_counter()
-        _, _, used = oracle.kda_fwd_packed(q, k, v, g, beta, h["h0"], cu)
-        elapsed += time.perf_counter() - t0
-        reps += 1
-    ntok = B * T
-    return {"value": ntok * reps / elapsed, "unit": "tokens/s", "cores": int(used),
-            "kind": "oracle",
-            "sample": f"whole workload ({B}x{T} tokens x {H} heads) x {reps} runs, "
-                      f"{elapsed:.1f} s; fp64 token-by-token C, OpenMP over (sequence, head)"}
+        o_ref, hT_ref, used = oracle.kda_fwd_packed(*args_)
+        el = time.perf_counter() - t0
+        ntok_equiv = T / H
+        parity["o"] = _err(o_g[0, :, hh:hh + 1], o_ref)
+        parity["hT"] = _err(hT_g[:, hh:hh + 1], hT_ref)
+        parity["sample"] = f"head {hh} of all {cu.numel() - 1} packed sequences, whole"
+        sample = (f"head {hh} of all {cu.numel() - 1} packed sequences ({T} tokens), "
+                  f"{el:.1f} s; fp64 token-by-token C, OpenMP over sequences")
+        return {"value": ntok_equiv / el, "unit": "tokens/s", "cores": int(used),
+                "kind": "oracle", "sample": sample, "parity": parity}
+    # fixed length: all heads of sequence 0 over its first Ts tokens (exact: the chains
+    # start from h0 at token 0), Ts sized to about budget_s of oracle time
+    Ts = min(T, 1024)
+    while True:
+        sl = lambda x, n=Ts: np.ascontiguousarray(x[0, :n].detach().cpu().double().numpy())  # noqa: E731
+        h0 = None if h["h0"] is None else np.ascontiguousarray(h["h0"][:1].cpu().double().numpy())
+        t0 = time.perf_counter()
+        o_ref, hT_ref, used = oracle.kda_fwd_packed(sl(h["q"]), sl(h["k"]), sl(h["v"]),
+                                                    sl(h["g"]), sl(h["beta"]), h0,
+                                                    np.array([0, Ts]))
+        el = time.perf_counter() - t0
+        if Ts >= T or el * 3 > budget_s:
+            break
+        Ts = min(T, int(Ts * min(8.0, max(2.0, budget_s / max(el, 1e-3) / 2))))
+    parity["o"] = _err(o_g[0, :Ts], o_ref)
+    parity["sample"] = f"all {H} heads of sequence 0, tokens [0, {Ts})"
+    if Ts >= T:
+        parity["hT"] = _err(hT_g[:1], hT_ref)
+    else:
+        # the final block and final state by a window restarted from zero L tokens
+        # earlier: every transition has operator norm <= max_c exp(g_tc), so the
+        # truncation error is at most exp(sum of per-token max g) times the state norm
+        L, blk = 4096, 64
+        a, s = T - blk - L, T - blk
+        gmax = inp["g"][0, a:s].amax(dim=-1).double().sum(dim=0).max().item()
+        snorm = T * float(inp["v"].abs().max()) * math.sqrt(w.dv)
+        slw = lambda x: np.ascontiguousarray(x[0, a:T].detach().cpu().double().numpy())  # noqa: E731
+        ow, hw, _ = oracle.kda_fwd_packed(slw(inp["q"]), slw(inp["k"]), slw(inp["v"]),
+                                          slw(inp["g"]), slw(inp["beta"]), None,
+                                          np.array([0, T - a]))
+        parity["o_last_block"] = _err(o_g[0, s:T], ow[L:])
+        if h["h0"] is None or B == 1:
+            parity["hT"] = _err(hT_g[:1], hw)
+        parity["window_truncation_bound"] = math.exp(gmax) * snorm
+        parity["sample"] += (f"; tokens [{s}, {T}) and the final states by a {L}-token "
+                             "window restarted from zero (truncation bound above)")
+    sample = (f"all {H} heads of sequence 0 over tokens [0, {Ts}) from h0, {el:.1f} s; "
+              "fp64 token-by-token C, OpenMP over heads")
+    return {"value": Ts / el, "unit": "tokens/s", "cores": int(used), "kind": "oracle",
+            "sample": sample, "parity": parity}
 
 
-def prefill_config(w, inp, world):
-    """The `config` object of a prefill workload (shared by both arms)."""
-    B, T, H, dk = inp["q"].shape
-    nseq = 0 if inp["cu_seqlens"] is None else inp["cu_seqlens"].numel() - 1
-    return {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": inp["v"].shape[-1],
-            "h0": "N(0, 0.1^2)" if inp["h0"] is not None else "zeros",
-            "varlen_seqs": nseq, "l2": "flushed between steps (256 MiB write)",
-            "parallelism": f"replicas x{world} (independent batches)"}
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+def measure_decode(steps, warmup, world=1, rank=0, local=0, cpu=True):
+    """Decode workload: 256 sequences x 96 heads x d=128, fp32 state updated in
+    place; each step consumes fresh pre-generated inputs (the state, 1.6 GB, is
+    larger than L2, so no flush is needed)."""
+    import numpy as np
+    import torch
+    import kimi_delta_attention_28_b200 as kda
+    from kimi_delta_attention_28_b200 import workloads as W
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    kda.load_library()
+    w = W.DECODE
+    nsteps = warmup + steps
+    inp = W.make_decode_inputs(w.B, w.H, w.dk, w.dv, nsteps, w.dtype, w.seed + rank, dev)
+    S = inp["S"].clone()
+    o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    rng = np.random.default_rng(1)
+    pairs = rng.choice(w.B * w.H, size=64, replace=False)
+    n_idx = torch.tensor(pairs // w.H, device=dev)
+    h_idx = torch.tensor(pairs % w.H, device=dev)
+    o_last = None
+
+    def step(t):
+        kda.kda_decode_step(inp["q"][t], inp["k"][t], inp["v"][t], inp["g"][t], inp["beta"][t],
+                            S, o)
+
+    for t in range(warmup):
+        step(t)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.02)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.perf_counter()
+    ev[0].record(stream)
+    for i in range(steps):
+        step(warmup + i)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.perf_counter()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.stop()
+    o_last = o[n_idx, h_idx].cpu()
+    total_ms = ev[0].elapsed_time(ev[-1])
+    total_ms = max_over_ranks(total_ms, world, dev)
+    if rank != 0:
+        return None
+    ms = total_ms / steps
+    units = w.B * w.H
+    per_unit = 2 * w.dk * w.dv * 4 + 3 * w.dk * 2 + w.dk * 4 + 4 + w.dv * 2
+    bytes_step = units * per_unit
+    hbm_peak, _, peak_src = load_peaks()
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    out = {
+        "metric": "KDA decode steps/s (256 sequences x 96 heads, d=128, fp32 state in place)",
+        "value": world * 1e3 / ms, "unit": "steps/s", "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "N": w.B, "H": w.H, "dk": w.dk, "dv": w.dv,
+                   "l2": "state (1.6 GB) larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "kernel": "kda_decode_kernel", "achieved": gbs,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                     "traffic": load_traffic("kda_decode_kernel", units),
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+                     "algorithmic_bytes_per_launch": bytes_step,
+                     "algorithmic_bytes_rule": "per (sequence, head): state read + write "
+                                               "2 x 64 KiB, q,k,v bf16, g fp32, beta, o bf16"},
+        "gpu_launches": steps,
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+    if cpu and world == 1:
+        out["cpu_baseline"] = decode_cpu_baseline(w, inp, S, o_last, pairs, nsteps)
+    return out
 
 
+def decode_cpu_baseline(w, inp, S_gpu, o_last, pairs, nsteps):
+    """The oracle on 64 sampled (sequence, head) chains over every step the GPU ran
+    (chains are independent, so the check is exact for them): steps/s scaled to the
+    whole batch, and the parity of the final outputs and states of those chains."""
+    import oracle
+    n_idx = pairs // w.H
+    h_idx = pairs % w.H
+    pick = lambda x: x[:, n_idx, h_idx].unsqueeze(2).transpose(0, 1).contiguous()  # noqa: E731
+    q, k, v, g = (pick(inp[n]).cpu() for n in ("q", "k", "v", "g"))
+    beta = inp["beta"][:, n_idx, h_idx].transpose(0, 1).unsqueeze(2).contiguous().cpu()
+    S0 = inp["S"][n_idx, h_idx].unsqueeze(1).contiguous().cpu()
+    t0 = time.perf_counter()
+    o_ref, S_ref = oracle.kda_fwd(q, k, v, g, beta, S0)
+    el = time.perf_counter() - t0
+    used = min(len(pairs), oracle.threads_available())
+    S_g = S_gpu[n_idx, h_idx].unsqueeze(1).cpu()
+    parity = {"tolerance": PARITY_TOL["bf16"],
+              "o_last_step": _err(o_last.double().numpy(), o_ref[:, -1, 0]),
+              "S": _err(S_g.double().numpy(), S_ref),
+              "sample": f"{len(pairs)} sampled (sequence, head) chains over all {nsteps} steps"}
+    steps_per_s = nsteps / el * len(pairs) / (w.B * w.H)
+    return {"value": steps_per_s, "unit": "steps/s", "cores": int(used), "kind": "oracle",
+            "sample": f"{len(pairs)} of {w.B * w.H} (sequence, head) chains x {nsteps} steps, "
+                      f"{el:.1f} s, scaled to the whole batch", "parity": parity}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle on a bounded sample of the workload
+# ---------------------------------------------------------------------------
 def run_reference(args, world, rank):
     """The oracle on a bounded sample of the workload, timed per step."""
     import numpy as np
-    import torch
     import oracle
     from kimi_delta_attention_28_b200 import workloads as W
-    w = {"prefill": W.PREFILL, "long": W.LONG, "varlen": W.VARLEN,
-         "few_chains": W.FEW_CHAINS}[args.workload]
+    w = workload_of(args.workload)
     inp = W.make_workload(w, "cpu")
     h = host_f64(inp)
     B, T, H, dk = h["q"].shape
-    dv = h["v"].shape[-1]
     # sample: whole (sequence, head) chains over the first Ts tokens of sequence 0,
     # sized so warmup + steps finish in about args.ref_seconds
     Ts = min(T, 4096)
@@ -567,16 +749,28 @@ def run_reference(args, world, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+def _free_device_memory():
+    import torch
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def default_steps(workload):
+    """Timed steps when --steps is not given (about a second of timed work or less)."""
+    return {"long": 10, "few_chains": 100, "varlen": 100, "prefill": 1000, "decode": 300}[workload]
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default: 1000 for the bench workload, whose step is "
-                         "~0.1 ms, so the timed region spans many clock samples; 300 otherwise)")
-    ap.add_argument("--warmup", type=int, default=20)
+                    help="timed steps (default: about a second of timed work for the workload)")
+    ap.add_argument("--warmup", type=int, default=None, help="untimed warm-up steps (>= 3)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "long", "varlen", "decode", "few_chains"],
-                    default="prefill")
+    ap.add_argument("--workload", choices=list(WORKLOAD_KEYS), default=HEADLINE)
+    ap.add_argument("--no-nested", action="store_true",
+                    help="skip the other workloads nested under `workloads` (one GPU only)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ckpt-every", type=int, default=0,
                     help="prefill workloads: also store the state every N tokens (multiple of 64)")
@@ -585,7 +779,9 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = 1000 if (args.impl == "ours" and args.workload == "prefill") else 300
+        args.steps = default_steps(args.workload) if args.impl == "ours" else 3
+    if args.warmup is None:
+        args.warmup = 3 if args.workload == "long" else 20
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -598,11 +794,32 @@ def main():
         print(json.dumps(run_reference(args, world, rank)), flush=True)
         return 0
     world, rank, local = dist_setup(args)
+    cpu = not args.no_cpu_baseline
     try:
         if args.workload == "decode":
-            out = run_ours_decode(args, world, rank, local)
+            out = measure_decode(args.steps, args.warmup, world, rank, local, cpu=cpu)
         else:
-            out = run_ours(args, world, rank, local)
+            out = measure_prefill(args.workload, args.steps, args.warmup, world, rank, local,
+                                  e2e=not args.no_e2e, cpu=cpu, cpu_seconds=args.cpu_seconds,
+                                  ckpt_every=args.ckpt_every)
+        if world == 1 and not args.no_nested and args.workload == HEADLINE and out is not None:
+            # the other workloads, each with its own roofline and parity sample
+            nested = {}
+            for name in ("prefill", "varlen"):
+                _free_device_memory()
+                r = measure_prefill(name, default_steps(name), 20, e2e=False, cpu=cpu,
+                                    cpu_seconds=min(args.cpu_seconds, 5.0))
+                nested[name] = {k_: r[k_] for k_ in ("value", "unit", "ms_per_step", "steps",
+                                                      "warmup", "config", "roofline", "path",
+                                                      "kernels_ms", "gpu_launches", "clocks",
+                                                      "cpu_baseline") if k_ in r}
+            _free_device_memory()
+            r = measure_decode(200, 20, cpu=cpu)
+            nested["decode"] = {k_: r[k_] for k_ in ("metric", "value", "unit", "ms_per_step",
+                                                      "steps", "warmup", "config", "roofline",
+                                                      "gpu_launches", "clocks", "cpu_baseline")
+                                if k_ in r}
+            out["workloads"] = nested
         if out is not None:
             print(json.dumps(out), flush=True)
     finally:

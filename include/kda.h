@@ -53,7 +53,8 @@ typedef enum {
     KDA_ERR_DEVICE_TIMEOUT = 6,       /* a bounded device-side wait gave up        */
     KDA_ERR_BAD_SEQLENS = 7,          /* cu_seqlens not monotone / out of range    */
     KDA_ERR_EXCEEDS_STATIC_SCRATCH = 8, /* kda_fwd_noalloc: problem too large      */
-    KDA_ERR_CHECKPOINT_CAPACITY = 9   /* kda_fwd_checkpointed: more checkpoints than slots */
+    KDA_ERR_CHECKPOINT_CAPACITY = 9,  /* kda_fwd_checkpointed: more checkpoints than slots */
+    KDA_ERR_DEBUG_BOUNDS = 10         /* debug build: a device-side bounds check failed */
 } kda_status;
 
 typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
@@ -63,6 +64,18 @@ int kda_version(void);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *kda_status_string(kda_status s);
+
+/*
+ * How this copy of the library was built.  KDA_BUILD_DEBUG_CHECKS is set in the
+ * debug build (libkda_b200_debug.so, compiled with -DKDA_DEBUG=1): at the top of
+ * every prefill kernel the indices that address global memory (chunk table
+ * entries, sequence token ranges, record slots) are checked against their
+ * buffers' extents, and a failed check makes the affected CTAs return before
+ * their first access and the call's device error KDA_ERR_DEBUG_BOUNDS, instead of
+ * an out-of-bounds access.  The release build (libkda_b200.so) has no checks.
+ */
+#define KDA_BUILD_DEBUG_CHECKS 1
+int kda_build_flags(void);
 
 /*
  * Bytes of device workspace that kda_fwd needs for these sizes.  The
@@ -245,8 +258,12 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
  *     call returns KDA_ERR_EXCEEDS_STATIC_SCRATCH and launches nothing.  32 MiB
  *     holds 339 (64-token chunk, head) records, e.g. B = 1, H = 8, T = 2,688.
  *   - Set-up: the first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it.  Make that
- *     first call on each device before any stream capture begins.
+ *     (cudaGetSymbolAddress, with that device current) and caches it for that
+ *     device's current CUDA context; a new context on the device (after
+ *     cudaDeviceReset, for instance) gets a fresh lookup on its first call, and a
+ *     lookup that fails is not cached (the call returns KDA_ERR_CUDA and the next
+ *     call tries again).  Make the first call on each device, and in each new
+ *     context, before any stream capture begins.
  *   - Sharing: every call on a device uses the same array, which keeps whatever
  *     the previous call left in it.  Nothing in it has to start at zero, because
  *     each call writes every scratch byte it later reads.  Calls whose work
@@ -263,8 +280,9 @@ kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const fl
 /*
  * Synchronises `stream`, then reads and clears the library's device error word
  * (cu_seqlens violations, bounded waits that gave up, checkpoints past the
- * capacity).  Returns KDA_OK, KDA_ERR_BAD_SEQLENS, KDA_ERR_DEVICE_TIMEOUT,
- * KDA_ERR_CHECKPOINT_CAPACITY or KDA_ERR_CUDA.
+ * capacity, debug bounds checks).  Returns KDA_OK, KDA_ERR_BAD_SEQLENS,
+ * KDA_ERR_DEVICE_TIMEOUT, KDA_ERR_CHECKPOINT_CAPACITY, KDA_ERR_DEBUG_BOUNDS or
+ * KDA_ERR_CUDA.
  */
 kda_status kda_get_last_device_error(void *stream);
 

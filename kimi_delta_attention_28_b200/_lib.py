@@ -14,6 +14,9 @@ import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkda_b200.so")
+# The same library built with device-side bounds checks (-DKDA_DEBUG=1); load it with
+# load_library(DEBUG_LIB_PATH) before any other call.
+DEBUG_LIB_PATH = os.path.join(HERE, "libkda_b200_debug.so")
 
 KDA_DTYPE_F32 = 0
 KDA_DTYPE_BF16 = 1
@@ -21,7 +24,8 @@ KDA_DTYPE_BF16 = 1
 STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED_SHAPE",
           3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_WORKSPACE_TOO_SMALL", 5: "KDA_ERR_CUDA",
           6: "KDA_ERR_DEVICE_TIMEOUT", 7: "KDA_ERR_BAD_SEQLENS",
-          8: "KDA_ERR_EXCEEDS_STATIC_SCRATCH", 9: "KDA_ERR_CHECKPOINT_CAPACITY"}
+          8: "KDA_ERR_EXCEEDS_STATIC_SCRATCH", 9: "KDA_ERR_CHECKPOINT_CAPACITY",
+          10: "KDA_ERR_DEBUG_BOUNDS"}
 
 # Size of the static scratch array behind kda_fwd_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -30,6 +34,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 _VP, _SZ, _I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
 SIGNATURES = {
     "kda_version": ([], _I),
+    "kda_build_flags": ([], _I),
     "kda_status_string": ([_I], ctypes.c_char_p),
     "kda_fwd_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "kda_fwd": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP,

@@ -24,6 +24,7 @@ namespace {
 constexpr int ERRBIT_SEQLENS = 1;
 constexpr int ERRBIT_TIMEOUT = 2;
 constexpr int ERRBIT_CKPT = 4;
+constexpr int ERRBIT_BOUNDS = kda::kErrBoundsBit;
 
 inline bool aligned_to(const void *p, size_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;  // NULL counts as aligned
@@ -145,27 +146,34 @@ kda_status launch_status() {
 template <int D, typename TIn>
 kda_status launch_simt(const void *q, const void *k, const void *v, const float *g,
                        const float *beta, const float *h0, float *hT, void *o, int T, int H,
-                       int nunits, const int *hdr, const int *cu, cudaStream_t s) {
+                       int nunits, const int *hdr, const int *cu, long long ntok,
+                       cudaStream_t s) {
     const size_t smem = sizeof(kda::simt::SimtSmem<D>);
     auto kern = kda::simt::kda_simt_fwd_kernel<D, TIn>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return KDA_ERR_CUDA;
+    int *err = device_error_word();
+    if (!err) return KDA_ERR_CUDA;
     kern<<<nunits, kda::simt::NT, smem, s>>>(
         static_cast<const TIn *>(q), static_cast<const TIn *>(k), static_cast<const TIn *>(v), g,
-        beta, h0, hT, static_cast<TIn *>(o), T, H, hdr, cu);
+        beta, h0, hT, static_cast<TIn *>(o), T, H, hdr, cu, ntok, err);
     return launch_status();
 }
 
 template <typename TIn>
 kda_status dispatch_simt(int D, const void *q, const void *k, const void *v, const float *g,
                          const float *beta, const float *h0, float *hT, void *o, int T, int H,
-                         int nunits, const int *hdr, const int *cu, cudaStream_t s) {
+                         int nunits, const int *hdr, const int *cu, long long ntok,
+                         cudaStream_t s) {
     switch (D) {
-        case 32: return launch_simt<32, TIn>(q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr, cu, s);
-        case 64: return launch_simt<64, TIn>(q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr, cu, s);
+        case 32:
+            return launch_simt<32, TIn>(q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr, cu, ntok, s);
+        case 64:
+            return launch_simt<64, TIn>(q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr, cu, ntok, s);
         case 128:
-            return launch_simt<128, TIn>(q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr, cu, s);
+            return launch_simt<128, TIn>(q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr, cu, ntok,
+                                         s);
         default: return KDA_ERR_UNSUPPORTED_SHAPE;
     }
 }
@@ -194,7 +202,9 @@ kda_status launch_state(kda::tc::StateArgs a, long long units, cudaStream_t s) {
 
 extern "C" {
 
-int kda_version(void) { return 100; }
+int kda_version(void) { return 200; }
+
+int kda_build_flags(void) { return KDA_DEBUG ? KDA_BUILD_DEBUG_CHECKS : 0; }
 
 const char *kda_status_string(kda_status s) {
     switch (s) {
@@ -212,6 +222,9 @@ const char *kda_status_string(kda_status s) {
         case KDA_ERR_CHECKPOINT_CAPACITY:
             return "KDA_ERR_CHECKPOINT_CAPACITY: the sequences have more state checkpoints than "
                    "ckpt_capacity slots";
+        case KDA_ERR_DEBUG_BOUNDS:
+            return "KDA_ERR_DEBUG_BOUNDS: a device-side bounds check of the debug build failed; "
+                   "the affected CTAs wrote nothing";
         default: return "KDA_ERR_UNKNOWN";
     }
 }
@@ -273,8 +286,8 @@ static kda_status tc_intra(const void *q, const void *k, const void *v, const fl
     if (cu) {
         int *err = device_error_word();
         if (!err) return KDA_ERR_CUDA;
-        kda_chunk_map_kernel<<<1, 1024, 0, s>>>(cu, N, T, hdr, seq_off, chunks, err,
-                                                ERRBIT_SEQLENS);
+        kda_chunk_map_kernel<<<1, 1024, 0, s>>>(cu, N, T, hdr, seq_off, chunks,
+                                                (int)L.max_chunks, err, ERRBIT_SEQLENS);
         if ((st = launch_status()) != KDA_OK) return st;
     } else {
         cps = (T + C - 1) / C;
@@ -323,6 +336,8 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
     a.ckpt = ckpt;
     a.ckpt_chunks = ckpt_chunks;
     a.ckpt_cap = ckpt_cap;
+    a.ntok = cu ? (long long)T : (long long)N * T;
+    a.max_chunks = (int)L.max_chunks;
     const long long chains = (long long)N * H;
     if (L.nseg <= 1) {
         // 32-column slices give the shortest per-chunk latency (they suit few chains);
@@ -403,15 +418,17 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
         if (!err) return KDA_ERR_CUDA;
         kda::tc::kda_chunk_map_kernel<<<1, 1024, 0, s>>>(
             cu_seqlens, N, T, hdr, reinterpret_cast<int *>(ws + L.seq_off),
-            reinterpret_cast<kda::tc::ChunkLoc *>(ws + L.chunks), err, ERRBIT_SEQLENS);
+            reinterpret_cast<kda::tc::ChunkLoc *>(ws + L.chunks), (int)L.max_chunks, err,
+            ERRBIT_SEQLENS);
         if ((st = launch_status()) != KDA_OK) return st;
     }
     const int nunits = N * H;
+    const long long ntok = (long long)B * T;
     if (dtype == KDA_DTYPE_F32)
         return dispatch_simt<float>(dk, q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr,
-                                    cu_seqlens, s);
+                                    cu_seqlens, ntok, s);
     return dispatch_simt<__nv_bfloat16>(dk, q, k, v, g, beta, h0, hT, o, T, H, nunits, hdr,
-                                        cu_seqlens, s);
+                                        cu_seqlens, ntok, s);
 }
 
 kda_status kda_fwd_checkpointed(const void *q, const void *k, const void *v, const float *g,
@@ -523,6 +540,7 @@ kda_status kda_get_last_device_error(void *stream) {
     if (word & ERRBIT_SEQLENS) return KDA_ERR_BAD_SEQLENS;
     if (word & ERRBIT_TIMEOUT) return KDA_ERR_DEVICE_TIMEOUT;
     if (word & ERRBIT_CKPT) return KDA_ERR_CHECKPOINT_CAPACITY;
+    if (word & ERRBIT_BOUNDS) return KDA_ERR_DEBUG_BOUNDS;
     return KDA_OK;
 }
 
@@ -537,20 +555,67 @@ static __device__ __align__(256) uint8_t g_kda_noalloc_scratch[KDA_NOALLOC_SCRAT
 
 namespace {
 constexpr int kNoallocMaxDevices = 64;
-std::once_flag g_noalloc_once[kNoallocMaxDevices];
-void *g_noalloc_ptr[kNoallocMaxDevices];
-cudaError_t g_noalloc_err[kNoallocMaxDevices];
 
-// Device address of the static scratch on the current device (nullptr on error).
+// The scratch array's device address is cached per device together with the
+// unique id of the CUDA context it was looked up in (cuCtxGetId, reached through
+// cudaGetDriverEntryPoint so the library needs no -lcuda).  A new context on the
+// device -- after cudaDeviceReset, say -- has a new id and reloads the module, so
+// the address is looked up again.  A failed lookup is not cached: the next call
+// tries again.  Without the driver entry points the address is looked up on every
+// call.
+struct NoallocSlot {
+    bool valid;
+    unsigned long long ctx_id;
+    void *ptr;
+};
+std::mutex g_noalloc_mu;
+NoallocSlot g_noalloc_slot[kNoallocMaxDevices];
+
+typedef int (*CtxGetCurrentFn)(void **);
+typedef int (*CtxGetIdFn)(void *, unsigned long long *);
+
+// Unique id of the current context; false when it cannot be read.
+bool current_context_id(unsigned long long *id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+        cudaGetLastError();   // a missing entry point is not an error of any later call
+    });
+    void *ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx) return false;
+    return get_id(ctx, id) == 0;
+}
+
+// Device address of the static scratch in the current context (nullptr on error).
 void *noalloc_scratch() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices)
         return nullptr;
-    std::call_once(g_noalloc_once[dev], [dev]() {
-        g_noalloc_err[dev] =
-            cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_kda_noalloc_scratch);
-    });
-    return g_noalloc_err[dev] == cudaSuccess ? g_noalloc_ptr[dev] : nullptr;
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoallocSlot &slot = g_noalloc_slot[dev];
+    if (have_id && slot.valid && slot.ctx_id == id) return slot.ptr;
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kda_noalloc_scratch) != cudaSuccess) {
+        cudaGetLastError();   // leave no error behind for a later launch check
+        slot.valid = false;
+        return nullptr;
+    }
+    slot.valid = have_id;
+    slot.ctx_id = id;
+    slot.ptr = p;
+    return p;
 }
 }  // namespace
 

@@ -14,9 +14,19 @@
 
 #define KDA_DEVINL __device__ __forceinline__
 
+// Debug builds (-DKDA_DEBUG=1, the library libkda_b200_debug.so) check, at the top
+// of every prefill kernel, the indices that address global memory -- chunk table
+// entries, sequence ranges, record slots -- against the extents of their buffers.
+// A failed check sets the bounds bit of the device error word and the CTA returns
+// before its first access, instead of faulting.  Release builds compile them out.
+#ifndef KDA_DEBUG
+#define KDA_DEBUG 0
+#endif
+
 namespace kda {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kErrBoundsBit = 8;   // device error word: a debug bounds check failed
 
 KDA_DEVINL uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

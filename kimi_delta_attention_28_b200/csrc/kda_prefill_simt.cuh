@@ -50,7 +50,7 @@ kda_simt_fwd_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                     const TIn *__restrict__ v, const float *__restrict__ g,
                     const float *__restrict__ beta, const float *h0, float *hT,
                     TIn *__restrict__ o, int T, int H, const int *__restrict__ hdr,
-                    const int *__restrict__ cu) {
+                    const int *__restrict__ cu, long long ntok, int *err_word) {
     static_assert(NT % D == 0, "thread mapping");
     constexpr int RG = NT / D;   // row groups
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -65,6 +65,12 @@ kda_simt_fwd_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     } else {
         seq_t0 = n * T;
         seq_len = T;
+    }
+    if constexpr (KDA_DEBUG) {   // the sequence's tokens inside q, k, v, g, beta and o
+        if (seq_len < 0 || seq_t0 < 0 || (long long)seq_t0 + seq_len > ntok) {
+            if (tid == 0) atomicOr(err_word, kErrBoundsBit);
+            return;
+        }
     }
     const size_t sbase = (size_t)chain * D * D;
     for (int e = tid; e < D * D; e += NT) sm.S[e] = h0 ? h0[sbase + e] : 0.f;

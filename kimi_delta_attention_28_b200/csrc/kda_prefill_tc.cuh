@@ -82,7 +82,8 @@ struct ChunkLoc {
 };
 
 constexpr int ERR_TIMEOUT_BIT = 2;
-constexpr int ERR_CKPT_BIT = 4;   // a state checkpoint fell past the caller's capacity
+constexpr int ERR_CKPT_BIT = 4;     // a state checkpoint fell past the caller's capacity
+constexpr int ERR_BOUNDS_BIT = kErrBoundsBit;   // debug builds: an index failed its bounds check
 
 // ---------------------------------------------------------------------------
 // Varlen chunk map: validates cu_seqlens and lays out each sequence's chunks.
@@ -90,8 +91,8 @@ constexpr int ERR_CKPT_BIT = 4;   // a state checkpoint fell past the caller's c
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) kda_chunk_map_kernel(const int *__restrict__ cu, int N,
                                                              int T, int *hdr, int *seq_off,
-                                                             ChunkLoc *chunks, int *err_word,
-                                                             int err_code) {
+                                                             ChunkLoc *chunks, int max_chunks,
+                                                             int *err_word, int err_code) {
     __shared__ int s_bad;
     __shared__ int s_scan[1024];
     const int tid = threadIdx.x;
@@ -120,6 +121,16 @@ __global__ void __launch_bounds__(1024) kda_chunk_map_kernel(const int *__restri
         __syncthreads();
         s_scan[tid] += x;
         __syncthreads();
+    }
+    if constexpr (KDA_DEBUG) {   // valid offsets give at most T / C + N chunks
+        if (s_scan[blockDim.x - 1] > max_chunks) {
+            if (tid == 0) {
+                hdr[0] = 0;
+                hdr[1] = 0;
+                atomicOr(err_word, ERR_BOUNDS_BIT);
+            }
+            return;
+        }
     }
     int base = s_scan[tid] - cnt;
     for (int n = n0; n < n1; ++n) {
@@ -258,6 +269,19 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
     };
 
+    if constexpr (KDA_DEBUG) {   // every item this CTA will take: a chunk of 1..C tokens
+        const long long ntok = chunks ? (long long)T : (long long)(slots / max(cps, 1)) * T;
+        bool bad = false;
+        for (int item = blockIdx.x + tid * gridDim.x; item < items; item += 256 * gridDim.x) {
+            const Item it = locate(item);
+            bad |= it.len < 1 || it.len > C || it.t0 < 0 || (long long)it.t0 + it.len > ntok ||
+                   item / H >= slots;
+        }
+        if (__syncthreads_or(bad)) {
+            if (tid == 0) atomicOr(err_word, ERR_BOUNDS_BIT);
+            return;
+        }
+    }
     if (warp == 0) {   // 256 tensor-memory columns, reused by the three products
         t5::alloc(tmem_slot, 2 * D);
         t5::relinquish();
@@ -737,6 +761,9 @@ struct StateArgs {
     float *ckpt;
     int ckpt_chunks;
     long long ckpt_cap;
+    // extents for the debug bounds checks: tokens in o (all sequences) and chunk slots
+    long long ntok;
+    int max_chunks;
 };
 template <int DVT>
 struct T5Layout {
@@ -826,6 +853,14 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
         c_end = c_begin + a.cps;
         seq_t0 = n * a.T;
         seq_len = a.T;
+    }
+    if constexpr (KDA_DEBUG) {   // the chain's chunks and tokens inside their buffers
+        const bool bad = c_begin < 0 || c_end > a.max_chunks || c_end - c_begin != (seq_len + C - 1) / C ||
+                         seq_len < 0 || seq_t0 < 0 || (long long)seq_t0 + seq_len > a.ntok;
+        if (bad) {
+            if (threadIdx.x == 0) atomicOr(a.err_word, ERR_BOUNDS_BIT);
+            return;
+        }
     }
     const int seq_tokens = seq_len;   // the whole sequence
     int seg_lo;                       // chunks of the sequence before this unit's segment

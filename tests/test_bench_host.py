@@ -34,15 +34,37 @@ def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monk
     sha = bench.kernel_source_sha()
     os.makedirs(os.path.join(root, "profiles"))
     with open(os.path.join(root, "profiles", "traffic.json"), "w") as f:
-        json.dump({"kernel_source_sha256": sha, "per_launch_dram_bytes": {"intra": 123.0}}, f)
-    assert bench.load_traffic("intra") == 123.0
-    assert bench.load_traffic("decode") is None
+        json.dump({"kernel_source_sha256": sha, "dram_bytes_per_unit": {"prep": 1.5}}, f)
+    assert bench.load_traffic("prep", 100) == 150.0      # per-unit figure x units
+    assert bench.load_traffic("decode", 100) is None
     # a comment-only edit keeps the figure ...
     _tree(root, "/* the same kernel */\n__global__ void k(int *p) { p[0] = 1; }  // store\n")
     assert bench.kernel_source_sha() == sha
-    assert bench.load_traffic("intra") == 123.0
+    assert bench.load_traffic("prep", 2) == 3.0
     # ... a code edit drops it
     _tree(root, "__global__ void k(int *p) { p[0] = 2; }\n")
     assert bench.kernel_source_sha() != sha
-    assert bench.load_traffic("intra") is None
+    assert bench.load_traffic("prep", 2) is None
     assert os.path.isdir(src)
+
+
+def test_compulsory_bytes_follow_the_method_not_the_records():
+    """1,540 B per token-head (q, k, v bf16, g fp32, beta, o bf16) plus each state once
+    (read if given, written always); the records are counted apart."""
+    from kimi_delta_attention_28_b200 import workloads as W
+    inp = W.make_prefill_inputs(2, 128, 3, 128, 128, BF16, True, seed=1)
+    A = bench.algorithmic(W.PREFILL, inp)
+    units = 2 * 128 * 3
+    assert A["units"] == units and A["per_unit_compulsory"] == 1540
+    assert A["compulsory"] == units * 1540 + 2 * (2 * 3 * 128 * 128 * 4)
+    assert A["prep_compulsory"] + A["state_compulsory"] == A["compulsory"]
+    assert A["intermediate"] == 2 * units * bench.record_bytes() / 64
+    inp0 = W.make_prefill_inputs(1, 64, 2, 128, 128, BF16, False, seed=1)
+    A0 = bench.algorithmic(W.LONG, inp0)
+    assert A0["compulsory"] == 64 * 2 * 1540 + 2 * 128 * 128 * 4     # final states only
+
+
+def test_headline_workload_is_the_largest_single_gpu_prefill():
+    from kimi_delta_attention_28_b200 import workloads as W
+    assert bench.HEADLINE == "long" and bench.workload_of(bench.HEADLINE) is W.LONG
+    assert bench.default_steps("long") >= 3

@@ -32,7 +32,12 @@ CHILD = textwrap.dedent("""
     torch.cuda.synchronize()
     o_ref, S_ref = oracle.kda_decode_step(d["q"][0], d["k"][0], d["v"][0], d["g"][0],
                                           d["beta"][0], d["S"])
-    rel = np.linalg.norm(S.double().cpu().numpy() - S_ref) / np.linalg.norm(S_ref)
+    def err(x, y):
+        x = x.double().cpu().numpy()
+        return max(np.linalg.norm(x - y) / np.linalg.norm(y), np.abs(x - y).max() / 5.0)
+    # both the updated state and the step's output must match (bf16 tolerances:
+    # rel-L2 <= 1e-2 and max-abs <= 5e-2, folded into one number <= 1e-2)
+    rel = max(err(S, S_ref), err(o, o_ref))
     print("CODE", code, "AFTER", kda.device_error(), "REL", rel)
 """) % ROOT
 
