@@ -671,7 +671,7 @@ def measure_decode(steps, warmup, world=1, rank=0, local=0, cpu=True):
     return out
 
 
-def decode_cpu_baseline(w, inp, S_gpu, o_last, pairs, nsteps):
+def decode_cpu_baseline(w, inp, S_gpu, o_last, pairs, nsteps, budget_s=10.0):
     """The oracle on 64 sampled (sequence, head) chains over every step the GPU ran
     (chains are independent, so the check is exact for them): steps/s scaled to the
     whole batch, and the parity of the final outputs and states of those chains."""
@@ -682,19 +682,166 @@ def decode_cpu_baseline(w, inp, S_gpu, o_last, pairs, nsteps):
     q, k, v, g = (pick(inp[n]).cpu() for n in ("q", "k", "v", "g"))
     beta = inp["beta"][:, n_idx, h_idx].transpose(0, 1).unsqueeze(2).contiguous().cpu()
     S0 = inp["S"][n_idx, h_idx].unsqueeze(1).contiguous().cpu()
-    t0 = time.perf_counter()
     o_ref, S_ref = oracle.kda_fwd(q, k, v, g, beta, S0)
-    el = time.perf_counter() - t0
-    used = min(len(pairs), oracle.threads_available())
+    # the timed sample: every step over the first `nt` (sequence, head) chains (whole
+    # sequences, all heads), sized to a few seconds of oracle time
+    nt, el = w.H, 0.0
+    while True:
+        ns = max(1, nt // w.H)
+        sel = lambda x: x[:, :ns].reshape(x.shape[0], ns * w.H, *x.shape[3:])  # noqa: E731
+        qs, ks, vs, gs = (sel(inp[n]).transpose(0, 1).unsqueeze(2).contiguous().cpu()
+                          for n in ("q", "k", "v", "g"))
+        bs = sel(inp["beta"].unsqueeze(-1)).transpose(0, 1).contiguous().cpu()
+        Ss = inp["S"][:ns].reshape(ns * w.H, 1, w.dk, w.dv).contiguous().cpu()
+        t0 = time.perf_counter()
+        oracle.kda_fwd(qs, ks, vs, gs, bs, Ss)
+        el = time.perf_counter() - t0
+        if el > budget_s / 4 or ns >= w.B:
+            break
+        nt = min(w.B * w.H, nt * 4)
+    used = min(ns * w.H, oracle.threads_available())
     S_g = S_gpu[n_idx, h_idx].unsqueeze(1).cpu()
     parity = {"tolerance": PARITY_TOL["bf16"],
               "o_last_step": _err(o_last.double().numpy(), o_ref[:, -1, 0]),
               "S": _err(S_g.double().numpy(), S_ref),
               "sample": f"{len(pairs)} sampled (sequence, head) chains over all {nsteps} steps"}
-    steps_per_s = nsteps / el * len(pairs) / (w.B * w.H)
+    steps_per_s = nsteps / el * (ns * w.H) / (w.B * w.H)
     return {"value": steps_per_s, "unit": "steps/s", "cores": int(used), "kind": "oracle",
-            "sample": f"{len(pairs)} of {w.B * w.H} (sequence, head) chains x {nsteps} steps, "
-                      f"{el:.1f} s, scaled to the whole batch", "parity": parity}
+            "sample": f"{ns * w.H} of {w.B * w.H} (sequence, head) chains (sequences 0..{ns - 1}, "
+                      f"all heads) x {nsteps} steps, {el:.1f} s, scaled to the whole batch",
+            "parity": parity}
+
+
+def measure_speculative(steps, warmup, K=4, cpu=True):
+    """Speculative decoding on the decode workload's shapes (256 sequences x 96 heads,
+    d = 128, fp32 states): every step verifies K drafted tokens per sequence
+    (kda_decode_verify, the state only read) and commits a seeded accepted count in
+    [0, K] per sequence (kda_decode_commit, the state advanced in place)."""
+    import torch
+    import kimi_delta_attention_28_b200 as kda
+    from kimi_delta_attention_28_b200 import workloads as W
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    kda.load_library()
+    w = W.DECODE
+    nsteps = warmup + steps
+    drafts = [W.make_prefill_inputs(w.B, K, w.H, w.dk, w.dv, w.dtype, i == 0,
+                                    seed=w.seed + 100 + i, device=dev) for i in range(4)]
+    S0 = drafts[0]["h0"]
+    S = S0.clone()
+    gen = torch.Generator(device="cpu").manual_seed(w.seed)
+    accs = torch.randint(0, K + 1, (nsteps, w.B), generator=gen, dtype=torch.int32).to(dev)
+    o = torch.empty(w.B, K, w.H, w.dv, dtype=w.dtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(t):
+        d = drafts[t % len(drafts)]
+        kda.kda_decode_verify(d["q"], d["k"], d["v"], d["g"], d["beta"], S, o)
+        kda.kda_decode_commit(d["k"], d["v"], d["g"], d["beta"], accs[t], S)
+
+    for t in range(warmup):
+        step(t)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.02)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.perf_counter()
+    e0.record(stream)
+    for i in range(steps):
+        step(warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.perf_counter()
+    clocks.stop()
+    assert kda.device_error() == 0
+    ms = e0.elapsed_time(e1) / steps
+    units = w.B * w.H
+    mean_acc = float(accs[warmup:].float().mean())
+    tok_in = 3 * w.dk * 2 + w.dk * 4 + 4           # q, k, v bf16, g fp32, beta
+    per_unit = (3 * w.dk * w.dv * 4                 # state: verify read, commit read + write
+                + K * (tok_in + w.dv * 2)           # verify: K drafted tokens in, K outputs out
+                + mean_acc * (tok_in - w.dk * 2))   # commit: k, v, g, beta of accepted tokens
+    bytes_step = units * per_unit
+    hbm_peak, _, peak_src = load_peaks()
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    out = {
+        "metric": f"KDA speculative decode rounds/s (verify {K} drafted tokens + commit the "
+                  "accepted prefix; 256 sequences x 96 heads, d=128)",
+        "value": 1e3 / ms, "unit": "rounds/s", "ms_per_step": ms, "steps": steps,
+        "warmup": warmup, "accepted_tokens_per_sequence_mean": mean_acc,
+        "config": {"workload": f"speculative_bf16_N{w.B}_H{w.H}_d{w.dk}_K{K}", "N": w.B,
+                   "H": w.H, "K": K, "accepted": "uniform in [0, K] per sequence (seeded)"},
+        "roofline": {"bound": "hbm", "kernel": "kda_decode_multi_kernel (verify + commit)",
+                     "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                     "traffic": None, "algorithmic_bytes_per_launch": bytes_step / 2,
+                     "algorithmic_bytes_rule": "per (sequence, head): state read (verify) + read "
+                                               "and write (commit), drafted inputs and outputs",
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)"},
+        "vs_single_token_steps": "K single decode steps would move K x 2 x 64 KiB of state "
+                                 "per (sequence, head); verify + commit move 3 x 64 KiB",
+        "gpu_launches": 2 * steps,
+        "clocks": clocks.summary(t_wall0, t_wall1),
+    }
+    if cpu:
+        out["cpu_baseline"] = speculative_cpu_baseline(w, drafts, accs, S0, S, o, K, nsteps)
+    return out
+
+
+def speculative_cpu_baseline(w, drafts, accs, S0, S_gpu, o_last, K, nsteps, nchains=64):
+    """The oracle on 64 sampled (sequence, head) chains over every round the GPU ran,
+    from the initial states: each chain's accepted tokens, round after round, then the
+    last round's verify from the oracle's own state before it.  Chains are
+    independent, so the check is exact for them; the time is scaled to the batch."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(2)
+    pairs = rng.choice(w.B * w.H, size=nchains, replace=False)
+    n_idx, h_idx = pairs // w.H, pairs % w.H
+    acc = accs.cpu().numpy()
+    host = [{k_: drafts[i][k_].cpu() for k_ in ("q", "k", "v", "g", "beta")}
+            for i in range(len(drafts))]
+
+    def packed(rounds):
+        """The accepted tokens of rounds [0, rounds) of every sampled chain, packed."""
+        cols = {k_: [] for k_ in ("k", "v", "g", "beta")}
+        cu = [0]
+        for n, h in zip(n_idx, h_idx):
+            for t in range(rounds):
+                a = int(acc[t, n])
+                d = host[t % len(host)]
+                for k_ in cols:
+                    x = d[k_][n, :a, h]
+                    cols[k_].append(x.double().numpy().reshape(a, 1, x.shape[-1])
+                                    if k_ != "beta" else x.double().numpy().reshape(a, 1))
+            cu.append(cu[-1] + sum(int(acc[t, n]) for t in range(rounds)))
+        arr = {k_: np.ascontiguousarray(np.concatenate(v_, axis=0)) for k_, v_ in cols.items()}
+        return arr, np.array(cu, dtype=np.int64)
+
+    S0s = S0[n_idx, h_idx].unsqueeze(1).double().cpu().numpy()
+    t0 = time.perf_counter()
+    arr, cu = packed(nsteps - 1)
+    _, S_before, used = oracle.kda_fwd_packed(np.zeros_like(arr["k"]), arr["k"], arr["v"],
+                                              arr["g"], arr["beta"], S0s, cu)
+    last = host[(nsteps - 1) % len(host)]
+    pick = lambda x: x[n_idx, :, h_idx].unsqueeze(2)  # noqa: E731  [64, K, 1, d]
+    o_ref = oracle.kda_decode_verify(pick(last["q"]), pick(last["k"]), pick(last["v"]),
+                                     pick(last["g"]), last["beta"][n_idx, :, h_idx].unsqueeze(2),
+                                     S_before)
+    S_ref = oracle.kda_decode_commit(pick(last["k"]), pick(last["v"]), pick(last["g"]),
+                                     last["beta"][n_idx, :, h_idx].unsqueeze(2),
+                                     acc[nsteps - 1, n_idx], S_before)
+    el = time.perf_counter() - t0
+    o_g = o_last[n_idx, :, h_idx].unsqueeze(2).double().cpu().numpy()
+    S_g = S_gpu[n_idx, h_idx].unsqueeze(1).double().cpu().numpy()
+    return {"value": nsteps / el * nchains / (w.B * w.H), "unit": "rounds/s",
+            "cores": int(min(used, nchains)), "kind": "oracle",
+            "sample": f"{nchains} sampled (sequence, head) chains over all {nsteps} rounds, "
+                      f"{el:.1f} s (tokens gathered in Python), scaled to the whole batch",
+            "parity": {"tolerance": PARITY_TOL["bf16"], "o_last_round": _err(o_g, o_ref),
+                       "S": _err(S_g, S_ref),
+                       "sample": f"{nchains} sampled chains, every round, from the initial states"}}
 
 
 # ---------------------------------------------------------------------------
@@ -819,6 +966,9 @@ def main():
                                                       "steps", "warmup", "config", "roofline",
                                                       "gpu_launches", "clocks", "cpu_baseline")
                                 if k_ in r}
+            _free_device_memory()
+            r = measure_speculative(200, 20, cpu=cpu)
+            nested["speculative"] = r
             out["workloads"] = nested
         if out is not None:
             print(json.dumps(out), flush=True)

@@ -54,7 +54,8 @@ typedef enum {
     KDA_ERR_BAD_SEQLENS = 7,          /* cu_seqlens not monotone / out of range    */
     KDA_ERR_EXCEEDS_STATIC_SCRATCH = 8, /* kda_fwd_noalloc: problem too large      */
     KDA_ERR_CHECKPOINT_CAPACITY = 9,  /* kda_fwd_checkpointed: more checkpoints than slots */
-    KDA_ERR_DEBUG_BOUNDS = 10         /* debug build: a device-side bounds check failed */
+    KDA_ERR_DEBUG_BOUNDS = 10,        /* debug build: a device-side bounds check failed */
+    KDA_ERR_BAD_ACCEPTED = 11         /* kda_decode_commit: accepted count outside [0, K] */
 } kda_status;
 
 typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
@@ -234,6 +235,42 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
                            int dv, int dtype, void *stream);
 
 /*
+ * Speculative decoding: verify K drafted tokens per sequence, then commit the
+ * accepted prefix.  Source: the "Kimi K3" open-weights field notes, panel
+ * "目标模型太大，缓存和草稿都必须理解 KDA": with a draft model the KDA recurrent
+ * state must follow only the tokens the target model accepts -- a rejected draft
+ * must not remain in the state -- and K3 keeps the projected inputs of the drafted
+ * tokens and replays the accepted ones on chip instead of storing a state per
+ * drafted token.  The recurrence is the one above (panel "KDA 单头递归"), token by
+ * token in draft order.
+ *
+ * kda_decode_verify: for every (sequence n, head h), run the K drafted tokens from
+ *   the state S and write their K outputs; S is only read.
+ *     q, k, g [N, K, H, d_k] dtype / fp32;  v [N, K, H, d_v] dtype;
+ *     beta [N, K, H] fp32;  S [N, H, d_k, d_v] fp32 (read);
+ *     o [N, K, H, d_v] dtype: o[n, t] is the read of the state after draft
+ *     tokens 0..t -- what K chained kda_decode_step calls would return.
+ * kda_decode_commit: for every (sequence n, head h), replay the first accepted[n]
+ *   drafted tokens (the same k, v, g, beta the verify call saw) from S and write
+ *   the resulting state to S in place: S becomes the state after the accepted
+ *   prefix, as if only those tokens had been decoded.  accepted is a DEVICE array
+ *   of N int32 counts in [0, K] (typically written by the sampler on the GPU);
+ *   accepted[n] = 0 leaves sequence n's state untouched.  A count outside [0, K]
+ *   leaves that sequence's state untouched and makes the call's device error
+ *   KDA_ERR_BAD_ACCEPTED (see kda_get_last_device_error).
+ * 1 <= K <= 16 (K = 0 or N = 0 is a no-op; K > 16 returns KDA_ERR_INVALID_ARG).
+ * Alignment: S 16 bytes, everything else its element size.  o must not alias an
+ * input.  Cost: verify reads each state once; commit reads and writes it once --
+ * against K reads and K writes for K single decode steps.
+ */
+kda_status kda_decode_verify(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *S, void *o, int N, int K, int H,
+                             int dk, int dv, int dtype, void *stream);
+kda_status kda_decode_commit(const void *k, const void *v, const float *g, const float *beta,
+                             const int32_t *accepted, float *S, int N, int K, int H, int dk,
+                             int dv, int dtype, void *stream);
+
+/*
  * Allocation-free prefill.  The source pages have no counterpart to this entry
  * point: it is a convenience of this library, not part of the method.
  *
@@ -280,9 +317,9 @@ kda_status kda_fwd_noalloc(const void *q, const void *k, const void *v, const fl
 /*
  * Synchronises `stream`, then reads and clears the library's device error word
  * (cu_seqlens violations, bounded waits that gave up, checkpoints past the
- * capacity, debug bounds checks).  Returns KDA_OK, KDA_ERR_BAD_SEQLENS,
- * KDA_ERR_DEVICE_TIMEOUT, KDA_ERR_CHECKPOINT_CAPACITY, KDA_ERR_DEBUG_BOUNDS or
- * KDA_ERR_CUDA.
+ * capacity, debug bounds checks, accepted counts out of range).  Returns KDA_OK,
+ * KDA_ERR_BAD_SEQLENS, KDA_ERR_DEVICE_TIMEOUT, KDA_ERR_CHECKPOINT_CAPACITY,
+ * KDA_ERR_DEBUG_BOUNDS, KDA_ERR_BAD_ACCEPTED or KDA_ERR_CUDA.
  */
 kda_status kda_get_last_device_error(void *stream);
 

@@ -11,16 +11,21 @@ panel "KDA 单头递归"), as a C-ABI CUDA library:
                        (per-segment affine maps combined in prefix order);
 * ``kda_fwd_checkpointed`` prefill that also stores the state every n tokens
                        (prefix caching);
-* ``kda_decode_step``  one token per sequence, state updated in place.
+* ``kda_decode_step``  one token per sequence, state updated in place;
+* ``kda_decode_verify`` / ``kda_decode_commit``  speculative decoding: run K
+                       drafted tokens without touching the state, then advance
+                       the state over the accepted prefix only.
 
 This package is the thin Python binding; ``include/kda.h`` is the interface.
 """
-from ._lib import (KDAError, checkpoint_count, device_error, kda_decode_step,  # noqa: F401
+from ._lib import (KDAError, checkpoint_count, device_error, kda_decode_commit,  # noqa: F401
+                   kda_decode_step, kda_decode_verify,
                    kda_fwd, kda_fwd_checkpointed, kda_fwd_inter, kda_fwd_intra,
                    kda_fwd_noalloc, kda_fwd_segmented, load_library, plan_segments,
                    segmented_workspace_size, workspace_size)
 
 __all__ = ["kda_fwd", "kda_fwd_intra", "kda_fwd_inter", "kda_fwd_noalloc", "kda_fwd_segmented",
-           "kda_fwd_checkpointed", "checkpoint_count", "kda_decode_step", "workspace_size",
+           "kda_fwd_checkpointed", "checkpoint_count", "kda_decode_step",
+           "kda_decode_verify", "kda_decode_commit", "workspace_size",
            "segmented_workspace_size", "plan_segments", "device_error", "load_library",
            "KDAError"]

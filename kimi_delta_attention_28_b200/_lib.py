@@ -25,7 +25,10 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED_SHAPE",
           3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_WORKSPACE_TOO_SMALL", 5: "KDA_ERR_CUDA",
           6: "KDA_ERR_DEVICE_TIMEOUT", 7: "KDA_ERR_BAD_SEQLENS",
           8: "KDA_ERR_EXCEEDS_STATIC_SCRATCH", 9: "KDA_ERR_CHECKPOINT_CAPACITY",
-          10: "KDA_ERR_DEBUG_BOUNDS"}
+          10: "KDA_ERR_DEBUG_BOUNDS", 11: "KDA_ERR_BAD_ACCEPTED"}
+
+# Largest number of drafted tokens kda_decode_verify / kda_decode_commit take.
+MAX_DRAFT = 16
 
 # Size of the static scratch array behind kda_fwd_noalloc (KDA_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -44,6 +47,8 @@ SIGNATURES = {
     "kda_fwd_inter": ([_VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP], _I),
     "kda_decode_step": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP], _I),
     "kda_get_last_device_error": ([_VP], _I),
+    "kda_decode_verify": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP], _I),
+    "kda_decode_commit": ([_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP], _I),
     "kda_fwd_noalloc": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP,
                          _VP], _I),
     "kda_fwd_segmented_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I], _SZ),
@@ -359,6 +364,63 @@ def kda_decode_step(q, k, v, g, beta, S, o=None):
     _check(lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
                                N, H, dk, dv, dt, _stream(dev)), "kda_decode_step")
     return o
+
+
+def _draft_shapes(k, v, g, beta, S, q=None):
+    if k.dim() != 4 or v.dim() != 4 or tuple(v.shape[:3]) != tuple(k.shape[:3]):
+        raise ValueError(f"k must be [N, K, H, d_k] and v [N, K, H, d_v], got {tuple(k.shape)} "
+                         f"and {tuple(v.shape)}")
+    N, K, H, dk = k.shape
+    dv = v.shape[-1]
+    _shape(q, "q", k.shape)
+    _shape(g, "g", k.shape)
+    _shape(beta, "beta", (N, K, H))
+    _shape(S, "S", (N, H, dk, dv))
+    if K > MAX_DRAFT:
+        raise ValueError(f"at most {MAX_DRAFT} drafted tokens, got K = {K}")
+    return N, K, H, dk, dv
+
+
+def kda_decode_verify(q, k, v, g, beta, S, o=None):
+    """Run K drafted tokens per (sequence, head) from the state S without changing it.
+    q, k, g: [N, K, H, d_k]; v: [N, K, H, d_v]; beta: [N, K, H]; S: [N, H, d_k, d_v]
+    fp32.  Returns o [N, K, H, d_v]: o[:, t] is what the t-th of K chained decode steps
+    would return."""
+    lib = load_library()
+    dev = k.device
+    N, K, H, dk, dv = _draft_shapes(k, v, g, beta, S, q)
+    _shape(o, "o", (N, K, H, dv))
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, n, k.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    if o is None:
+        o = torch.empty(N, K, H, dv, dtype=k.dtype, device=dev)
+    _check(lib.kda_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                                 _ptr(o), N, K, H, dk, dv, _dtype_code(k.dtype), _stream(dev)),
+           "kda_decode_verify")
+    return o
+
+
+def kda_decode_commit(k, v, g, beta, accepted, S):
+    """Advance S in place over the first accepted[n] of the K drafted tokens of each
+    sequence n (the inputs given to kda_decode_verify); accepted is an int32 CUDA
+    tensor [N] with values in [0, K].  Returns S."""
+    lib = load_library()
+    dev = k.device
+    N, K, H, dk, dv = _draft_shapes(k, v, g, beta, S)
+    _shape(accepted, "accepted", (N,))
+    for t, n in ((k, "k"), (v, "v")):
+        _need(t, n, k.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    _need(accepted, "accepted", torch.int32, dev)
+    _check(lib.kda_decode_commit(_ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(accepted), _ptr(S),
+                                 N, K, H, dk, dv, _dtype_code(k.dtype), _stream(dev)),
+           "kda_decode_commit")
+    return S
 
 
 def kda_fwd_noalloc(q, k, v, g, beta, h0, cu_seqlens, o, hT):

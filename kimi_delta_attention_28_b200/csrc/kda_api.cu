@@ -25,6 +25,7 @@ constexpr int ERRBIT_SEQLENS = 1;
 constexpr int ERRBIT_TIMEOUT = 2;
 constexpr int ERRBIT_CKPT = 4;
 constexpr int ERRBIT_BOUNDS = kda::kErrBoundsBit;
+constexpr int ERRBIT_ACCEPTED = kda::dec::kErrAcceptedBit;
 
 inline bool aligned_to(const void *p, size_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;  // NULL counts as aligned
@@ -222,6 +223,9 @@ const char *kda_status_string(kda_status s) {
         case KDA_ERR_CHECKPOINT_CAPACITY:
             return "KDA_ERR_CHECKPOINT_CAPACITY: the sequences have more state checkpoints than "
                    "ckpt_capacity slots";
+        case KDA_ERR_BAD_ACCEPTED:
+            return "KDA_ERR_BAD_ACCEPTED: an accepted token count of kda_decode_commit is outside "
+                   "[0, K]; that sequence's state was left unchanged";
         case KDA_ERR_DEBUG_BOUNDS:
             return "KDA_ERR_DEBUG_BOUNDS: a device-side bounds check of the debug build failed; "
                    "the affected CTAs wrote nothing";
@@ -528,6 +532,87 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
     return launch_status();
 }
 
+// Shared host checks of the verify / commit entry points.
+static kda_status check_multi(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *S, int N, int K, int H, int dk,
+                              int dv, int dtype, bool need_q) {
+    if (N < 0 || K < 0) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_shape(H, dk, dv, dtype);
+    if (st != KDA_OK) return st;
+    if (K > kda::dec::kMaxDraft) return KDA_ERR_INVALID_ARG;
+    if (N == 0 || K == 0) return KDA_OK;
+    if ((need_q && !q) || !k || !v || !g || !beta || !S) return KDA_ERR_INVALID_ARG;
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    if (!aligned_to(S, 16) || !aligned_to(q, es) || !aligned_to(k, es) || !aligned_to(v, es) ||
+        !aligned_to(g, 4) || !aligned_to(beta, 4))
+        return KDA_ERR_MISALIGNED;
+    if ((long long)N * H > 0x7fffffffLL || (long long)N * K * H > 0x7fffffffLL)
+        return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
+kda_status kda_decode_verify(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *S, void *o, int N, int K, int H,
+                             int dk, int dv, int dtype, void *stream) {
+    kda_status st = check_multi(q, k, v, g, beta, S, N, K, H, dk, dv, dtype, true);
+    if (st != KDA_OK) return st;
+    if (N == 0 || K == 0) return KDA_OK;
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    if (!o) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(o, es)) return KDA_ERR_MISALIGNED;
+    if (o == q || o == k || o == v || o == g || o == beta || o == S) return KDA_ERR_INVALID_ARG;
+    int *err = device_error_word();
+    if (!err) return KDA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned grid = (unsigned)(N * H);
+    using namespace kda::dec;
+#define KDA_VER(DD, TT)                                                                         \
+    kda_decode_multi_kernel<DD, TT, false><<<grid, NT, 0, s>>>(                                 \
+        static_cast<const TT *>(q), static_cast<const TT *>(k), static_cast<const TT *>(v), g,   \
+        beta, const_cast<float *>(S), static_cast<TT *>(o), nullptr, K, H, err)
+    if (dtype == KDA_DTYPE_BF16) {
+        if (dk == 32) KDA_VER(32, __nv_bfloat16);
+        else if (dk == 64) KDA_VER(64, __nv_bfloat16);
+        else KDA_VER(128, __nv_bfloat16);
+    } else {
+        if (dk == 32) KDA_VER(32, float);
+        else if (dk == 64) KDA_VER(64, float);
+        else KDA_VER(128, float);
+    }
+#undef KDA_VER
+    return launch_status();
+}
+
+kda_status kda_decode_commit(const void *k, const void *v, const float *g, const float *beta,
+                             const int32_t *accepted, float *S, int N, int K, int H, int dk,
+                             int dv, int dtype, void *stream) {
+    kda_status st = check_multi(nullptr, k, v, g, beta, S, N, K, H, dk, dv, dtype, false);
+    if (st != KDA_OK) return st;
+    if (N == 0 || K == 0) return KDA_OK;
+    if (!accepted) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(accepted, 4)) return KDA_ERR_MISALIGNED;
+    int *err = device_error_word();
+    if (!err) return KDA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned grid = (unsigned)(N * H);
+    using namespace kda::dec;
+#define KDA_COM(DD, TT)                                                                         \
+    kda_decode_multi_kernel<DD, TT, true><<<grid, NT, 0, s>>>(                                  \
+        nullptr, static_cast<const TT *>(k), static_cast<const TT *>(v), g, beta, S, nullptr,    \
+        accepted, K, H, err)
+    if (dtype == KDA_DTYPE_BF16) {
+        if (dk == 32) KDA_COM(32, __nv_bfloat16);
+        else if (dk == 64) KDA_COM(64, __nv_bfloat16);
+        else KDA_COM(128, __nv_bfloat16);
+    } else {
+        if (dk == 32) KDA_COM(32, float);
+        else if (dk == 64) KDA_COM(64, float);
+        else KDA_COM(128, float);
+    }
+#undef KDA_COM
+    return launch_status();
+}
+
 kda_status kda_get_last_device_error(void *stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
@@ -541,6 +626,7 @@ kda_status kda_get_last_device_error(void *stream) {
     if (word & ERRBIT_TIMEOUT) return KDA_ERR_DEVICE_TIMEOUT;
     if (word & ERRBIT_CKPT) return KDA_ERR_CHECKPOINT_CAPACITY;
     if (word & ERRBIT_BOUNDS) return KDA_ERR_DEBUG_BOUNDS;
+    if (word & ERRBIT_ACCEPTED) return KDA_ERR_BAD_ACCEPTED;
     return KDA_OK;
 }
 

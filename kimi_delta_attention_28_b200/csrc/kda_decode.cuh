@@ -103,5 +103,128 @@ kda_decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     }
 }
 
+// ---------------------------------------------------------------------------
+// Speculative decoding: verify K drafted tokens, then commit the accepted prefix.
+//
+// A draft proposes K tokens per sequence; the target model runs them as one small
+// batch and accepts a prefix of a <= K of them ("Kimi K3" open-weights field notes,
+// panel "目标模型太大，缓存和草稿都必须理解 KDA": the draft and the cache must follow
+// the KDA state, a rejected draft must not leave its tokens in the state, and the
+// accepted states are replayed on chip from the cached projected inputs).
+//   verify: from S, run the K tokens of the recurrence in registers and write the
+//           K outputs; S is only read (one HBM read of the state).
+//   commit: from S, replay the first a_n tokens (a_n from the device array
+//           `accepted`) and write the state back (one read and one write); a_n = 0
+//           leaves S untouched, a_n outside [0, K] sets the error bit and leaves S
+//           untouched.
+// Layouts: q, k, g [N, K, H, D]; v, o [N, K, H, D]; beta [N, K, H]; S [N, H, D, D].
+// Same thread mapping as kda_decode_kernel (float4 column groups, RPT rows per
+// thread); a token's inputs are staged in shared memory up front.
+// ---------------------------------------------------------------------------
+constexpr int kMaxDraft = 16;        // largest K
+constexpr int kErrAcceptedBit = 16;  // device error word: an accepted count out of range
+
+template <int D, typename TIn, bool COMMIT>
+__global__ void __launch_bounds__(NT, 2)
+kda_decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
+                        const TIn *__restrict__ v, const float *__restrict__ g,
+                        const float *__restrict__ beta, float *__restrict__ S,
+                        TIn *__restrict__ o, const int *__restrict__ accepted, int K, int H,
+                        int *err_word) {
+    constexpr int CG = D / 4, RS = NT / CG, RPT = D / RS;
+    static_assert(NT % CG == 0 && D % RS == 0, "thread mapping");
+    __shared__ float s_k[kMaxDraft][D], s_a[kMaxDraft][D], s_v[kMaxDraft][D];
+    __shared__ float s_q[COMMIT ? 1 : kMaxDraft][D];
+    __shared__ float s_b[kMaxDraft], s_kq[kMaxDraft];
+    __shared__ __align__(16) float s_p[RS][D];
+    __shared__ __align__(16) float s_r[COMMIT ? 1 : RS][D];
+    __shared__ __align__(16) float s_delta[D];
+
+    const int tid = threadIdx.x, cg = tid % CG, rs = tid / CG;
+    const size_t unit = blockIdx.x;                 // (sequence, head)
+    const int n = (int)(unit / H), h = (int)(unit % H);
+    int ntok = K;
+    if constexpr (COMMIT) {
+        ntok = accepted[n];
+        if (ntok < 0 || ntok > K) {
+            if (tid == 0 && h == 0) atomicOr(err_word, kErrAcceptedBit);
+            return;
+        }
+        if (ntok == 0) return;   // nothing accepted: the state stays as it is
+    }
+    float4 *Sp = reinterpret_cast<float4 *>(S + unit * D * D);
+    float4 s[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(Sp + (rs + i * RS) * CG + cg);
+
+    // stage the tokens' inputs: token t of (n, h) sits at row (n K + t) H + h
+    for (int e = tid; e < ntok * D; e += NT) {
+        const int t = e / D, c = e % D;
+        const size_t row = ((size_t)n * K + t) * H + h;
+        s_k[t][c] = ld1<TIn>(k + row * D + c);
+        s_a[t][c] = expf(__ldg(g + row * D + c));
+        s_v[t][c] = ld1<TIn>(v + row * D + c);
+        if constexpr (!COMMIT) s_q[t][c] = ld1<TIn>(q + row * D + c);
+    }
+    if (tid < ntok) s_b[tid] = __ldg(beta + ((size_t)n * K + tid) * H + h);
+    __syncthreads();
+    if constexpr (!COMMIT) {   // k_t . q_t, one warp per token
+        for (int t = tid >> 5; t < ntok; t += NT / 32) {
+            float x = 0.f;
+            for (int i = tid & 31; i < D; i += 32) x += s_k[t][i] * s_q[t][i];
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+            if ((tid & 31) == 0) s_kq[t] = x;
+        }
+    }
+    for (int t = 0; t < ntok; ++t) {
+        // decay, then partial column sums of k^T S' (and q^T S') over this thread's rows
+        float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const int row = rs + i * RS;
+            const float a = s_a[t][row], kr = s_k[t][row];
+            s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+            pk.x += kr * s[i].x; pk.y += kr * s[i].y; pk.z += kr * s[i].z; pk.w += kr * s[i].w;
+            if constexpr (!COMMIT) {
+                const float qr = s_q[t][row];
+                pq.x += qr * s[i].x; pq.y += qr * s[i].y; pq.z += qr * s[i].z; pq.w += qr * s[i].w;
+            }
+        }
+        *reinterpret_cast<float4 *>(&s_p[rs][cg * 4]) = pk;
+        if constexpr (!COMMIT) *reinterpret_cast<float4 *>(&s_r[rs][cg * 4]) = pq;
+        __syncthreads();
+        if (tid < D) {
+            float p = 0.f, r = 0.f;
+#pragma unroll
+            for (int j = 0; j < RS; ++j) {
+                p += s_p[j][tid];
+                if constexpr (!COMMIT) r += s_r[j][tid];
+            }
+            const float d = s_b[t] * (s_v[t][tid] - p);
+            s_delta[tid] = d;
+            if constexpr (!COMMIT) {
+                const float out = r + s_kq[t] * d;
+                const size_t row = ((size_t)n * K + t) * H + h;
+                if constexpr (sizeof(TIn) == 2)
+                    o[row * D + tid] = f2bf(out);
+                else
+                    o[row * D + tid] = out;
+            }
+        }
+        __syncthreads();
+        const float4 dl = *reinterpret_cast<const float4 *>(&s_delta[cg * 4]);
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const float kr = s_k[t][rs + i * RS];
+            s[i].x += kr * dl.x; s[i].y += kr * dl.y; s[i].z += kr * dl.z; s[i].w += kr * dl.w;
+        }
+    }
+    if constexpr (COMMIT) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) __stcs(Sp + (rs + i * RS) * CG + cg, s[i]);
+    }
+}
+
 }  // namespace dec
 }  // namespace kda

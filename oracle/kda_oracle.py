@@ -24,6 +24,12 @@ Parity status of each function (what pins it, beside itself, lives in
                        invariants (linearity, split runs, varlen).
 * ``kda_decode_step``  pinned: equals ``kda_fwd`` with T=1 and chained decode
                        equals prefill.
+* ``kda_decode_verify`` / ``kda_decode_commit``  (speculative decoding, same page,
+                       panel "目标模型太大，缓存和草稿都必须理解 KDA": the state must
+                       follow only the accepted draft tokens) pinned: against the
+                       brute-force operator products on every drafted prefix, with
+                       a different accepted count per sequence, and commit of zero
+                       tokens returns the state unchanged.
 """
 from __future__ import annotations
 
@@ -132,3 +138,40 @@ def kda_decode_step(q, k, v, g, beta, S, nthreads: int = 0):
     cu = np.arange(N + 1, dtype=np.int64)
     o, hT, _ = kda_fwd_packed(q, k, v, g, beta, S, cu, nthreads)
     return o, hT
+
+
+def kda_decode_verify(q, k, v, g, beta, S, nthreads: int = 0):
+    """K drafted tokens per sequence, run from the state S (which is not changed):
+    q, k, g [N, K, H, d_k]; v [N, K, H, d_v]; beta [N, K, H]; S [N, H, d_k, d_v].
+    Returns o [N, K, H, d_v]: o[n, t] is the read of the state after drafted tokens
+    0..t of sequence n, i.e. the recurrence over the K tokens from S."""
+    q, k, v, g, beta, S = map(_f64, (q, k, v, g, beta, S))
+    N, K, H, dk = q.shape
+    dv = v.shape[3]
+    cu = np.arange(N + 1, dtype=np.int64) * K
+    o, _, _ = kda_fwd_packed(q.reshape(N * K, H, dk), k.reshape(N * K, H, dk),
+                             v.reshape(N * K, H, dv), g.reshape(N * K, H, dk),
+                             beta.reshape(N * K, H), S, cu, nthreads)
+    return o.reshape(N, K, H, dv)
+
+
+def kda_decode_commit(k, v, g, beta, accepted, S, nthreads: int = 0):
+    """The state of every sequence after only its first accepted[n] drafted tokens
+    (k, g [N, K, H, d_k]; v [N, K, H, d_v]; beta [N, K, H]; S [N, H, d_k, d_v];
+    accepted [N] integers in [0, K]): the recurrence from S over that prefix, the
+    rejected tokens never entering the state.  Returns the new states [N, H, d_k, d_v]."""
+    k, v, g, beta, S = map(_f64, (k, v, g, beta, S))
+    if hasattr(accepted, "detach"):
+        accepted = accepted.detach().cpu().numpy()
+    acc = np.asarray(accepted, dtype=np.int64)
+    N, K, H, dk = k.shape
+    dv = v.shape[3]
+    if acc.shape != (N,) or (acc < 0).any() or (acc > K).any():
+        raise ValueError("accepted must hold N counts in [0, K]")
+    take = lambda x: np.ascontiguousarray(  # noqa: E731
+        np.concatenate([x[n, :acc[n]] for n in range(N)], axis=0))
+    cu = np.concatenate([[0], np.cumsum(acc)]).astype(np.int64)
+    kp, vp, gp, bp = take(k), take(v), take(g), take(beta)
+    qp = np.zeros_like(kp)                     # outputs are not needed here
+    _, hT, _ = kda_fwd_packed(qp, kp, vp, gp, bp, S, cu, nthreads)
+    return hT

@@ -207,7 +207,9 @@ DEBUG_CHILD = textwrap.dedent("""
     kda.kda_fwd_intra(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["cu_seqlens"],
                       workspace=ws)
     assert kda.device_error() == 0
-    ws[256:260].view(torch.int32)[0] = 1 << 20      # seq_off[1]: far past the chunk table
+    # seq_off[0..N] sits 256 bytes into the workspace: seq_off[1] (bytes 260..263) ends
+    # sequence 0 and starts sequence 1, so both sequences' chunk ranges turn invalid
+    ws[260:264].view(torch.int32)[0] = 1 << 20      # seq_off[1]: far past the chunk table
     o = torch.full((B, T, H, 128), 7.0, dtype=torch.bfloat16, device=dev)
     hT = torch.full((4, H, 128, 128), 7.0, device=dev)
     kda.kda_fwd_inter(inp["h0"], inp["cu_seqlens"], o, hT, B=B, T=T, H=H, dk=128, dv=128,

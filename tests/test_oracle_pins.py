@@ -263,3 +263,60 @@ def test_oracle_rejects_bad_offsets():
     z = np.zeros((1, 4, 1, 2))
     with pytest.raises(ValueError):
         oracle.kda_fwd(z, z, z, z, np.zeros((1, 4, 1)), cu_seqlens=np.array([0, 3, 2, 4]))
+
+
+def _draft_batch(rng, N, K, H, dk, dv):
+    """N sequences x H heads of K drafted tokens, [N, K, H, d] layouts, plus states."""
+    chains = [[rand_chain(rng, K, dk, dv) for _ in range(H)] for _ in range(N)]
+    st = lambda i: np.stack([np.stack([chains[n][h][i] for h in range(H)], axis=1)  # noqa: E731
+                             for n in range(N)])
+    q, k, v, g = st(0), st(1), st(2), st(3)
+    beta = np.stack([np.stack([chains[n][h][4] for h in range(H)], axis=1) for n in range(N)])
+    S = np.stack([np.stack([chains[n][h][5] for h in range(H)]) for n in range(N)])
+    return chains, q, k, v, g, beta, S
+
+
+def test_decode_verify_equals_brute_force_on_every_prefix():
+    """Verify = the recurrence over the K drafted tokens from S, read after each token:
+    against the dense operator products, chain by chain; S itself is not changed."""
+    rng = np.random.default_rng(40)
+    N, K, H, dk, dv = 3, 5, 2, 4, 3
+    chains, q, k, v, g, beta, S = _draft_batch(rng, N, K, H, dk, dv)
+    S_before = S.copy()
+    o = oracle.kda_decode_verify(q, k, v, g, beta, S)
+    assert o.shape == (N, K, H, dv) and np.array_equal(S, S_before)
+    for n in range(N):
+        for h in range(H):
+            cq, ck, cv, cg, cb, _ = chains[n][h]
+            o_bf, _ = brute_force(cq, ck, cv, cg, cb, S[n, h])
+            assert np.allclose(o[n, :, h], o_bf, rtol=1e-12, atol=1e-12)
+
+
+def test_decode_commit_keeps_only_the_accepted_prefix():
+    """Commit = the state after only the first a_n drafted tokens (a different a_n per
+    sequence, 0 and K included): against the dense operator products on that prefix;
+    a_n = 0 returns the state exactly; counts outside [0, K] are refused."""
+    rng = np.random.default_rng(41)
+    N, K, H, dk, dv = 4, 6, 2, 5, 3
+    chains, q, k, v, g, beta, S = _draft_batch(rng, N, K, H, dk, dv)
+    acc = np.array([0, 3, 6, 1])
+    S_new = oracle.kda_decode_commit(k, v, g, beta, acc, S)
+    for n in range(N):
+        for h in range(H):
+            if acc[n] == 0:
+                assert np.array_equal(S_new[n, h], S[n, h])
+                continue
+            cq, ck, cv, cg, cb, _ = chains[n][h]
+            a = acc[n]
+            _, S_bf = brute_force(cq[:a], ck[:a], cv[:a], cg[:a], cb[:a], S[n, h])
+            assert np.allclose(S_new[n, h], S_bf, rtol=1e-12, atol=1e-12)
+    # a rejected token changes nothing: the tail of the draft is irrelevant
+    k2, v2, g2 = k.copy(), v.copy(), g.copy()
+    k2[1, 3:] = rng.standard_normal(k2[1, 3:].shape)
+    v2[1, 3:] += 1.0
+    g2[1, 3:] = -4.0
+    assert np.array_equal(oracle.kda_decode_commit(k2, v2, g2, beta, acc, S)[1], S_new[1])
+    with pytest.raises(ValueError):
+        oracle.kda_decode_commit(k, v, g, beta, np.array([0, 7, 1, 1]), S)
+    with pytest.raises(ValueError):
+        oracle.kda_decode_commit(k, v, g, beta, np.array([0, -1, 1, 1]), S)
