@@ -24,6 +24,12 @@ Parity status of each function (what pins it, beside itself, lives in
                        invariants (linearity, split runs, varlen).
 * ``kda_decode_step``  pinned: equals ``kda_fwd`` with T=1 and chained decode
                        equals prefill.
+* ``kda_bwd`` / ``kda_bwd_packed``  (the gradient of the recurrence, by reverse
+                       accumulation through the token loop) pinned: against central
+                       finite differences of ``kda_fwd`` in every input, element by
+                       element on tiny chains and along random directions on larger
+                       packed batches (empty sequences included); planted mistakes in
+                       its C source fail those pins.
 * ``kda_decode_verify`` / ``kda_decode_commit``  (speculative decoding, same page,
                        panel "目标模型太大，缓存和草稿都必须理解 KDA": the state must
                        follow only the accepted draft tokens) pinned: against the
@@ -54,6 +60,10 @@ def _lib():
                                        ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                        ctypes.c_int64, ctypes.c_int, dp, dp]
         lib.kda_oracle_fwd.restype = ctypes.c_int
+        lib.kda_oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, lp, ctypes.c_int64,
+                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, dp, dp,
+                                       ctypes.c_int, dp, dp, dp, dp, dp, dp]
+        lib.kda_oracle_bwd.restype = ctypes.c_int
         _LIB = lib
     return _LIB
 
@@ -175,3 +185,48 @@ def kda_decode_commit(k, v, g, beta, accepted, S, nthreads: int = 0):
     qp = np.zeros_like(kp)                     # outputs are not needed here
     _, hT, _ = kda_fwd_packed(qp, kp, vp, gp, bp, S, cu, nthreads)
     return hT
+
+
+def kda_bwd_packed(q, k, v, g, beta, h0, cu_seqlens, do, dhT=None, nthreads: int = 0):
+    """Gradient of the recurrence on packed sequences (layouts as kda_fwd_packed):
+    given do = dL/do [T_total, H, d_v] and dhT = dL/dhT [N, H, d_k, d_v] (None: zero),
+    returns (dq, dk, dv, dg, dbeta, dh0) = dL/d(input) in fp64."""
+    q, k, v, g, beta, h0, do, dhT = map(_f64, (q, k, v, g, beta, h0, do, dhT))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    N = cu.shape[0] - 1
+    assert cu[-1] == T and do.shape == (T, H, dv)
+    if dhT is not None:
+        assert dhT.shape == (N, H, dk, dv)
+    dq, dkk, dg = (np.zeros((T, H, dk)) for _ in range(3))
+    dvv = np.zeros((T, H, dv))
+    db = np.zeros((T, H))
+    dh0 = np.zeros((N, H, dk, dv))
+    used = _lib().kda_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                 cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), N, H, dk, dv,
+                                 _ptr(do), _ptr(dhT), int(nthreads), _ptr(dq), _ptr(dkk),
+                                 _ptr(dvv), _ptr(dg), _ptr(db), _ptr(dh0))
+    if used < 0:
+        raise ValueError("kda_oracle_bwd rejected its arguments")
+    return dq, dkk, dvv, dg, db, dh0
+
+
+def kda_bwd(q, k, v, g, beta, h0, do, dhT=None, cu_seqlens=None, nthreads: int = 0):
+    """Gradient on [B, T, H, d] inputs (or packed [1, T_total, H, d] with cu_seqlens):
+    returns (dq, dk, dv, dg, dbeta, dh0) shaped like the inputs (dh0 [N, H, d_k, d_v])."""
+    q, k, v, g, beta, do = map(_f64, (q, k, v, g, beta, do))
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    cu = np.arange(B + 1, dtype=np.int64) * T if cu_seqlens is None else cu_seqlens
+    r = kda_bwd_packed(q.reshape(B * T, H, dk), k.reshape(B * T, H, dk), v.reshape(B * T, H, dv),
+                       g.reshape(B * T, H, dk), beta.reshape(B * T, H), h0, cu,
+                       do.reshape(B * T, H, dv), dhT, nthreads)
+    dq, dkk, dvv, dg, db, dh0 = r
+    return (dq.reshape(B, T, H, dk), dkk.reshape(B, T, H, dk), dvv.reshape(B, T, H, dv),
+            dg.reshape(B, T, H, dk), db.reshape(B, T, H), dh0)
