@@ -789,6 +789,91 @@ def measure_speculative(steps, warmup, K=4, cpu=True):
     return out
 
 
+def measure_backward(name, steps, warmup, cpu=True, cpu_seconds=10.0):
+    """The backward pass (kda_bwd) on a prefill workload: per step one call with
+    seeded upstream gradients do (dtype of q) and dhT; inputs already on the device."""
+    import torch
+    import kimi_delta_attention_28_b200 as kda
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    kda.load_library()
+    w, inp = workload_inputs(name, dev)
+    B, T, H, dk = inp["q"].shape
+    dv = inp["v"].shape[-1]
+    cu = inp["cu_seqlens"]
+    N = B if cu is None else cu.numel() - 1
+    nseq = 0 if cu is None else N
+    gen = torch.Generator(device=dev).manual_seed(w.seed + 7)
+    do = torch.randn(B, T, H, dv, generator=gen, device=dev).to(w.dtype)
+    dhT = 0.1 * torch.randn(N, H, dk, dv, generator=gen, device=dev)
+    ws = torch.empty(kda.bwd_workspace_size(B, T, H, dk, dv, nseq, w.dtype), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    res = None
+    for _ in range(warmup):
+        res = kda.kda_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], cu, do,
+                          dhT, workspace=ws)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.02)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    t_wall0 = time.perf_counter()
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        res = kda.kda_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], cu, do,
+                          dhT, workspace=ws)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.perf_counter()
+    clocks.stop()
+    assert kda.device_error() == 0
+    ms = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    units = B * T * H
+    # fp32 work per token-head as executed: the forward recurrence twice (the checkpoint
+    # pass and the chunk recompute, ~4 d^2 each) and the reverse step (~10 d^2)
+    flops = units * 18.0 * dk * dv
+    peak_fp32 = 148 * 128 * 2 * 1.965e9 / 1e12    # CUDA-core fp32 FMA peak, TFLOP/s
+    tf = flops / (ms * 1e-3) / 1e12
+    out = {"metric": "KDA backward tokens/s (gradients of q, k, v, g, beta, h0)",
+           "value": B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+           "warmup": warmup, "config": prefill_config(w, inp, 1),
+           "roofline": {"bound": "alu", "kernel": "kda_bwd_slice_kernel + kda_bwd_reduce_kernel",
+                        "achieved": tf, "peak": peak_fp32, "unit": "TFLOP/s",
+                        "frac": tf / peak_fp32, "traffic": None,
+                        "algorithmic_flops_per_launch": flops,
+                        "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz "
+                                       "(CUDA-core fp32, nominal clock)",
+                        "flops_rule": "18 d_k d_v per token-head: two forward recurrences "
+                                      "(checkpoints, chunk recompute) and the reverse step"},
+           "gpu_launches": steps * (2 + (1 if cu is not None else 0)),
+           "clocks": clocks.summary(t_wall0, t_wall1)}
+    if cpu:
+        import numpy as np
+        import oracle
+        # whole sequence 0, all heads (a gradient depends on every later token)
+        s0 = lambda x: x[:1].contiguous()  # noqa: E731
+        t0 = time.perf_counter()
+        ref = oracle.kda_bwd(s0(inp["q"]), s0(inp["k"]), s0(inp["v"]), s0(inp["g"]),
+                             s0(inp["beta"]), None if inp["h0"] is None else s0(inp["h0"]),
+                             s0(do), s0(dhT))
+        el = time.perf_counter() - t0
+        par = {"tolerance": "fp32-stored gradients rel-L2 <= 1e-4; bf16-stored rel-L2 <= 1e-2",
+               "sample": "all heads of sequence 0, every token"}
+        for nm, got, r in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), res, ref):
+            if got is not None:
+                par[nm] = _err(got[:1].double().cpu().numpy(), r.reshape(got[:1].shape))
+        out["cpu_baseline"] = {"value": T / el, "unit": "tokens/s",
+                               "cores": min(H, oracle.threads_available()), "kind": "oracle",
+                               "sample": f"sequence 0 ({T} tokens x {H} heads), {el:.1f} s; "
+                                         "fp64 reverse accumulation, OpenMP over heads",
+                               "parity": par}
+        del np
+    return out
+
+
 def speculative_cpu_baseline(w, drafts, accs, S0, S_gpu, o_last, K, nsteps, nchains=64):
     """The oracle on 64 sampled (sequence, head) chains over every round the GPU ran,
     from the initial states: each chain's accepted tokens, round after round, then the
@@ -969,6 +1054,8 @@ def main():
             _free_device_memory()
             r = measure_speculative(200, 20, cpu=cpu)
             nested["speculative"] = r
+            _free_device_memory()
+            nested["backward"] = measure_backward("prefill", 5, 2, cpu=cpu)
             out["workloads"] = nested
         if out is not None:
             print(json.dumps(out), flush=True)

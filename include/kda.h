@@ -235,6 +235,72 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
                            int dv, int dtype, void *stream);
 
 /*
+ * Context parallelism across devices: one sequence batch split in time over
+ * `world` ranks (rank r holds tokens [r T_local, (r + 1) T_local) of every
+ * sequence).  Source: the "Kimi K3" field notes, panel "传固定状态片段" (pass
+ * fixed-size state fragments): each rank summarises its stretch as a cumulative
+ * transform plus a state grown from zero, one all-gather exchanges those
+ * fixed-size summaries, and each rank combines the summaries of the ranks before it
+ * in prefix order to get its starting state.  This works because every chunk's map
+ * on the state is affine, S -> P S + R (panel "KDA 单头递归" unrolled over a chunk).
+ *
+ *   1. kda_cp_local_map: the intra-chunk pass over the local tokens, then the map
+ *      pass over the whole local stretch: seg_map [B, H, d_k, 2 d_v] fp32 = [R | P]
+ *      per (sequence, head) -- R the local final state from zero, P the linear part.
+ *      The chunk records stay in `workspace` for step 3.
+ *   2. (caller) all-gather seg_map over the ranks, in rank order, into
+ *      maps [world, B, H, d_k, 2 d_v] -- 128 KiB per (sequence, head) per rank.
+ *   3. kda_cp_finish: S_in = fold over ranks 0 .. rank-1 of S <- P_s S + R_s from h0
+ *      (the sequences' initial states, NULL: zero; the same on every rank), written
+ *      to s_in [B, H, d_k, d_v]; then the state pass from S_in over the local
+ *      records, writing the local outputs o [B, T_local, H, d_v] and hT, the state
+ *      after the local stretch (on the last rank: the sequences' final states).
+ *      maps may be NULL on rank 0.
+ * Fixed-length input and the tensor-core path only (bf16, d_k = d_v = 128), else
+ * KDA_ERR_UNSUPPORTED_SHAPE.  The workspace must hold kda_cp_workspace_size bytes
+ * and be the same buffer, unchanged, in steps 1 and 3.  s_in must not alias h0, o
+ * or hT.  Alignment as kda_fwd; seg_map, maps and s_in 16 bytes.
+ */
+size_t kda_cp_workspace_size(int B, int T_local, int H, int dk, int dv, int dtype);
+kda_status kda_cp_local_map(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, int B, int T_local, int H, int dk, int dv,
+                            int dtype, float *seg_map, void *workspace, size_t ws_bytes,
+                            void *stream);
+kda_status kda_cp_finish(const float *maps, int rank, int world, const float *h0, float *s_in,
+                         int B, int T_local, int H, int dk, int dv, int dtype, void *o,
+                         float *hT, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Backward pass: the gradient of a loss L through kda_fwd.  Given grad_o = dL/do and
+ * grad_hT = dL/dhT (NULL: zero), writes dL/dq, dL/dk, dL/dv (dtype of q, k, v),
+ * dL/dg, dL/dbeta (fp32) and dL/dh0 (fp32, NULL to skip).  Same inputs, layouts,
+ * packed-sequence rules and alignment as kda_fwd; grad_o [B, T, H, d_v] has the
+ * dtype of q; grad_hT, grad_h0 [N, H, d_k, d_v].  No gradient buffer may alias an
+ * input.  The workspace must hold kda_bwd_workspace_size(...) bytes: the state every
+ * 8 tokens of every (sequence, head) plus partial sums (about 16 KiB per
+ * token-head at d = 128).
+ *
+ * What it computes is the chain rule through the recurrence (panel "KDA 单头递归"),
+ * token by token from the last to the first, with G = dL/dS_t, S' = Diag(exp g_t)
+ * S_{t-1}, u = S'^T k and delta = v - u:
+ *     G += q do^T;  dq = S_t do;  w = G delta;  dbeta = k . w;  dv = beta G^T k;
+ *     dk = beta w - S' dv;  G' = G - k dv^T;  dg_i = sum_j S'_ij G'_ij;
+ *     G = Diag(exp g) G';  and dh0 = G after the first token.
+ * The source pages name the training kernel ("FlashKDA / FLA" panel) but give no
+ * formulas for it; this is the gradient of the recurrence they print, in fp32 on
+ * CUDA cores (one CTA per (sequence, head) and 32 value columns, the states of
+ * every 8-token chunk recomputed from stored checkpoints).  All head sizes and
+ * dtypes of kda_fwd are supported.
+ */
+size_t kda_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype);
+kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
+                   int B, int T, int H, int dk, int dv, int dtype, const void *grad_o,
+                   const float *grad_hT, void *grad_q, void *grad_k, void *grad_v,
+                   float *grad_g, float *grad_beta, float *grad_h0, void *workspace,
+                   size_t ws_bytes, void *stream);
+
+/*
  * Speculative decoding: verify K drafted tokens per sequence, then commit the
  * accepted prefix.  Source: the "Kimi K3" open-weights field notes, panel
  * "目标模型太大，缓存和草稿都必须理解 KDA": with a draft model the KDA recurrent

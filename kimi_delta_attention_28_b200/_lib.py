@@ -47,6 +47,14 @@ SIGNATURES = {
     "kda_fwd_inter": ([_VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP], _I),
     "kda_decode_step": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP], _I),
     "kda_get_last_device_error": ([_VP], _I),
+    "kda_cp_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
+    "kda_cp_local_map": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _SZ, _VP],
+                         _I),
+    "kda_cp_finish": ([_VP, _I, _I, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP],
+                      _I),
+    "kda_bwd_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
+    "kda_bwd": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP,
+                 _VP, _VP, _VP, _VP, _VP, _SZ, _VP], _I),
     "kda_decode_verify": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP], _I),
     "kda_decode_commit": ([_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP], _I),
     "kda_fwd_noalloc": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP,
@@ -364,6 +372,122 @@ def kda_decode_step(q, k, v, g, beta, S, o=None):
     _check(lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
                                N, H, dk, dv, dt, _stream(dev)), "kda_decode_step")
     return o
+
+
+def cp_workspace_size(B: int, T_local: int, H: int, dk: int, dv: int,
+                      dtype: torch.dtype) -> int:
+    return int(load_library().kda_cp_workspace_size(B, T_local, H, dk, dv, _dtype_code(dtype)))
+
+
+def kda_cp_local_map(q, k, v, g, beta, *, workspace):
+    """Step 1 of context parallelism: the local stretch's map [R | P] per (sequence,
+    head), fp32 [B, H, d_k, 2 d_v]; the chunk records stay in ``workspace``."""
+    lib = load_library()
+    dev = q.device
+    B, T, H, dk, dv, _, _ = _prefill_shapes(q, k, v, g, beta, workspace=workspace)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    seg_map = torch.empty(B, H, dk, 2 * dv, dtype=torch.float32, device=dev)
+    _check(lib.kda_cp_local_map(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), B, T, H, dk, dv,
+                                _dtype_code(q.dtype), _ptr(seg_map), _ptr(workspace),
+                                workspace.numel(), _stream(dev)), "kda_cp_local_map")
+    return seg_map
+
+
+def kda_cp_finish(maps, rank, h0, *, B, T_local, H, dk, dv, dtype, o, hT, workspace):
+    """Step 3: fold the gathered maps [world, B, H, d_k, 2 d_v] of ranks before `rank`
+    onto h0, then run the local state pass; writes o [B, T_local, H, d_v] and hT (the
+    state after the local stretch).  Returns (o, hT, s_in)."""
+    lib = load_library()
+    dev = o.device
+    world = maps.shape[0]
+    _shape(maps, "maps", (world, B, H, dk, 2 * dv))
+    _shape(h0, "h0", (B, H, dk, dv))
+    _shape(o, "o", (B, T_local, H, dv))
+    _shape(hT, "hT", (B, H, dk, dv))
+    _need(maps, "maps", torch.float32, dev)
+    _need(h0, "h0", torch.float32, dev)
+    _need(o, "o", dtype, dev)
+    _need(hT, "hT", torch.float32, dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    s_in = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    _check(lib.kda_cp_finish(_ptr(maps), rank, world, _ptr(h0), _ptr(s_in), B, T_local, H, dk,
+                             dv, _dtype_code(dtype), _ptr(o), _ptr(hT), _ptr(workspace),
+                             workspace.numel(), _stream(dev)), "kda_cp_finish")
+    return o, hT, s_in
+
+
+def gather_segment_maps(seg_map, group=None):
+    """Step 2: all-gather every rank's [R | P] in rank order -> [world, ...] (one
+    collective through torch.distributed; NCCL on GPUs)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(seg_map) for _ in range(world)]
+    dist.all_gather(parts, seg_map.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+def kda_fwd_context_parallel(q, k, v, g, beta, h0=None, *, group=None, workspace=None):
+    """Prefill of a batch split in time over the ranks of ``group``: this rank holds
+    tokens [rank T_local, (rank + 1) T_local) of every sequence (q, k, v, g [B, T_local,
+    H, d]; beta [B, T_local, H]); h0 [B, H, d_k, d_v] are the sequences' initial states
+    (the same on every rank; None: zeros).  Returns this rank's outputs o and the state
+    after its stretch (on the last rank: the final states)."""
+    import torch.distributed as dist
+    B, T, H, dk, dv, _, _ = _prefill_shapes(q, k, v, g, beta, h0, workspace=workspace)
+    dev = q.device
+    if workspace is None:
+        workspace = torch.empty(max(cp_workspace_size(B, T, H, dk, dv, q.dtype), 256),
+                                dtype=torch.uint8, device=dev)
+    seg_map = kda_cp_local_map(q, k, v, g, beta, workspace=workspace)
+    maps = gather_segment_maps(seg_map, group)
+    rank = dist.get_rank(group)
+    o = torch.empty(B, T, H, dv, dtype=q.dtype, device=dev)
+    hT = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    kda_cp_finish(maps, rank, h0, B=B, T_local=T, H=H, dk=dk, dv=dv, dtype=q.dtype, o=o, hT=hT,
+                  workspace=workspace)
+    return o, hT
+
+
+def bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
+                       dtype: torch.dtype) -> int:
+    return int(load_library().kda_bwd_workspace_size(B, T, H, dk, dv, num_seqs,
+                                                     _dtype_code(dtype)))
+
+
+def kda_bwd(q, k, v, g, beta, h0, cu_seqlens, grad_o, grad_hT=None, *, workspace=None):
+    """Gradient of a loss through kda_fwd: given grad_o = dL/do [B, T, H, d_v] (dtype of
+    q) and grad_hT = dL/dhT [N, H, d_k, d_v] fp32 (None: zero), returns (dq, dk, dv, dg,
+    dbeta, dh0): dq, dk, dv in the dtype of q, the rest fp32 (dh0 None when h0 is None)."""
+    lib = load_library()
+    dev = q.device
+    B, T, H, dk, dv, num_seqs, N = _prefill_shapes(q, k, v, g, beta, h0, cu_seqlens,
+                                                   workspace=workspace)
+    _shape(grad_o, "grad_o", (B, T, H, dv))
+    _shape(grad_hT, "grad_hT", (N, H, dk, dv))
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (grad_o, "grad_o")):
+        _need(t, n, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(h0, "h0", torch.float32, dev)
+    _need(grad_hT, "grad_hT", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    dq, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg, db = torch.empty_like(g), torch.empty_like(beta)
+    dh0 = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev) if h0 is not None else None
+    need = bwd_workspace_size(B, T, H, dk, dv, num_seqs, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.kda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                       _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, _dtype_code(q.dtype),
+                       _ptr(grad_o), _ptr(grad_hT), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg),
+                       _ptr(db), _ptr(dh0), _ptr(workspace), workspace.numel(), _stream(dev)),
+           "kda_bwd")
+    return dq, dk_, dv_, dg, db, dh0
 
 
 def _draft_shapes(k, v, g, beta, S, q=None):

@@ -3,6 +3,8 @@
 // Host-side argument validation, workspace layout and kernel dispatch.  All
 // kernels are compiled into this one translation unit so they can share the
 // device error word without relocatable device code.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -11,6 +13,7 @@
 #include <mutex>
 
 #include "../../include/kda.h"
+#include "kda_bwd.cuh"
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
 #include "kda_prefill_simt.cuh"
@@ -199,6 +202,54 @@ kda_status launch_state(kda::tc::StateArgs a, long long units, cudaStream_t s) {
 }
 
 
+// ---------------------------------------------------------------------------
+// Backward pass.  Workspace: the forward path's header region (offsets check and
+// chunk table of the packed layout), then the state checkpoints every bwd::CB tokens
+// of every (sequence, head), then the per-slice partial sums of dq, dk, dg, dbeta.
+// ---------------------------------------------------------------------------
+struct BwdLayout {
+    size_t hdr_end, ckpt, part, total;
+};
+BwdLayout bwd_layout(int B, int T, int H, int dk, int num_seqs, int dtype) {
+    BwdLayout L{};
+    const WsLayout F = ws_layout(B, T, H, dk, num_seqs, dtype, 1);
+    L.hdr_end = F.recs;   // header, sequence offsets and chunk table only
+    const long long ntok = (long long)B * T, N = num_seqs > 0 ? num_seqs : B;
+    const long long slots = ntok / kda::bwd::CB + N + 1;
+    L.ckpt = round_up(L.hdr_end, 256);
+    L.part = round_up(L.ckpt + (size_t)slots * H * dk * dk * sizeof(float), 256);
+    L.total = L.part + (size_t)(dk / kda::bwd::SLC) * ntok * H * (3 * dk + 1) * sizeof(float);
+    return L;
+}
+
+template <int D, typename TIn>
+kda_status launch_bwd(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *h0, const int32_t *cu,
+                             const int *hdr, const void *dO, const float *dhT, int T, int H,
+                             long long ntok, long long chains, float *ckpt, float *part,
+                             void *dq, void *dkk, void *dvv, float *dg, float *db, float *dh0,
+                             int *err, cudaStream_t s) {
+    using namespace kda::bwd;
+    const size_t smem = sizeof(BwdSmem<D>);
+    auto kern = kda_bwd_slice_kernel<D, TIn>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return KDA_ERR_CUDA;
+    const long long grid = chains * (D / SLC);
+    if (grid > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    kern<<<(unsigned)grid, 2 * D, smem, s>>>(
+        static_cast<const TIn *>(q), static_cast<const TIn *>(k), static_cast<const TIn *>(v), g,
+        beta, h0, cu, hdr, static_cast<const TIn *>(dO), dhT, T, H, ckpt, part,
+        static_cast<TIn *>(dvv), dh0, ntok, err);
+    kda_status st = launch_status();
+    if (st != KDA_OK) return st;
+    const long long n = ntok * H * (D + 1);
+    if (n == 0) return KDA_OK;
+    kda_bwd_reduce_kernel<D, TIn><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+        part, ntok, H, static_cast<TIn *>(dq), static_cast<TIn *>(dkk), dg, db);
+    return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -276,6 +327,43 @@ static kda_status validate_fwd(const void *q, const void *k, const void *v, cons
     return KDA_OK;
 }
 
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry points (no
+// -lcuda); null if the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+        }
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// Tensor map of a [B, T, H, 128] input seen as the 4-D tensor (channel, head, token,
+// sequence), innermost first: boxes of `box_c` channels x 1 head x `box_t` tokens x 1
+// sequence.  bf16 inputs use 64-channel boxes with the 128-byte swizzle (the tensor
+// core's K-major operand layout); fp32 g uses whole 512-byte rows without swizzle.
+bool encode_input_map(CUtensorMap *m, const void *base, bool bf16, int H, long long T, int B,
+                      int box_c, int box_t) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t es = bf16 ? 2 : 4, D = kda::tc::D;
+    const cuuint64_t dims[4] = {D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {D * es, (cuuint64_t)H * D * es, (cuuint64_t)T * H * D * es};
+    const cuuint32_t box[4] = {(cuuint32_t)box_c, 1, (cuuint32_t)box_t, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Tensor-core path, phase 1: chunk map (varlen) and the per-(chunk, head) records.
 static kda_status tc_intra(const void *q, const void *k, const void *v, const float *g,
                            const float *beta, const int32_t *cu, int N, int T, int H,
@@ -308,10 +396,20 @@ static kda_status tc_intra(const void *q, const void *k, const void *v, const fl
     const int sms = device_sms();
     const long long cap = 2LL * (sms > 0 ? sms : 148);
     const unsigned grid = (unsigned)(items < cap ? items : cap);
-    kda_tc_prep_kernel<<<grid, 256, smem, s>>>(
-        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-        static_cast<const __nv_bfloat16 *>(v), g, beta, T, H, cps, (int)L.max_chunks, hdr,
-        cu ? chunks : nullptr, ws + L.recs, device_error_word());
+    // inputs as (channel, head, token, sequence); packed sequences are one long sequence
+    // whose per-chunk bounds the kernel applies itself
+    const int nb = cu ? 1 : N;
+    CUtensorMap tq, tk, tv, tg;
+    if (!encode_input_map(&tq, q, true, H, T, nb, 64, C) ||
+        !encode_input_map(&tk, k, true, H, T, nb, 64, C) ||
+        !encode_input_map(&tv, v, true, H, T, nb, 64, C) ||
+        !encode_input_map(&tg, g, false, H, T, nb, D, C / 2))
+        return KDA_ERR_CUDA;
+    int *err = device_error_word();
+    if (!err) return KDA_ERR_CUDA;
+    kda_tc_prep_kernel<<<grid, 256, smem, s>>>(tq, tk, tv, tg, beta, T, H, cps,
+                                               (int)L.max_chunks, hdr, cu ? chunks : nullptr,
+                                               ws + L.recs, err);
     return launch_status();
 }
 
@@ -611,6 +709,141 @@ kda_status kda_decode_commit(const void *k, const void *v, const float *g, const
     }
 #undef KDA_COM
     return launch_status();
+}
+
+size_t kda_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype) {
+    if (B < 0 || T < 0 || num_seqs < 0) return 0;
+    if (check_shape(H, dk, dv, dtype) != KDA_OK) return 0;
+    if (num_seqs > 0 && B != 1) return 0;
+    return bwd_layout(B, T, H, dk, num_seqs, dtype).total;
+}
+
+kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
+                   int B, int T, int H, int dk, int dv, int dtype, const void *grad_o,
+                   const float *grad_hT, void *grad_q, void *grad_k, void *grad_v,
+                   float *grad_g, float *grad_beta, float *grad_h0, void *workspace,
+                   size_t ws_bytes, void *stream) {
+    int N;
+    WsLayout F;
+    // the forward's checks cover the inputs; the outputs are checked here
+    kda_status st = validate_fwd(q, k, v, g, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv,
+                                 dtype, grad_q, grad_h0, reinterpret_cast<void *>(uintptr_t(256)),
+                                 SIZE_MAX, true, false, &N, &F, 1);
+    if (st != KDA_OK) return st;
+    const long long ntok = (long long)B * T;
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    if (ntok > 0 && (!grad_o || !grad_q || !grad_k || !grad_v || !grad_g || !grad_beta))
+        return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(grad_o, es) || !aligned_to(grad_q, es) || !aligned_to(grad_k, es) ||
+        !aligned_to(grad_v, es) || !aligned_to(grad_g, 4) || !aligned_to(grad_beta, 4) ||
+        !aligned_to(grad_hT, 16) || !aligned_to(grad_h0, 16))
+        return KDA_ERR_MISALIGNED;
+    const void *ins[] = {q, k, v, g, beta, h0, grad_o, grad_hT};
+    const void *outs[] = {grad_q, grad_k, grad_v, grad_g, grad_beta, grad_h0};
+    for (const void *o : outs)
+        for (const void *i : ins)
+            if (o && o == i) return KDA_ERR_INVALID_ARG;
+    const BwdLayout L = bwd_layout(B, T, H, dk, cu_seqlens ? num_seqs : 0, dtype);
+    if (!workspace || ws_bytes < L.total) return KDA_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned_to(workspace, 16)) return KDA_ERR_MISALIGNED;
+    if (N == 0 || ntok == 0 && !grad_h0) return KDA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *hdr = reinterpret_cast<int *>(ws + F.hdr);
+    int *err = device_error_word();
+    if (!err) return KDA_ERR_CUDA;
+    if (cu_seqlens) {   // offsets check (the chunk table it also writes is not used here)
+        kda::tc::kda_chunk_map_kernel<<<1, 1024, 0, s>>>(
+            cu_seqlens, N, T, hdr, reinterpret_cast<int *>(ws + F.seq_off),
+            reinterpret_cast<kda::tc::ChunkLoc *>(ws + F.chunks), (int)F.max_chunks, err,
+            ERRBIT_SEQLENS);
+        if ((st = launch_status()) != KDA_OK) return st;
+    }
+    float *ckpt = reinterpret_cast<float *>(ws + L.ckpt);
+    float *part = reinterpret_cast<float *>(ws + L.part);
+    const long long chains = (long long)N * H;
+#define KDA_BWD(DD, TT)                                                                    \
+    return launch_bwd<DD, TT>(q, k, v, g, beta, h0, cu_seqlens, hdr, grad_o, grad_hT, T, H, \
+                              ntok, chains, ckpt, part, grad_q, grad_k, grad_v, grad_g,     \
+                              grad_beta, grad_h0, err, s)
+    if (dtype == KDA_DTYPE_BF16) {
+        if (dk == 32) KDA_BWD(32, __nv_bfloat16);
+        if (dk == 64) KDA_BWD(64, __nv_bfloat16);
+        KDA_BWD(128, __nv_bfloat16);
+    }
+    if (dk == 32) KDA_BWD(32, float);
+    if (dk == 64) KDA_BWD(64, float);
+    KDA_BWD(128, float);
+#undef KDA_BWD
+}
+
+// ---------------------------------------------------------------------------
+// Context parallelism across devices (fixed-length input, tensor-core path).
+// ---------------------------------------------------------------------------
+size_t kda_cp_workspace_size(int B, int T_local, int H, int dk, int dv, int dtype) {
+    if (!is_tc_path(dtype, dk) || dk != dv) return 0;
+    return kda_fwd_segmented_workspace_size(B, T_local, H, dk, dv, 0, dtype, 1);
+}
+
+kda_status kda_cp_local_map(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, int B, int T_local, int H, int dk, int dv,
+                            int dtype, float *seg_map, void *workspace, size_t ws_bytes,
+                            void *stream) {
+    int N;
+    WsLayout L;
+    kda_status st = validate_fwd(q, k, v, g, beta, nullptr, nullptr, 0, B, T_local, H, dk, dv,
+                                 dtype, nullptr, nullptr, workspace, ws_bytes, true, false, &N,
+                                 &L, 1);
+    if (st != KDA_OK) return st;
+    if (!is_tc_path(dtype, dk)) return KDA_ERR_UNSUPPORTED_SHAPE;
+    if (N > 0 && !seg_map) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(seg_map, 16)) return KDA_ERR_MISALIGNED;
+    if (N == 0) return KDA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = tc_intra(q, k, v, g, beta, nullptr, N, T_local, H, L, workspace, s)) != KDA_OK)
+        return st;
+    // the map pass over the whole local segment: [R | P] per (sequence, head)
+    using namespace kda::tc;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    StateArgs m{};
+    m.recs = ws + L.recs;
+    m.T = T_local;
+    m.H = H;
+    m.cps = (T_local + C - 1) / C;
+    m.hdr = reinterpret_cast<int *>(ws + L.hdr);
+    m.seq_off = reinterpret_cast<int *>(ws + L.seq_off);
+    m.nseg = 1;
+    m.mode = kStateMap;
+    m.seg_map = seg_map;
+    m.ntok = (long long)N * T_local;
+    m.max_chunks = (int)L.max_chunks;
+    return launch_state<32>(m, (long long)N * H, s);
+}
+
+kda_status kda_cp_finish(const float *maps, int rank, int world, const float *h0, float *s_in,
+                         int B, int T_local, int H, int dk, int dv, int dtype, void *o,
+                         float *hT, void *workspace, size_t ws_bytes, void *stream) {
+    if (world < 1 || rank < 0 || rank >= world) return KDA_ERR_INVALID_ARG;
+    if (rank > 0 && !maps) return KDA_ERR_INVALID_ARG;
+    int N;
+    WsLayout L;
+    kda_status st = validate_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, h0, nullptr, 0, B,
+                                 T_local, H, dk, dv, dtype, o, hT, workspace, ws_bytes, false,
+                                 true, &N, &L, 1);
+    if (st != KDA_OK) return st;
+    if (!is_tc_path(dtype, dk)) return KDA_ERR_UNSUPPORTED_SHAPE;
+    if (N > 0 && !s_in) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(maps, 16) || !aligned_to(s_in, 16)) return KDA_ERR_MISALIGNED;
+    if (s_in == h0 || s_in == hT || (const void *)s_in == o) return KDA_ERR_INVALID_ARG;
+    if (N == 0) return KDA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long chains = (long long)N * H;
+    if (chains > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    kda::tc::kda_cp_combine_kernel<<<dim3((unsigned)chains, kda::tc::D / 32), 256, 0, s>>>(
+        h0, maps, s_in, rank, (int)chains);
+    if ((st = launch_status()) != KDA_OK) return st;
+    return tc_inter(s_in, nullptr, N, T_local, H, L, o, hT, workspace, s);
 }
 
 kda_status kda_get_last_device_error(void *stream) {

@@ -8,6 +8,8 @@
 //   C regs: (gid, 2tig), (gid, 2tig+1), (gid+8, 2tig), (gid+8, 2tig+1).
 #pragma once
 
+#include <cuda.h>   // CUtensorMap (the type only; maps are encoded through the runtime's
+                    // driver entry points)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -157,6 +159,20 @@ KDA_DEVINL bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
         if (global_timer_ns() - t0 > kWaitLimitNs) return false;
     return true;
 }
+// Tiled 4-D tensor copy global -> this CTA's shared memory by the tensor-memory-access
+// engine, completing on `bar`: the box of the tensor map `tm` at coordinates
+// (c0, c1, c2, c3), innermost first.  Coordinates past the tensor's extent read zeros.
+// No cluster multicast.
+KDA_DEVINL void tma_load_4d(void *smem_dst, const CUtensorMap *tm, int c0, int c1, int c2,
+                            int c3, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];\n"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1),
+          "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
 KDA_DEVINL void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar) {
     asm volatile(

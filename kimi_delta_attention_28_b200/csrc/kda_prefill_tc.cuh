@@ -161,16 +161,18 @@ constexpr int LDA = C + 8;      // padded bf16 row stride of the 64x64 blocks (1
 __constant__ int2 kPairs[6] = {{1, 0}, {2, 0}, {3, 0}, {2, 1}, {3, 1}, {3, 2}};
 
 struct PrepSmem {
-    // Five 16 KB tiles, reused across phases (an item's inputs arrive as: g rows 0-31
-    // in ka and rows 32-63 in xk, 512-byte rows; k in qa, q in kb (swz128); V in xv):
-    //   ka: g (rows 0-31); k*exp(G_r - G_ref(a)) (swz128); then T' = (I + A)^-1 Diag(b)
-    //       (first 8 KB, umma_k128)
-    //   qa: raw k; q*exp(G_r - G_ref(a)) (swz128); then, with kb, [W|U] (four umma_k128
-    //       planes)
-    //   kb: raw q; k*exp(G_ref(b) - G_i) (swz128)
-    //   xk: g (rows 32-63); K*exp(G) (umma_k128 planes); then Kt (umma_k128 planes)
-    //   xv: V (umma_k128 planes); then Qg (swz128).  xk and xv are contiguous: together
-    //       they are the N = 256 right operand [K*exp G | V] of the [W|U] product.
+    // Five 16 KB tiles, reused across phases.  Every bf16 tile uses the tensor core's
+    // K-major 128-byte-swizzled layout (umma_k128: two 64-column planes of 128-byte
+    // rows), which is also the layout the tensor-memory-access engine writes with its
+    // 128-byte swizzle, and in which ldmatrix reads 8 rows of a column chunk without
+    // bank conflicts.  An item's inputs arrive as: g rows 0-31 in ka and rows 32-63 in
+    // xk (fp32, 512-byte rows); k in qa, q in kb; V in xv.
+    //   ka: g (rows 0-31); k*exp(G_r - G_ref(a)); then T' = (I + A)^-1 Diag(b) (first 8 KB)
+    //   qa: raw k; q*exp(G_r - G_ref(a)); then, with kb, [W|U] (four planes)
+    //   kb: raw q; k*exp(G_ref(a) - G_r)
+    //   xk: g (rows 32-63); K*exp(G); then Kt
+    //   xv: V; then Qg.  xk and xv are contiguous: together they are the N = 256 right
+    //       operand [K*exp G | V] of the [W|U] product.
     uint8_t ka[C * D * 2], qa[C * D * 2], kb[C * D * 2], xk[C * D * 2], xv[C * D * 2];
     __nv_bfloat16 akkn[C * LDA];   // -b_r A_ri, sub-tile blocks b < a (bf16)
     uint8_t aqk[C * C * 2];        // masked query-key block, umma_k128 plane (bf16)
@@ -185,12 +187,13 @@ struct PrepSmem {
     } u;
     float beta[C];
     uint64_t mma_bar;              // tcgen05 completion barrier
+    uint64_t ld_bar[4];            // input loads: g rows 0-31, g rows 32-63, k and q, V
     uint32_t tmem_slot;            // tensor-memory base address (written by tcgen05.alloc)
 };
 
 __global__ void __launch_bounds__(256, 2)
-kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                   const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
+kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                    const float *__restrict__ beta, int T, int H, int cps, int slots,
                    const int *__restrict__ hdr, const ChunkLoc *__restrict__ chunks,
                    uint8_t *__restrict__ recs, int *err_word) {
@@ -204,12 +207,11 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     if (chunks && !hdr[0]) return;
     const int items = (chunks ? min(hdr[1], slots) : slots) * H;
     if ((int)blockIdx.x >= items) return;
-    const size_t rowstride = (size_t)H * D;  // elements between consecutive tokens
     const uint32_t s_ka = smem_u32(sm.ka), s_qa = smem_u32(sm.qa), s_kb = smem_u32(sm.kb);
 
     struct Item {
         int t0, len, h;
-        size_t base;       // element offset of (token t0, head h, channel 0)
+        int tl, b;         // the chunk's token and batch coordinates in the tensor maps
         uint8_t *rec;
     };
     auto locate = [&](int item) {
@@ -219,54 +221,64 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         if (chunks) {
             it.t0 = chunks[cid].t0;
             it.len = chunks[cid].len;
+            it.tl = it.t0;
+            it.b = 0;
         } else {
             const int n = cid / cps, j = cid % cps;
             it.t0 = n * T + j * C;
             it.len = min(C, T - j * C);
+            it.tl = j * C;
+            it.b = n;
         }
-        it.base = ((size_t)it.t0 * H + it.h) * D;
         it.rec = recs + ((size_t)cid * H + it.h) * REC_BYTES;
         return it;
     };
-    // input loads (16-byte cp.async, zero-filled past len), in the pieces the tail of
-    // the previous item releases them
-    auto load_g_half = [&](const Item &it, int half) {   // g rows 32 half .. +31
-        uint8_t *dst0 = half ? sm.xk : sm.ka;
+    // Input loads by the tensor-memory-access engine (one thread issues them), in four
+    // groups that complete on their own barriers and are issued as the previous item's
+    // last phases release the tiles:
+    //   ld_bar[0]: g rows 0-31 -> ka      ld_bar[1]: g rows 32-63 -> xk  (fp32 rows)
+    //   ld_bar[2]: k -> qa, q -> kb       ld_bar[3]: V -> xv  (two 128B-swizzled planes)
+    // Rows past the end of the tensor (fixed-length input: past T) arrive as zeros;
+    // rows past the end of a packed sequence hold the next sequence's tokens and are
+    // neutralised in P1: their g counts as zero and their beta is zero, so they neither
+    // decay nor write the state.  beta comes by 4-byte cp.async beside k and q.
+    uint32_t pend = 0, pend_par = 0;   // load groups in flight and the parity each completes
+    auto issue = [&](int grp, const Item &it, uint32_t par) {
+        if (tid == 0) {
+            uint64_t *bar = &sm.ld_bar[grp];
+            fence_proxy_async_smem();   // earlier generic accesses of the tile come first
+            if (grp < 2) {
+                mbar_arrive_expect_tx(bar, 32 * D * 4);
+                tma_load_4d(grp ? sm.xk : sm.ka, &tm_g, 0, it.h, it.tl + 32 * grp, it.b, bar);
+            } else if (grp == 2) {
+                mbar_arrive_expect_tx(bar, 2 * C * D * 2);
 #pragma unroll
-        for (int m = 0; m < 32 * (D / 4) / 256; ++m) {
-            const int i = tid + m * 256, rr = i / (D / 4), c4 = (i % (D / 4)) * 4;
-            const int r = 32 * half + rr;
-            const bool ok = r < it.len;
-            cp_async16(dst0 + rr * (D * 4) + c4 * 4, ok ? g + it.base + r * rowstride + c4 : g,
-                       ok ? 16 : 0);
+                for (int pl = 0; pl < 2; ++pl) {
+                    tma_load_4d(sm.qa + pl * C * 128, &tm_k, 64 * pl, it.h, it.tl, it.b, bar);
+                    tma_load_4d(sm.kb + pl * C * 128, &tm_q, 64 * pl, it.h, it.tl, it.b, bar);
+                }
+            } else {
+                mbar_arrive_expect_tx(bar, C * D * 2);
+#pragma unroll
+                for (int pl = 0; pl < 2; ++pl)
+                    tma_load_4d(sm.xv + pl * C * 128, &tm_v, 64 * pl, it.h, it.tl, it.b, bar);
+            }
         }
+        if (grp == 2) {
+            if (tid < C) {
+                const bool in = tid < it.len;
+                cp_async4(&sm.beta[tid], in ? beta + (size_t)(it.t0 + tid) * H + it.h : beta,
+                          in ? 4 : 0);
+            }
+            cp_async_commit();
+        }
+        pend |= 1u << grp;
+        pend_par = (pend_par & ~(1u << grp)) | ((par & 1u) << grp);
     };
-    auto load_kq = [&](const Item &it) {                 // k -> qa, q -> kb (swz128), beta
-#pragma unroll
-        for (int m = 0; m < 2 * C * (D / 8) / 256; ++m) {
-            const int i = tid + m * 256, w = i / (C * (D / 8)), rem = i % (C * (D / 8));
-            const int r = rem / (D / 8), c8 = (rem % (D / 8)) * 8;
-            const bool ok = r < it.len;
-            const __nv_bfloat16 *src = w ? q : k;
-            cp_async16((w ? sm.kb : sm.qa) + swz128(r, c8),
-                       ok ? src + it.base + r * rowstride + c8 : src, ok ? 16 : 0);
-        }
-        if (tid < C) {
-            const bool ok = tid < it.len;
-            cp_async4(&sm.beta[tid], ok ? beta + (size_t)(it.t0 + tid) * H + it.h : beta,
-                      ok ? 4 : 0);
-        }
-    };
-    // V -> xv (umma_k128), in a cp.async group of its own: it is needed only by the
-    // [W|U] product, so an item starts without waiting for it
-    auto load_v = [&](const Item &it) {
-#pragma unroll
-        for (int m = 0; m < C * (D / 8) / 256; ++m) {
-            const int i = tid + m * 256, r = i / (D / 8), c8 = (i % (D / 8)) * 8;
-            const bool ok = r < it.len;
-            cp_async16(sm.xv + umma_k128(C, r, c8), ok ? v + it.base + r * rowstride + c8 : v,
-                       ok ? 16 : 0);
-        }
+    auto wait_ld = [&](int grp) {
+        const bool done = mbar_wait_bounded(&sm.ld_bar[grp], (pend_par >> grp) & 1u);
+        if (done) pend &= ~(1u << grp);
+        return done;
     };
 
     if constexpr (KDA_DEBUG) {   // every item this CTA will take: a chunk of 1..C tokens
@@ -288,6 +300,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     if (tid == 0) {
         mbar_init(&sm.mma_bar, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&sm.ld_bar[i], 1);
         fence_mbar_init();
     }
     // the query-key block is read whole by the tensor core: its upper blocks stay zero
@@ -298,27 +311,35 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             make_uint4(0u, 0u, 0u, 0u);
     }
     uint32_t mma_phase = 0;   // completions of mma_bar so far
+    uint32_t ld_phase = 0;    // items whose loads have been consumed
     bool ok = true;
+    __syncthreads();          // barrier initialisation is visible to every thread
 
     Item cur = locate(blockIdx.x);
-    load_g_half(cur, 0);
-    load_g_half(cur, 1);
-    load_kq(cur);
-    cp_async_commit();
-    load_v(cur);
-    cp_async_commit();
+    for (int grp = 0; grp < 4; ++grp) issue(grp, cur, 0);
 
     for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
     const int nxt_item = item + gridDim.x;
     const bool has_next = nxt_item < items;
-    const Item nxt = locate(has_next ? nxt_item : item);
     uint8_t *rec = cur.rec;
-    cp_async_wait<1>();   // g, k, q, beta (V, the newest group, may still be in flight)
-    __syncthreads();
+    // g, k, q (tensor loads) and beta (cp.async); V may still be in flight.  One warp
+    // polls the load barriers and the CTA barrier passes the loads' completion (and
+    // their data) on to the rest, instead of 256 threads polling the same words.
+    if (warp == 0) {
+        ok = wait_ld(0) && ok;
+        ok = wait_ld(1) && ok;
+        ok = wait_ld(2) && ok;
+    } else {
+        pend &= ~7u;
+    }
+    cp_async_wait<0>();
+    ok = __syncthreads_and(ok) != 0;
+    if (!ok) break;
 
     // ---- P1: cumulative decay and the scaled operands ----
     // thread -> channel pair (c0, c0+1) x sub-tile a1 (rows 16a1..16a1+15).  gam holds
-    // the cumsum local to the sub-tile, in log2 units (g rows past len arrive as zero).
+    // the cumsum local to the sub-tile, in log2 units; g rows past the chunk's length
+    // (zeros past the tensor, or the next packed sequence's tokens) count as zero.
     const int c0 = 2 * (tid & 63), a1 = tid >> 6;
     float2 gam[ST];
     {
@@ -327,8 +348,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
         for (int j = 0; j < ST; ++j) {
             const float2 gv = *reinterpret_cast<const float2 *>(gsrc + j * (D * 4));
-            run.x += gv.x * kLog2e;
-            run.y += gv.y * kLog2e;
+            const bool in = a1 * ST + j < cur.len;
+            run.x += in ? gv.x * kLog2e : 0.f;
+            run.y += in ? gv.y * kLog2e : 0.f;
             gam[j] = run;
         }
         *reinterpret_cast<float2 *>(&sm.u.p1.tot[a1][c0]) = run;
@@ -338,11 +360,11 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     // pair factors exp(G_ref(a) - G_ref(b)) <= 1 for the off-diagonal sub-tile blocks
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
-        const int e = tid + 256 * m, p = e >> 7, c = e & (D - 1);
-        const int pa = kPairs[p].x, pb = kPairs[p].y;
+        const int e = tid + 256 * m, pp = e >> 7, c = e & (D - 1);
+        const int pa = kPairs[pp].x, pb = kPairs[pp].y;
         float d = sm.u.p1.ref[pa][c] - sm.u.p1.ref[pb][c];
         for (int a = pb; a < pa; ++a) d += sm.u.p1.tot[a][c];
-        sm.mfac[p][c] = fast_exp2(d);
+        sm.mfac[pp][c] = fast_exp2(d);
     }
     {
         float2 Ba = make_float2(0.f, 0.f), GC = make_float2(0.f, 0.f);
@@ -364,7 +386,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
         for (int j = 0; j < ST; ++j) {
             const int r = a1 * ST + j;
-            const int off = swz128(r, c0);
+            const int off = umma_k128(C, r, c0);
             // every factor below lies in [e^-80, e^40] for g in (-5, 0]
             const float2 E1 = make_float2(fast_exp2(gam[j].x), fast_exp2(gam[j].y));
             const float2 E2 = make_float2(fast_exp2(Gend.x - gam[j].x), fast_exp2(Gend.y - gam[j].y));
@@ -373,17 +395,17 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             const float2 kf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.qa + off));
             const float2 qf = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm.kb + off));
             *reinterpret_cast<uint32_t *>(sm.ka + off) =
-                pack_bf16x2(kf.x * E1.x * f1.x, kf.y * E1.y * f1.y);
+                pack_bf16x2(kf.x * E1.x * f1.x, kf.y * E1.y * f1.y);          // k e^(G_r - G_ref)
             *reinterpret_cast<uint32_t *>(sm.qa + off) =
-                pack_bf16x2(qf.x * E1.x * f1.x, qf.y * E1.y * f1.y);
+                pack_bf16x2(qf.x * E1.x * f1.x, qf.y * E1.y * f1.y);          // q e^(G_r - G_ref)
             *reinterpret_cast<uint32_t *>(sm.kb + off) =
-                pack_bf16x2(kf.x * E2.x * f2.x, kf.y * E2.y * f2.y);
-            *reinterpret_cast<uint32_t *>(sm.xk + umma_k128(C, r, c0)) =
-                pack_bf16x2(kf.x * E1.x * eB.x, kf.y * E1.y * eB.y);
+                pack_bf16x2(kf.x * E2.x * f2.x, kf.y * E2.y * f2.y);          // k e^(G_ref - G_r)
+            *reinterpret_cast<uint32_t *>(sm.xk + off) =
+                pack_bf16x2(kf.x * E1.x * eB.x, kf.y * E1.y * eB.y);          // k e^G_r
             *reinterpret_cast<uint32_t *>(rec + REC_QG_SCRATCH + off) =
-                pack_bf16x2(qf.x * E1.x * eB.x, qf.y * E1.y * eB.y);
-            *reinterpret_cast<uint32_t *>(rec + REC_KT_SCRATCH + umma_k128(C, r, c0)) =
-                pack_bf16x2(kf.x * E2.x * fC.x, kf.y * E2.y * fC.y);
+                pack_bf16x2(qf.x * E1.x * eB.x, qf.y * E1.y * eB.y);          // q e^G_r
+            *reinterpret_cast<uint32_t *>(rec + REC_KT_SCRATCH + off) =
+                pack_bf16x2(kf.x * E2.x * fC.x, kf.y * E2.y * fC.y);          // k e^(G_C - G_r)
         }
         if (a1 == NST - 1)
             *reinterpret_cast<float2 *>(rec + REC_GC + c0 * 4) =
@@ -401,9 +423,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             uint32_t lk[4], lq[4], bfr[4];
-            ldsm_x4(lk, s_ka + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-            ldsm_x4(lq, s_qa + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-            ldsm_x4(bfr, s_kb + swz128(b * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
+            ldsm_x4(lk, s_ka + umma_k128(C, a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+            ldsm_x4(lq, s_qa + umma_k128(C, a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+            ldsm_x4(bfr, s_kb + umma_k128(C, b * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
             // right rows of sub-tile b move their reference from G_ref(b) to G_ref(a)
             const int cc = ks * 16 + 2 * tig;
             const float2 m01 = *reinterpret_cast<const float2 *>(&sm.mfac[warp][cc]);
@@ -440,9 +462,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
                 uint32_t lk[4], lq[4], bfr[4];
-                ldsm_x4(lk, s_ka + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-                ldsm_x4(lq, s_qa + swz128(a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
-                ldsm_x4(bfr, s_kb + swz128(a * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
+                ldsm_x4(lk, s_ka + umma_k128(C, a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+                ldsm_x4(lq, s_qa + umma_k128(C, a * ST + frag_a_row(lane), ks * 16 + frag_a_col(lane)));
+                ldsm_x4(bfr, s_kb + umma_k128(C, a * ST + frag_bn_row(lane), ks * 16 + frag_bn_col(lane)));
                 mma_bf16_16816(ak[0], lk, bfr[0], bfr[1]);
                 mma_bf16_16816(ak[1], lk, bfr[2], bfr[3]);
                 mma_bf16_16816(aq[d][0], lq, bfr[0], bfr[1]);
@@ -545,18 +567,21 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
     }
 
+    const Item nxt = locate(has_next ? nxt_item : item);   // its loads start in P4
+
     // ---- P4: three tcgen05 products, accumulators in tensor memory (256 columns) ----
     //   Y  = T' [K*exp G | V]  (M = 64, N = 256, K = 64):  [W|U], to shared memory as bf16
     //   D1 = Kt^T [W|U]        (M = 128 key rows):         M' = -D1[:, :128], R = D1[:, 128:]
     //   D2 = Aqk  [W|U]        (M = 64 chunk rows):        Q' = Qg - D2[:, :128], O0 = D2[:, 128:]
     {
-        cp_async_wait<0>();         // V
-        fence_proxy_async_smem();   // T' (generic stores), V -> tensor core
+        if (warp == 0) ok = wait_ld(3) && ok;   // V (read by the tensor core only)
+        else pend &= ~8u;
+        fence_proxy_async_smem();   // T' (generic stores) -> tensor core
         t5::fence_before_sync();
-        __syncthreads();
+        ok = __syncthreads_and(ok) != 0;
         const uint32_t tmem = *tmem_slot;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        if (warp == 0) {
+        if (ok && warp == 0) {
             if (t5::elect_one()) {
                 t5::fence_after_sync();
                 const uint64_t tdesc = t5::smem_desc(s_ka, 16, 1024, t5::kSwz128);                  // T', K-major
@@ -570,7 +595,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
             __syncwarp();
         }
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, mma_phase++ & 1));
+        ok = __all_sync(0xffffffffu, ok && mbar_wait_bounded(&sm.mma_bar, mma_phase++ & 1));
         t5::fence_after_sync();
         // X is consumed: bring Kt (into xk) and Qg (into xv) back from the record's scratch
         // area while [W|U] leaves tensor memory; T' is consumed too: the next item's g
@@ -583,8 +608,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                        rec + (m == 0 ? REC_KT_SCRATCH : REC_QG_SCRATCH) + off);
         }
         cp_async_commit();
-        if (has_next) load_g_half(nxt, 0);
-        cp_async_commit();
+        if (has_next) issue(0, nxt, ld_phase + 1);
         if (ok) {   // M = 64 accumulator: rows 16(w&3)..+15; warps 0-3 -> W, warps 4-7 -> U
             const int r0 = (warp & 3) * 16 + gid, cb = (warp >> 2) * D;
 #pragma unroll
@@ -601,7 +625,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 }
             }
         }
-        cp_async_wait<1>();         // Kt and Qg (the next item's g may still be in flight)
+        cp_async_wait<0>();         // Kt and Qg
         fence_proxy_async_smem();   // [W|U] (generic stores), Kt (cp.async) -> tensor core
         t5::fence_before_sync();
         ok = __syncthreads_and(ok) != 0;
@@ -621,8 +645,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, mma_phase++ & 1));
         t5::fence_after_sync();
-        if (has_next) load_g_half(nxt, 1);   // Kt is consumed: g rows 32-63 to xk
-        cp_async_commit();
+        if (has_next) issue(1, nxt, ld_phase + 1);   // Kt is consumed: g rows 32-63 to xk
         if (ok) {   // lane = key row; warps 0-3 -> M' (columns 0..127), warps 4-7 -> R
             const int m = (warp & 3) * 32 + lane, cb = (warp >> 2) * D;
 #pragma unroll
@@ -660,8 +683,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, mma_phase++ & 1));
         t5::fence_after_sync();
-        if (has_next) load_kq(nxt);   // [W|U] is consumed: the next k and q to qa and kb
-        cp_async_commit();
+        if (has_next) issue(2, nxt, ld_phase + 1);   // [W|U] is consumed: next k, q, beta
         if (ok) {   // M = 64 accumulator: rows 16(w&3)..+15; warps 0-3 -> Q', warps 4-7 -> O0
             const int r0 = (warp & 3) * 16 + gid, cb = (warp >> 2) * D;
             uint8_t *dst0 = rec + (warp < 4 ? REC_QP : REC_O0);
@@ -678,7 +700,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                         float x0 = vv[4 * j8 + 2 * hh], x1 = vv[4 * j8 + 2 * hh + 1];
                         if (warp < 4) {   // Q' = Qg - Aqk W
                             const float2 f = unpack_bf16x2(
-                                *reinterpret_cast<const uint32_t *>(sm.xv + swz128(r, c)));
+                                *reinterpret_cast<const uint32_t *>(sm.xv + umma_k128(C, r, c)));
                             x0 = f.x - x0;
                             x1 = f.y - x1;
                         }
@@ -690,14 +712,18 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         t5::fence_before_sync();
         ok = __syncthreads_and(ok) != 0;   // Qg in xv is consumed
         t5::fence_after_sync();
-        if (has_next) load_v(nxt);
-        cp_async_commit();
+        if (has_next) issue(3, nxt, ld_phase + 1);
     }
     cur = nxt;
+    ++ld_phase;
     }   // item loop
 
     if (!ok && tid == 0) atomicOr(err_word, ERR_TIMEOUT_BIT);
-    cp_async_wait<0>();   // nothing may land in shared memory after the CTA ends
+    // nothing may land in shared memory after the CTA ends: loads still in flight (after
+    // a wait that gave up) are waited for, again with the time limit
+    for (int grp = 0; grp < 4; ++grp)
+        if (pend & (1u << grp)) wait_ld(grp);
+    cp_async_wait<0>();
     t5::fence_before_sync();
     __syncthreads();
     t5::fence_after_sync();
@@ -1232,6 +1258,66 @@ __global__ void __launch_bounds__(256) kda_tc_seg_combine_kernel(
         }
         __syncthreads();
     }
+}
+
+// ---------------------------------------------------------------------------
+// Context parallelism across devices: the starting state of rank `rank`'s time
+// segment.  maps holds every rank's segment map [R | P] ([world][chains][D][2D], the
+// map pass's layout), gathered from all ranks; S_in(rank) = fold over ranks
+// 0 .. rank-1 of S <- P_s S + R_s, from h0 (or zero).  grid = (chains, D / 32), 256
+// threads: thread t owns row t / 2, columns 16 (t & 1) .. +15 of the 32-column slice.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) kda_cp_combine_kernel(
+    const float *__restrict__ h0, const float *__restrict__ maps, float *__restrict__ s_in,
+    int rank, int chains) {
+    __shared__ __align__(16) float Ssm[D][32];
+    const int chain = blockIdx.x, c0 = blockIdx.y * 32;
+    const int r = threadIdx.x >> 1, cl = (threadIdx.x & 1) * 16;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (h0) v = *reinterpret_cast<const float4 *>(h0 + ((size_t)chain * D + r) * D + c0 + cl + i);
+        x[i] = v.x;
+        x[i + 1] = v.y;
+        x[i + 2] = v.z;
+        x[i + 3] = v.w;
+    }
+    for (int s = 0; s < rank; ++s) {
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4 *>(&Ssm[r][cl + i]) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+        __syncthreads();
+        const float *row = maps + (((size_t)s * chains + chain) * D + r) * (2 * D);   // [R | P]
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(row + c0 + cl + i);
+            x[i] = v.x;
+            x[i + 1] = v.y;
+            x[i + 2] = v.z;
+            x[i + 3] = v.w;
+        }
+        for (int k4 = 0; k4 < D; k4 += 4) {
+            const float4 p = *reinterpret_cast<const float4 *>(row + D + k4);
+            const float pk[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                for (int i = 0; i < 16; i += 4) {
+                    const float4 sv = *reinterpret_cast<const float4 *>(&Ssm[k4 + u][cl + i]);
+                    x[i] = fmaf(pk[u], sv.x, x[i]);
+                    x[i + 1] = fmaf(pk[u], sv.y, x[i + 1]);
+                    x[i + 2] = fmaf(pk[u], sv.z, x[i + 2]);
+                    x[i + 3] = fmaf(pk[u], sv.w, x[i + 3]);
+                }
+            }
+        }
+        __syncthreads();
+    }
+    float *dst = s_in + ((size_t)chain * D + r) * D + c0 + cl;
+#pragma unroll
+    for (int i = 0; i < 16; i += 4)
+        *reinterpret_cast<float4 *>(dst + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
 }
 
 }  // namespace tc
