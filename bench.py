@@ -40,7 +40,7 @@ L2_BYTES = 126 << 20
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 HEADLINE = "long"
-WORKLOAD_KEYS = ("prefill", "long", "varlen", "few_chains", "decode")
+WORKLOAD_KEYS = ("prefill", "long", "varlen", "few_chains", "decode", "profile")
 
 
 def load_peaks():
@@ -142,7 +142,7 @@ def max_over_ranks(x, world, device):
 def workload_of(name):
     from kimi_delta_attention_28_b200 import workloads as W
     return {"prefill": W.PREFILL, "long": W.LONG, "varlen": W.VARLEN,
-            "few_chains": W.FEW_CHAINS, "decode": W.DECODE}[name]
+            "few_chains": W.FEW_CHAINS, "decode": W.DECODE, "profile": W.PROFILE}[name]
 
 
 def workload_inputs(name, device, seed_offset=0):
@@ -990,7 +990,8 @@ def _free_device_memory():
 
 def default_steps(workload):
     """Timed steps when --steps is not given (about a second of timed work or less)."""
-    return {"long": 10, "few_chains": 100, "varlen": 100, "prefill": 1000, "decode": 300}[workload]
+    return {"long": 10, "few_chains": 100, "varlen": 100, "prefill": 1000, "decode": 300,
+            "profile": 100}[workload]
 
 
 def main():

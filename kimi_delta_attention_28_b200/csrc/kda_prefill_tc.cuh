@@ -37,6 +37,10 @@ constexpr int D = 128;          // head size (d_k = d_v)
 constexpr int C = 64;           // chunk length
 constexpr int ST = 16;          // sub-tile length for the decay reference rows
 constexpr int NST = C / ST;     // sub-tiles per chunk
+// Largest total decay of a chunk (log2 units, per channel) for which the prep uses
+// one reference row and whole-chunk tensor-core products: factors up to 2^120 stay
+// inside the bf16 / fp32 range (2^127) with room for |k| <= 1.
+constexpr float kDenseSpan = 120.f;
 
 // Per (chunk, head) record, written by kernel 1 and read by kernel 2: the
 // chunk's affine map.  With W, U, Kt = K*exp(G_C - G), Qg = Q*exp(G) and the
@@ -342,6 +346,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // (zeros past the tensor, or the next packed sequence's tokens) count as zero.
     const int c0 = 2 * (tid & 63), a1 = tid >> 6;
     float2 gam[ST];
+    bool dense;
     {
         float2 run = make_float2(0.f, 0.f);
         const uint8_t *gsrc = (a1 < 2 ? sm.ka : sm.xk) + (a1 & 1) * ST * (D * 4) + c0 * 4;
@@ -355,8 +360,15 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         *reinterpret_cast<float2 *>(&sm.u.p1.tot[a1][c0]) = run;
         *reinterpret_cast<float2 *>(&sm.u.p1.ref[a1][c0]) = gam[ST / 2 - 1];
+        // Dense path: when every channel decays by at most 2^-(kDenseSpan / 4) over each
+        // 16-token sub-tile (so by 2^-kDenseSpan over the chunk), one reference row (31,
+        // the middle) keeps k e^(G_r - G_31) and k e^(G_31 - G_i) inside the bf16 range
+        // for every r, i, and the key-key and query-key blocks are two whole 64 x 64
+        // products on the tensor core.  Otherwise (decays near the -5 bound) the
+        // 16-token sub-tile references are used.
+        dense = __syncthreads_and(run.x >= -0.25f * kDenseSpan && run.y >= -0.25f * kDenseSpan) != 0;
     }
-    __syncthreads();   // every g value is in registers; ka and xk may be overwritten
+    // (the barrier above: every g value is in registers; ka and xk may be overwritten)
     // pair factors exp(G_ref(a) - G_ref(b)) <= 1 for the off-diagonal sub-tile blocks
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
@@ -379,15 +391,25 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             GC.y += x.y;
         }
         const float2 Gref = gam[ST / 2 - 1], Gend = gam[ST - 1];   // local to the sub-tile
-        const float2 f1 = make_float2(fast_exp2(-Gref.x), fast_exp2(-Gref.y));                   // >= 1
-        const float2 f2 = make_float2(fast_exp2(Gref.x - Gend.x), fast_exp2(Gref.y - Gend.y));   // >= 1
+        float2 f1, f2;
+        if (dense) {   // M = G_31 = the first two sub-tiles' totals
+            const float2 t0 = *reinterpret_cast<const float2 *>(&sm.u.p1.tot[0][c0]);
+            const float2 t1 = *reinterpret_cast<const float2 *>(&sm.u.p1.tot[1][c0]);
+            const float2 M = make_float2(t0.x + t1.x, t0.y + t1.y);
+            f1 = make_float2(fast_exp2(Ba.x - M.x), fast_exp2(Ba.y - M.y));                      // 2^(Ba - G_31)
+            f2 = make_float2(fast_exp2(M.x - Ba.x - Gend.x), fast_exp2(M.y - Ba.y - Gend.y));   // 2^(G_31 - Ba - Gend)
+        } else {
+            f1 = make_float2(fast_exp2(-Gref.x), fast_exp2(-Gref.y));                   // >= 1
+            f2 = make_float2(fast_exp2(Gref.x - Gend.x), fast_exp2(Gref.y - Gend.y));   // >= 1
+        }
         const float2 eB = make_float2(fast_exp2(Ba.x), fast_exp2(Ba.y));                         // <= 1
         const float2 fC = make_float2(fast_exp2(GC.x - Ba.x - Gend.x), fast_exp2(GC.y - Ba.y - Gend.y));
 #pragma unroll
         for (int j = 0; j < ST; ++j) {
             const int r = a1 * ST + j;
             const int off = umma_k128(C, r, c0);
-            // every factor below lies in [e^-80, e^40] for g in (-5, 0]
+            // every factor below lies in [2^-126, 2^126]: sub-tile path, [e^-80, e^40] for
+            // g in (-5, 0]; dense path, within 2^kDenseSpan
             const float2 E1 = make_float2(fast_exp2(gam[j].x), fast_exp2(gam[j].y));
             const float2 E2 = make_float2(fast_exp2(Gend.x - gam[j].x), fast_exp2(Gend.y - gam[j].y));
             // raw k sits in qa and raw q in kb at the same offset; this thread reads
@@ -400,6 +422,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 pack_bf16x2(qf.x * E1.x * f1.x, qf.y * E1.y * f1.y);          // q e^(G_r - G_ref)
             *reinterpret_cast<uint32_t *>(sm.kb + off) =
                 pack_bf16x2(kf.x * E2.x * f2.x, kf.y * E2.y * f2.y);          // k e^(G_ref - G_r)
+            // (G_ref: the sub-tile's reference row, or row 31 on the dense path)
             *reinterpret_cast<uint32_t *>(sm.xk + off) =
                 pack_bf16x2(kf.x * E1.x * eB.x, kf.y * E1.y * eB.y);          // k e^G_r
             *reinterpret_cast<uint32_t *>(rec + REC_QG_SCRATCH + off) =
@@ -411,12 +434,92 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             *reinterpret_cast<float2 *>(rec + REC_GC + c0 * 4) =
                 make_float2(fast_exp2(GC.x), fast_exp2(GC.y));
     }
+    fence_proxy_async_smem();   // the dense path's products read ka, qa, kb
+    t5::fence_before_sync();
     __syncthreads();
 
     // ---- P2: key-key and query-key blocks ----
-    // warps 0-5: one off-diagonal sub-tile pair each (both products share the
-    // rescaled right operand); warps 6-7: two diagonal blocks each, whose
-    // key-key blocks they also invert.
+    // (I + A_aa)^-1 of diagonal sub-tile blocks: lane -> (block a0 + lane/16, column j)
+    // (lanes 16-31 only when two blocks are given): solve (I + A_aa) x = e_j in fp32,
+    // column by column (x_i is final when row i is reached; depth 16, not 120)
+    auto invert_diagonal = [&](int a0) {
+        const int a = a0 + (lane >> 4), j = lane & 15;
+        float x[ST];
+#pragma unroll
+        for (int r = 0; r < ST; ++r) x[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < ST - 1; ++i)
+#pragma unroll
+            for (int r = i + 1; r < ST; ++r) x[r] = fmaf(-sm.u.akd[a][r][i], x[i], x[r]);
+#pragma unroll
+        for (int r = 0; r < ST; ++r) sm.taa[a][r * (ST + 8) + j] = f2bf(x[r]);
+    };
+    if (dense) {
+        // Two tcgen05 products with the row-31 reference: A_kk = Kl Kr^T and
+        // A_qk = Ql Kr^T (M = 64, N = 64, K = 128; ka, qa, kb all K-major), into tensor
+        // memory columns 0-63 and 64-127; then every thread takes its rows of one block
+        // (warps 0-3: A_kk, 4-7: A_qk) to the masked, beta-scaled forms the
+        // substitution and the record products use.
+        const uint32_t tmem = *tmem_slot;
+        if (warp == 0) {
+            if (t5::elect_one()) {
+                t5::fence_after_sync();
+                const uint64_t kd = t5::smem_desc(s_ka, 16, 1024, t5::kSwz128);
+                const uint64_t qd = t5::smem_desc(s_qa, 16, 1024, t5::kSwz128);
+                const uint64_t bd = t5::smem_desc(s_kb, 16, 1024, t5::kSwz128);
+                constexpr uint32_t id = t5::idesc_bf16(64, 64, 0, 0);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t o = (uint64_t)(((ks >> 2) * C * 128 + (ks & 3) * 32) >> 4);
+                    t5::mma_bf16(tmem, kd + o, bd + o, id, ks > 0);
+                    t5::mma_bf16(tmem + 64, qd + o, bd + o, id, ks > 0);
+                }
+                t5::commit(&sm.mma_bar);
+            }
+            __syncwarp();
+        }
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sm.mma_bar, mma_phase++ & 1));
+        t5::fence_after_sync();
+        if (ok) {   // M = 64 accumulators: rows 16(w&3) + gid (+8) = sub-tile w&3
+            const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+            const bool kk = warp < 4;
+            const int rb = (warp & 3) * 16 + gid;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float vv[16];
+                t5::ld16x256b_x4(tmem + lane_base + (kk ? 0 : 64) + half * 32, vv);
+#pragma unroll
+                for (int j8 = 0; j8 < 4; ++j8)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int r = rb + 8 * hh, i = half * 32 + j8 * 8 + 2 * tig;
+                        const float x0 = vv[4 * j8 + 2 * hh], x1 = vv[4 * j8 + 2 * hh + 1];
+                        const int ar = r / ST, bi = i / ST;
+                        if (bi > ar) continue;                       // upper blocks: unused / zero
+                        if (kk) {
+                            const float br = sm.beta[r];
+                            if (bi < ar) {
+                                *reinterpret_cast<uint32_t *>(sm.akkn + r * LDA + i) =
+                                    pack_bf16x2(-x0 * br, -x1 * br);
+                            } else {
+                                sm.u.akd[ar][r % ST][i % ST] = (i < r) ? x0 * br : 0.f;
+                                sm.u.akd[ar][r % ST][i % ST + 1] = (i + 1 < r) ? x1 * br : 0.f;
+                            }
+                        } else {
+                            *reinterpret_cast<uint32_t *>(sm.aqk + umma_k128(C, r, i)) =
+                                pack_bf16x2(i <= r ? x0 : 0.f, i + 1 <= r ? x1 : 0.f);
+                        }
+                    }
+            }
+        }
+        // warps 0-3 hold their own sub-tile's diagonal block: invert it at once, while
+        // warps 4-7 still write the query-key rows
+        if (warp < 4) {
+            __syncwarp();
+            if (lane < ST) invert_diagonal(warp);
+        }
+        t5::fence_before_sync();
+    } else {
     if (warp < 6) {
         const int a = kPairs[warp].x, b = kPairs[warp].y;
         float ak[2][4] = {}, aq[2][4] = {};
@@ -481,19 +584,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
         }
         __syncwarp();
-        {   // lane -> (block a0 + lane/16, column j): solve (I + A_aa) x = e_j in fp32,
-            // column by column (x_i is final when row i is reached; depth 16, not 120)
-            const int a = a0 + (lane >> 4), j = lane & 15;
-            float x[ST];
-#pragma unroll
-            for (int r = 0; r < ST; ++r) x[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-            for (int i = 0; i < ST - 1; ++i)
-#pragma unroll
-                for (int r = i + 1; r < ST; ++r) x[r] = fmaf(-sm.u.akd[a][r][i], x[i], x[r]);
-#pragma unroll
-            for (int r = 0; r < ST; ++r) sm.taa[a][r * (ST + 8) + j] = f2bf(x[r]);
-        }
+        invert_diagonal(a0);
 #pragma unroll
         for (int d = 0; d < 2; ++d)
 #pragma unroll
@@ -506,6 +597,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         pack_bf16x2(il <= rl ? aq[d][nt][2 * hh] : 0.f,
                                     il + 1 <= rl ? aq[d][nt][2 * hh + 1] : 0.f);
                 }
+    }
     }
     __syncthreads();
 

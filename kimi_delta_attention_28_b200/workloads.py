@@ -63,7 +63,14 @@ FEW_CHAINS = Workload("few_chains_bf16_B1_H2_T262144_d128", B=1, H=2, T=1 << 18,
                       note="two (sequence, head) chains of 4,096 chunks: too few to fill "
                            "the GPU, so the state pass is split in time")
 
-ALL = (TINY, PREFILL, LONG, VARLEN, DECODE, FEW_CHAINS)
+PROFILE = Workload("profile_bf16_B1_H16_T16384_d128", B=1, H=16, T=1 << 14, dk=128, dv=128,
+                   dtype=torch.bfloat16, h0=False, seed=1006,
+                   note="the 1M-token workload's shape at 1/64 of its length: inputs and "
+                        "records (about 0.7 GB) far larger than L2 but small enough for "
+                        "profiler captures; DRAM bytes per token-head measured here scale "
+                        "to the full workload")
+
+ALL = (TINY, PREFILL, LONG, VARLEN, DECODE, FEW_CHAINS, PROFILE)
 BY_NAME = {w.name: w for w in ALL}
 
 
