@@ -40,7 +40,8 @@ L2_BYTES = 126 << 20
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 HEADLINE = "long"
-WORKLOAD_KEYS = ("prefill", "long", "varlen", "few_chains", "decode", "profile")
+WORKLOAD_KEYS = ("prefill", "long", "varlen", "few_chains", "decode", "profile", "speculative",
+                 "backward")
 
 
 def load_peaks():
@@ -991,7 +992,7 @@ def _free_device_memory():
 def default_steps(workload):
     """Timed steps when --steps is not given (about a second of timed work or less)."""
     return {"long": 10, "few_chains": 100, "varlen": 100, "prefill": 1000, "decode": 300,
-            "profile": 100}[workload]
+            "profile": 100, "speculative": 200, "backward": 5}[workload]
 
 
 def main():
@@ -1019,7 +1020,7 @@ def main():
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
-    if args.impl == "reference" and args.workload == "decode":
+    if args.impl == "reference" and args.workload in ("decode", "speculative", "backward"):
         ap.error("the reference arm covers the prefill workloads")
     if args.impl == "reference":
         if rank != 0:
@@ -1031,6 +1032,10 @@ def main():
     try:
         if args.workload == "decode":
             out = measure_decode(args.steps, args.warmup, world, rank, local, cpu=cpu)
+        elif args.workload == "speculative":
+            out = measure_speculative(args.steps, args.warmup, cpu=cpu) if rank == 0 else None
+        elif args.workload == "backward":
+            out = measure_backward("prefill", args.steps, args.warmup, cpu=cpu) if rank == 0 else None
         else:
             out = measure_prefill(args.workload, args.steps, args.warmup, world, rank, local,
                                   e2e=not args.no_e2e, cpu=cpu, cpu_seconds=args.cpu_seconds,
@@ -1056,7 +1061,7 @@ def main():
             r = measure_speculative(200, 20, cpu=cpu)
             nested["speculative"] = r
             _free_device_memory()
-            nested["backward"] = measure_backward("prefill", 5, 2, cpu=cpu)
+            nested["backward"] = measure_backward("prefill", 5, 3, cpu=cpu)
             out["workloads"] = nested
         if out is not None:
             print(json.dumps(out), flush=True)
