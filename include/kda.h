@@ -120,9 +120,11 @@ size_t kda_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
  * The cu_seqlens preconditions are checked on the device; a violation makes
  * the call write no outputs and is reported by kda_get_last_device_error.
  * T = 0 (or B = 0) is a valid empty call that only copies h0 to hT.
- * On the tensor-core path the call picks the number of time segments of the
- * state pass itself (kda_fwd_segmented with a policy based on the SM count:
- * split only when N * H chains are too few to fill the GPU).
+ * On the tensor-core path the call picks its schedule itself from the SM count:
+ * the number of time segments of the state pass (kda_fwd_segmented: split only
+ * when N * H chains are too few to fill the GPU), and, for fixed-length input
+ * without a split, whether both phases run as one overlapped launch
+ * (kda_fwd_overlapped) or as two (kda_fwd_segmented with one segment).
  */
 kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                    const float *beta, const float *h0, const int32_t *cu_seqlens,
@@ -133,7 +135,9 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
  * The two phases of kda_fwd on the tensor-core path (bf16, d_k = d_v = 128),
  * exposed so callers can schedule or time them separately.  Calling
  * kda_fwd_intra and then kda_fwd_inter on the same stream and workspace is
- * exactly kda_fwd.  Other dtype / head-size combinations return
+ * exactly kda_fwd_segmented with one segment (and kda_fwd, where kda_fwd neither
+ * splits nor overlaps: kda_fwd_plan_segments and kda_fwd_plan_overlap say which).
+ * Other dtype / head-size combinations return
  * KDA_ERR_UNSUPPORTED_SHAPE (kda_fwd handles them in a single kernel).
  *
  * kda_fwd_intra: everything inside a chunk, in parallel over (chunk, head):
@@ -168,8 +172,9 @@ kda_status kda_fwd_inter(const float *h0, const int32_t *cu_seqlens, int num_seq
  * Pass 1 computes every segment's map [R | P] from zero / identity, a combine
  * kernel walks the segments in order in fp32 (S_{s+1} = P_s S_s + R_s) to get
  * each segment's starting state, and pass 2 reruns the segments from those
- * states, writing o and (from the last segment) hT.  num_segments = 1 is
- * exactly kda_fwd without a split.  num_segments > 1 needs the tensor-core path
+ * states, writing o and (from the last segment) hT.  num_segments = 1 is the
+ * unsplit pass as two launches (kda_fwd_intra, then kda_fwd_inter), which is what
+ * kda_fwd runs when it neither splits nor overlaps.  num_segments > 1 needs the tensor-core path
  * (bf16, d_k = d_v = 128), else KDA_ERR_UNSUPPORTED_SHAPE; at most 4,096.
  * The workspace must hold kda_fwd_segmented_workspace_size(..., num_segments)
  * bytes: the records plus N * H * num_segments * 192 KiB.
@@ -185,6 +190,37 @@ kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const 
                              int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
                              int num_segments, void *o, float *hT, void *workspace,
                              size_t ws_bytes, void *stream);
+
+/*
+ * Prefill with both phases in ONE launch, overlapped in time (fixed-length input,
+ * tensor-core path: bf16, d_k = d_v = 128).  The state pass of a chain is
+ * sequential over its chunks, while the chunk records are independent; with few
+ * chains the state pass occupies few SMs for a long time.  Here one block per SM
+ * is launched: 2 * B * H of them run the state pass (64-column slices of each
+ * (sequence, head) state) and every other block runs two workers of the record
+ * kernel, which write the records in time order (chunk j of every chain before
+ * chunk j + 1) and publish each through a flag in the workspace; a state block
+ * waits (bounded, 1 s) for a record's flag before copying it in.  The record
+ * kernel never waits for the state pass, so the blocks cannot deadlock, and the
+ * launch is cooperative so that every block is resident.  Results equal those of
+ * kda_fwd_segmented with one segment up to the state pass's bf16 rounding (the two
+ * schedules slice the state differently), and are checked against the oracle at
+ * the same tolerance.
+ *
+ * Needs 2 * B * H below the device's SM count (else KDA_ERR_UNSUPPORTED_SHAPE);
+ * packed input is not supported (no cu_seqlens argument).  Workspace: at least
+ * kda_fwd_segmented_workspace_size(B, T, H, 128, 128, 0, dtype, 1) bytes (which
+ * kda_fwd_workspace_size covers).  A record that is never published makes the
+ * state blocks give up after the bounded wait: the call's device error becomes
+ * KDA_ERR_DEVICE_TIMEOUT.  Other arguments and results as for kda_fwd.
+ */
+kda_status kda_fwd_overlapped(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *h0, int B, int T, int H, int dk,
+                              int dv, int dtype, void *o, float *hT, void *workspace,
+                              size_t ws_bytes, void *stream);
+/* 1 if kda_fwd runs the overlapped single launch for these sizes on the current
+ * device, else 0 (also for invalid sizes, packed input or no device). */
+int kda_fwd_plan_overlap(int B, int T, int H, int dk, int dv, int num_seqs, int dtype);
 
 /*
  * kda_fwd that also stores the state at fixed token intervals, for prefix caching
@@ -277,8 +313,8 @@ kda_status kda_cp_finish(const float *maps, int rank, int world, const float *h0
  * packed-sequence rules and alignment as kda_fwd; grad_o [B, T, H, d_v] has the
  * dtype of q; grad_hT, grad_h0 [N, H, d_k, d_v].  No gradient buffer may alias an
  * input.  The workspace must hold kda_bwd_workspace_size(...) bytes: the state every
- * 8 tokens of every (sequence, head) plus partial sums (about 16 KiB per
- * token-head at d = 128).
+ * 64 tokens of every (sequence, head) (d_k d_v / 16 bytes per token-head, 1 KiB at
+ * d = 128) plus 8 states of scratch per (sequence, head).
  *
  * What it computes is the chain rule through the recurrence (panel "KDA 单头递归"),
  * token by token from the last to the first, with G = dL/dS_t, S' = Diag(exp g_t)
@@ -288,9 +324,9 @@ kda_status kda_cp_finish(const float *maps, int rank, int world, const float *h0
  *     G = Diag(exp g) G';  and dh0 = G after the first token.
  * The source pages name the training kernel ("FlashKDA / FLA" panel) but give no
  * formulas for it; this is the gradient of the recurrence they print, in fp32 on
- * CUDA cores (one CTA per (sequence, head) and 32 value columns, the states of
- * every 8-token chunk recomputed from stored checkpoints).  All head sizes and
- * dtypes of kda_fwd are supported.
+ * CUDA cores (one CTA per (sequence, head) and 32 value columns, the slices of a
+ * chain one thread-block cluster; states recomputed from stored checkpoints).  All
+ * head sizes and dtypes of kda_fwd are supported.
  */
 size_t kda_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype);
 kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,

@@ -9,6 +9,8 @@ panel "KDA 单头递归"), as a C-ABI CUDA library:
                        initial and final states);
 * ``kda_fwd_segmented`` the same prefill with the state pass split in time
                        (per-segment affine maps combined in prefix order);
+* ``kda_fwd_overlapped`` the same prefill (fixed-length) as one launch in which
+                       the state pass consumes each chunk record once published;
 * ``kda_fwd_checkpointed`` prefill that also stores the state every n tokens
                        (prefix caching);
 * ``kda_fwd_context_parallel``  prefill split in time over the ranks of a process
@@ -27,11 +29,13 @@ from ._lib import (KDAError, bwd_workspace_size, checkpoint_count, cp_workspace_
                    kda_fwd_context_parallel,
                    kda_bwd, kda_decode_commit, kda_decode_step, kda_decode_verify,
                    kda_fwd, kda_fwd_checkpointed, kda_fwd_inter, kda_fwd_intra,
-                   kda_fwd_noalloc, kda_fwd_segmented, load_library, plan_segments,
-                   segmented_workspace_size, workspace_size)
+                   kda_fwd_noalloc, kda_fwd_overlapped, kda_fwd_segmented, load_library,
+                   plan_overlap, plan_segments, segmented_workspace_size, workspace_size)
 
 __all__ = ["kda_fwd", "kda_bwd", "bwd_workspace_size", "kda_fwd_context_parallel",
-           "kda_cp_local_map", "kda_cp_finish", "gather_segment_maps", "cp_workspace_size", "kda_fwd_intra", "kda_fwd_inter", "kda_fwd_noalloc", "kda_fwd_segmented",
+           "kda_cp_local_map", "kda_cp_finish", "gather_segment_maps", "cp_workspace_size",
+           "kda_fwd_intra", "kda_fwd_inter", "kda_fwd_noalloc", "kda_fwd_segmented",
+           "kda_fwd_overlapped", "plan_overlap",
            "kda_fwd_checkpointed", "checkpoint_count", "kda_decode_step",
            "kda_decode_verify", "kda_decode_commit", "workspace_size",
            "segmented_workspace_size", "plan_segments", "device_error", "load_library",

@@ -59,6 +59,9 @@ SIGNATURES = {
     "kda_decode_commit": ([_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP], _I),
     "kda_fwd_noalloc": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP,
                          _VP], _I),
+    "kda_fwd_overlapped": ([_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP,
+                            _SZ, _VP], _I),
+    "kda_fwd_plan_overlap": ([_I, _I, _I, _I, _I, _I, _I], _I),
     "kda_fwd_segmented_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I], _SZ),
     "kda_fwd_plan_segments": ([_I, _I, _I, _I, _I, _I, _I], _I),
     "kda_fwd_segmented": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I,
@@ -253,6 +256,42 @@ def kda_fwd_segmented(q, k, v, g, beta, h0=None, cu_seqlens=None, *, num_segment
                                  _dtype_code(q.dtype), num_segments, _ptr(o), _ptr(hT),
                                  _ptr(workspace), workspace.numel(), _stream(dev)),
            "kda_fwd_segmented")
+    return o, hT
+
+
+def plan_overlap(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
+                 dtype: torch.dtype) -> bool:
+    """Whether kda_fwd runs both phases as one overlapped launch for these sizes."""
+    return bool(load_library().kda_fwd_plan_overlap(B, T, H, dk, dv, num_seqs,
+                                                    _dtype_code(dtype)))
+
+
+def kda_fwd_overlapped(q, k, v, g, beta, h0=None, *, o=None, hT=None, workspace=None):
+    """Fixed-length prefill with the record and state phases in one launch (the
+    state blocks consume each chunk record as soon as it is published).  Needs
+    2 * B * H below the SM count.  Arguments as for kda_fwd; returns (o, hT)."""
+    lib = load_library()
+    dev = q.device
+    B, T, H, dk, dv, num_seqs, N = _prefill_shapes(q, k, v, g, beta, h0, None, o, hT,
+                                                   workspace)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, n, q.dtype, dev)
+    _need(g, "g", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(h0, "h0", torch.float32, dev)
+    _need(hT, "hT", torch.float32, dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=q.dtype, device=dev)
+    if hT is None:
+        hT = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    need = segmented_workspace_size(B, T, H, dk, dv, 0, q.dtype, 1)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.kda_fwd_overlapped(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                  B, T, H, dk, dv, _dtype_code(q.dtype), _ptr(o), _ptr(hT),
+                                  _ptr(workspace), workspace.numel(), _stream(dev)),
+           "kda_fwd_overlapped")
     return o, hT
 
 

@@ -44,7 +44,7 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 //   seg_map  : (T-split only) units * D * 2D fp32 segment maps [R | P]
 // where units = chains (N * H) * nseg.
 struct WsLayout {
-    size_t hdr, seq_off, chunks, recs, s_in, seg_map, total;
+    size_t hdr, seq_off, chunks, recs, ready, prog, s_in, seg_map, total;
     long long max_chunks;
     int nseg;
 };
@@ -59,6 +59,7 @@ inline bool is_tc_path(int dtype, int dk) { return dtype == KDA_DTYPE_BF16 && dk
 constexpr int kMaxSegments = 32;
 constexpr int kMinSegChunks = 16;
 constexpr int kSplitSmBound = 192;   // workspace sizing assumes at most this many SMs
+constexpr int kProgressSlots = kSplitSmBound;   // state CTAs of the overlapped schedule
 constexpr int kMaxSegmentsExplicit = 4096;   // cap of kda_fwd_segmented's num_segments
 
 int split_segments(long long chains, long long chunks_per_chain, int sms) {
@@ -103,6 +104,10 @@ WsLayout ws_layout(int B, int T, int H, int dk, int num_seqs, int dtype, int nse
     L.nseg = 1;
     if (is_tc_path(dtype, dk)) {
         L.total += (size_t)L.max_chunks * H * kda::tc::REC_BYTES;
+        // the overlapped schedule's per-record ready flags and per-CTA progress counters
+        L.ready = round_up(L.total, 256);
+        L.prog = L.ready + (size_t)L.max_chunks * H * sizeof(int);
+        L.total = L.prog + kProgressSlots * kda::tc::kProgStride * sizeof(int);
         const long long N = num_seqs > 0 ? num_seqs : B;
         L.nseg = nseg > 0 ? nseg
                           : split_segments(N * H, chunks_per_chain(B, T, num_seqs, L.max_chunks), sms);
@@ -204,31 +209,31 @@ kda_status launch_state(kda::tc::StateArgs a, long long units, cudaStream_t s) {
 
 // ---------------------------------------------------------------------------
 // Backward pass.  Workspace: the forward path's header region (offsets check and
-// chunk table of the packed layout), then the state checkpoints every bwd::CB tokens
-// of every (sequence, head), then the per-slice partial sums of dq, dk, dg, dbeta.
+// chunk table of the packed layout), then the state checkpoints every bwd::CK
+// tokens of every (sequence, head), then each CTA's scratch for the state every
+// bwd::CB tokens of the chunk it is working on.
 // ---------------------------------------------------------------------------
 struct BwdLayout {
-    size_t hdr_end, ckpt, part, total;
+    size_t hdr_end, ckpt, sub, total;
 };
 BwdLayout bwd_layout(int B, int T, int H, int dk, int num_seqs, int dtype) {
     BwdLayout L{};
     const WsLayout F = ws_layout(B, T, H, dk, num_seqs, dtype, 1);
     L.hdr_end = F.recs;   // header, sequence offsets and chunk table only
     const long long ntok = (long long)B * T, N = num_seqs > 0 ? num_seqs : B;
-    const long long slots = ntok / kda::bwd::CB + N + 1;
+    const long long slots = ntok / kda::bwd::CK + N + 1;
     L.ckpt = round_up(L.hdr_end, 256);
-    L.part = round_up(L.ckpt + (size_t)slots * H * dk * dk * sizeof(float), 256);
-    L.total = L.part + (size_t)(dk / kda::bwd::SLC) * ntok * H * (3 * dk + 1) * sizeof(float);
+    L.sub = round_up(L.ckpt + (size_t)slots * H * dk * dk * sizeof(float), 256);
+    L.total = L.sub + (size_t)N * H * kda::bwd::NSUB * dk * dk * sizeof(float);
     return L;
 }
 
 template <int D, typename TIn>
 kda_status launch_bwd(const void *q, const void *k, const void *v, const float *g,
-                             const float *beta, const float *h0, const int32_t *cu,
-                             const int *hdr, const void *dO, const float *dhT, int T, int H,
-                             long long ntok, long long chains, float *ckpt, float *part,
-                             void *dq, void *dkk, void *dvv, float *dg, float *db, float *dh0,
-                             int *err, cudaStream_t s) {
+                      const float *beta, const float *h0, const int32_t *cu, const int *hdr,
+                      const void *dO, const float *dhT, int T, int H, long long ntok,
+                      long long chains, float *ckpt, float *sub, void *dq, void *dkk, void *dvv,
+                      float *dg, float *db, float *dh0, int *err, cudaStream_t s) {
     using namespace kda::bwd;
     const size_t smem = sizeof(BwdSmem<D>);
     auto kern = kda_bwd_slice_kernel<D, TIn>;
@@ -237,16 +242,27 @@ kda_status launch_bwd(const void *q, const void *k, const void *v, const float *
         return KDA_ERR_CUDA;
     const long long grid = chains * (D / SLC);
     if (grid > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
-    kern<<<(unsigned)grid, 2 * D, smem, s>>>(
-        static_cast<const TIn *>(q), static_cast<const TIn *>(k), static_cast<const TIn *>(v), g,
-        beta, h0, cu, hdr, static_cast<const TIn *>(dO), dhT, T, H, ckpt, part,
-        static_cast<TIn *>(dvv), dh0, ntok, err);
-    kda_status st = launch_status();
-    if (st != KDA_OK) return st;
-    const long long n = ntok * H * (D + 1);
-    if (n == 0) return KDA_OK;
-    kda_bwd_reduce_kernel<D, TIn><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-        part, ntok, H, static_cast<TIn *>(dq), static_cast<TIn *>(dkk), dg, db);
+    // the D / 32 column slices of a chain are one thread-block cluster
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(NTB);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = D / SLC;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, static_cast<const TIn *>(q), static_cast<const TIn *>(k),
+                           static_cast<const TIn *>(v), g, beta, h0, (const int *)cu, hdr,
+                           static_cast<const TIn *>(dO), dhT, T, H, ckpt, sub,
+                           static_cast<TIn *>(dq), static_cast<TIn *>(dkk),
+                           static_cast<TIn *>(dvv), dg, db, dh0, ntok, err) != cudaSuccess) {
+        cudaGetLastError();
+        return KDA_ERR_CUDA;
+    }
     return launch_status();
 }
 
@@ -364,6 +380,18 @@ bool encode_input_map(CUtensorMap *m, const void *base, bool bf16, int H, long l
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The prep's four input tensor maps: q, k, v as 64-channel x 64-token boxes, g as
+// 32 whole rows.
+static bool encode_inputs(const void *q, const void *k, const void *v, const float *g, int H, int T,
+                   int nb, CUtensorMap *tq, CUtensorMap *tk, CUtensorMap *tv, CUtensorMap *tg) {
+    using kda::tc::C;
+    using kda::tc::D;
+    return encode_input_map(tq, q, true, H, T, nb, 64, C) &&
+           encode_input_map(tk, k, true, H, T, nb, 64, C) &&
+           encode_input_map(tv, v, true, H, T, nb, 64, C) &&
+           encode_input_map(tg, g, false, H, T, nb, D, C / 2);
+}
+
 // Tensor-core path, phase 1: chunk map (varlen) and the per-(chunk, head) records.
 static kda_status tc_intra(const void *q, const void *k, const void *v, const float *g,
                            const float *beta, const int32_t *cu, int N, int T, int H,
@@ -400,17 +428,49 @@ static kda_status tc_intra(const void *q, const void *k, const void *v, const fl
     // whose per-chunk bounds the kernel applies itself
     const int nb = cu ? 1 : N;
     CUtensorMap tq, tk, tv, tg;
-    if (!encode_input_map(&tq, q, true, H, T, nb, 64, C) ||
-        !encode_input_map(&tk, k, true, H, T, nb, 64, C) ||
-        !encode_input_map(&tv, v, true, H, T, nb, 64, C) ||
-        !encode_input_map(&tg, g, false, H, T, nb, D, C / 2))
-        return KDA_ERR_CUDA;
+    if (!encode_inputs(q, k, v, g, H, T, nb, &tq, &tk, &tv, &tg)) return KDA_ERR_CUDA;
     int *err = device_error_word();
     if (!err) return KDA_ERR_CUDA;
-    kda_tc_prep_kernel<<<grid, 256, smem, s>>>(tq, tk, tv, tg, beta, T, H, cps,
-                                               (int)L.max_chunks, hdr, cu ? chunks : nullptr,
-                                               ws + L.recs, err);
+    PrepArgs p{};
+    p.beta = beta;
+    p.T = T;
+    p.H = H;
+    p.cps = cps;
+    p.slots = (int)L.max_chunks;
+    p.hdr = hdr;
+    p.chunks = cu ? chunks : nullptr;
+    p.recs = ws + L.recs;
+    p.err_word = err;
+    p.nseq = N;
+    kda_tc_prep_kernel<<<grid, kPrepThreads, smem, s>>>(tq, tk, tv, tg, p);
     return launch_status();
+}
+
+// The state pass's arguments for an output pass over the records (no T-split).
+static kda::tc::StateArgs state_args(const float *h0, const int32_t *cu, int N, int T, int H,
+                                     const WsLayout &L, void *o, float *hT, void *workspace,
+                                     float *ckpt, int ckpt_chunks, long long ckpt_cap) {
+    using namespace kda::tc;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    StateArgs a{};
+    a.recs = ws + L.recs;
+    a.h0 = h0;
+    a.hT = hT;
+    a.o = static_cast<__nv_bfloat16 *>(o);
+    a.T = T;
+    a.H = H;
+    a.cps = cu ? 0 : (T + C - 1) / C;
+    a.hdr = reinterpret_cast<int *>(ws + L.hdr);
+    a.seq_off = reinterpret_cast<int *>(ws + L.seq_off);
+    a.cu = cu;
+    a.nseg = 1;
+    a.mode = kStateOutput;
+    a.ckpt = ckpt;
+    a.ckpt_chunks = ckpt_chunks;
+    a.ckpt_cap = ckpt_cap;
+    a.ntok = cu ? (long long)T : (long long)N * T;
+    a.max_chunks = (int)L.max_chunks;
+    return a;
 }
 
 // Tensor-core path, phase 2: the state pass over the records.
@@ -421,25 +481,8 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
     using namespace kda::tc;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *hdr = reinterpret_cast<int *>(ws + L.hdr);
-    int *seq_off = reinterpret_cast<int *>(ws + L.seq_off);
-    StateArgs a{};
-    a.recs = ws + L.recs;
-    a.h0 = h0;
-    a.hT = hT;
-    a.o = static_cast<__nv_bfloat16 *>(o);
-    a.T = T;
-    a.H = H;
-    a.cps = cu ? 0 : (T + C - 1) / C;
-    a.hdr = hdr;
-    a.seq_off = seq_off;
-    a.cu = cu;
+    StateArgs a = state_args(h0, cu, N, T, H, L, o, hT, workspace, ckpt, ckpt_chunks, ckpt_cap);
     a.nseg = L.nseg;
-    a.mode = kStateOutput;
-    a.ckpt = ckpt;
-    a.ckpt_chunks = ckpt_chunks;
-    a.ckpt_cap = ckpt_cap;
-    a.ntok = cu ? (long long)T : (long long)N * T;
-    a.max_chunks = (int)L.max_chunks;
     const long long chains = (long long)N * H;
     if (L.nseg <= 1) {
         // 32-column slices give the shortest per-chunk latency (they suit few chains);
@@ -464,6 +507,109 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
     if ((st = launch_status()) != KDA_OK) return st;
     a.s_in = s_in;
     return launch_state<32>(a, chains * L.nseg, s);
+}
+
+// Overlapped schedule (kda_tc_fused_kernel): one block per SM, 2 state CTAs
+// (64-column slices) per chain and two prep workers in every other block.  Chosen by
+// kda_fwd for fixed-length input without a T-split when its estimated time beats the
+// two launches by 5%.  The estimates use per-unit times measured on a B200 (1,965 MHz):
+//   two launches: a prep item takes a worker 12.2 us with 2 workers on every SM, then
+//     the 32-column state pass takes 0.79 us per chunk per wave of 4 CTAs per chain;
+//   one launch: a prep item takes 14.5 us (it shares the GPU with the state pass), a
+//     64-column chunk 1.19 us, and the chain starts about 5 us after the launch.
+// (B=1, H=16, T=1M: 19.7 against 23.8 ms; B=2, H=8, T=4,096: 0.139 against 0.140 ms.)
+constexpr double kPrepUsTwo = 12.2, kState32Us = 0.79;
+constexpr double kPrepUsOne = 14.5, kState64OneUs = 1.19, kRampUs = 5.0;
+static bool overlap_schedule(long long chains, long long cps, int sms) {
+    if (chains <= 0 || cps <= 0 || sms <= 0) return false;
+    const long long nstate = 2 * chains;
+    if (nstate > sms / 2) return false;
+    const double c = (double)chains, n = (double)cps;
+    const double prep_one = c * kPrepUsOne / (2.0 * (double)(sms - nstate));
+    const double one = n * (prep_one > kState64OneUs ? prep_one : kState64OneUs) + kRampUs;
+    const double two = n * (c * kPrepUsTwo / (2.0 * sms) +
+                            kState32Us * (double)((4 * chains + sms - 1) / sms));
+    return one < 0.95 * two;
+}
+
+// Both phases as one launch (fixed-length input, no T-split).
+static kda_status tc_fused(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const float *h0, int N, int T, int H,
+                           const WsLayout &L, void *o, float *hT, void *workspace,
+                           cudaStream_t s, float *ckpt = nullptr, int ckpt_chunks = 0,
+                           long long ckpt_cap = 0) {
+    using namespace kda::tc;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const long long chains = (long long)N * H, items = L.max_chunks * H;
+    if (items == 0 || items > 0x7fffffffLL - 4096) return KDA_ERR_INVALID_ARG;
+    const int sms = device_sms();
+    if (sms <= 0) return KDA_ERR_CUDA;
+    const long long nstate = 2 * chains;   // 64-column slices
+    if (nstate >= sms) return KDA_ERR_INVALID_ARG;
+    int *err = device_error_word();
+    if (!err) return KDA_ERR_CUDA;
+    CUtensorMap tq, tk, tv, tg;
+    if (!encode_inputs(q, k, v, g, H, T, N, &tq, &tk, &tv, &tg)) return KDA_ERR_CUDA;
+    int *ready = reinterpret_cast<int *>(ws + L.ready);
+    int *prog = reinterpret_cast<int *>(ws + L.prog);
+    if (nstate > kProgressSlots) return KDA_ERR_INVALID_ARG;
+    // flags and counters are contiguous: one memset
+    if (cudaMemsetAsync(ready, 0, L.prog + kProgressSlots * kProgStride * sizeof(int) - L.ready, s) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return KDA_ERR_CUDA;
+    }
+    PrepArgs p{};
+    p.beta = beta;
+    p.T = T;
+    p.H = H;
+    p.cps = (T + C - 1) / C;
+    p.slots = (int)L.max_chunks;
+    p.hdr = reinterpret_cast<int *>(ws + L.hdr);
+    p.chunks = nullptr;
+    p.recs = ws + L.recs;
+    p.err_word = err;
+    p.ready = ready;
+    p.nseq = N;
+    p.progress = prog;
+    // records in flight between the roles: about 48 MiB, well inside L2
+    const long long win = (48LL << 20) / (chains * (long long)REC_BYTES);
+    p.window = (int)(win < 2 ? 2 : win);
+    StateArgs a = state_args(h0, nullptr, N, T, H, L, o, hT, workspace, ckpt, ckpt_chunks, ckpt_cap);
+    a.err_word = err;
+    a.debug_drop_first_copy = debug_drop_first_copy();
+    a.ready = ready;
+    a.progress = prog;
+    if (cudaFuncSetAttribute(kda_tc_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kFusedSmem) != cudaSuccess) {
+        cudaGetLastError();
+        return KDA_ERR_CUDA;
+    }
+    // every block must be resident at once (state blocks wait for prep blocks): one
+    // block per SM, launched cooperatively
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)sms);
+    cfg.blockDim = dim3(kFusedThreads);
+    cfg.dynamicSmemBytes = kFusedSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kda_tc_fused_kernel, tq, tk, tv, tg, p, a, (int)nstate) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return KDA_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+// Whether kda_fwd takes the overlapped schedule for this problem.
+static bool use_overlap(const int32_t *cu, int N, int T, int H, const WsLayout &L) {
+    if (cu || L.nseg > 1 || T <= 0) return false;
+    return overlap_schedule((long long)N * H, ((long long)T + kda::tc::C - 1) / kda::tc::C,
+                            device_sms());
 }
 
 kda_status kda_fwd_intra(const void *q, const void *k, const void *v, const float *g,
@@ -508,6 +654,8 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
     if (N == 0) return KDA_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (is_tc_path(dtype, dk)) {
+        if (use_overlap(cu_seqlens, N, T, H, L))
+            return tc_fused(q, k, v, g, beta, h0, N, T, H, L, o, hT, workspace, s);
         if ((st = tc_intra(q, k, v, g, beta, cu_seqlens, N, T, H, L, workspace, s)) != KDA_OK)
             return st;
         return tc_inter(h0, cu_seqlens, N, T, H, L, o, hT, workspace, s);
@@ -552,10 +700,39 @@ kda_status kda_fwd_checkpointed(const void *q, const void *k, const void *v, con
     if (!cu_seqlens && (long long)B * (T / ckpt_every) > ckpt_capacity) return KDA_ERR_INVALID_ARG;
     if (N == 0) return KDA_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (use_overlap(cu_seqlens, N, T, H, L))
+        return tc_fused(q, k, v, g, beta, h0, N, T, H, L, o, hT, workspace, s, ckpts,
+                        ckpt_every / kda::tc::C, ckpt_capacity);
     if ((st = tc_intra(q, k, v, g, beta, cu_seqlens, N, T, H, L, workspace, s)) != KDA_OK)
         return st;
     return tc_inter(h0, cu_seqlens, N, T, H, L, o, hT, workspace, s, ckpts,
                     ckpt_every / kda::tc::C, ckpt_capacity);
+}
+
+int kda_fwd_plan_overlap(int B, int T, int H, int dk, int dv, int num_seqs, int dtype) {
+    if (B < 0 || T < 0 || num_seqs != 0) return 0;
+    if (check_shape(H, dk, dv, dtype) != KDA_OK || !is_tc_path(dtype, dk)) return 0;
+    const WsLayout L = ws_layout(B, T, H, dk, 0, dtype, 0, device_sms());
+    return use_overlap(nullptr, B, T, H, L) ? 1 : 0;
+}
+
+kda_status kda_fwd_overlapped(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *h0, int B, int T, int H, int dk,
+                              int dv, int dtype, void *o, float *hT, void *workspace,
+                              size_t ws_bytes, void *stream) {
+    int N;
+    WsLayout L;
+    kda_status st = validate_fwd(q, k, v, g, beta, h0, nullptr, 0, B, T, H, dk, dv, dtype, o, hT,
+                                 workspace, ws_bytes, true, true, &N, &L, /*nseg_req=*/1);
+    if (st != KDA_OK) return st;
+    if (!is_tc_path(dtype, dk)) return KDA_ERR_UNSUPPORTED_SHAPE;
+    const int sms = device_sms();
+    if (sms <= 0) return KDA_ERR_CUDA;
+    if (2LL * N * H >= sms) return KDA_ERR_UNSUPPORTED_SHAPE;
+    if (N == 0) return KDA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) return tc_inter(h0, nullptr, N, T, H, L, o, hT, workspace, s);   // hT = h0
+    return tc_fused(q, k, v, g, beta, h0, N, T, H, L, o, hT, workspace, s);
 }
 
 int kda_fwd_plan_segments(int B, int T, int H, int dk, int dv, int num_seqs, int dtype) {
@@ -761,11 +938,11 @@ kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
         if ((st = launch_status()) != KDA_OK) return st;
     }
     float *ckpt = reinterpret_cast<float *>(ws + L.ckpt);
-    float *part = reinterpret_cast<float *>(ws + L.part);
+    float *sub = reinterpret_cast<float *>(ws + L.sub);
     const long long chains = (long long)N * H;
 #define KDA_BWD(DD, TT)                                                                    \
     return launch_bwd<DD, TT>(q, k, v, g, beta, h0, cu_seqlens, hdr, grad_o, grad_hT, T, H, \
-                              ntok, chains, ckpt, part, grad_q, grad_k, grad_v, grad_g,     \
+                              ntok, chains, ckpt, sub, grad_q, grad_k, grad_v, grad_g,      \
                               grad_beta, grad_h0, err, s)
     if (dtype == KDA_DTYPE_BF16) {
         if (dk == 32) KDA_BWD(32, __nv_bfloat16);

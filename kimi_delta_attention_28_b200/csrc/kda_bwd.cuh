@@ -10,12 +10,20 @@
 //     G' = G - k dd^T;  dg_i = sum_j S'_ij G'_ij;  G = Diag(exp g) G';   dh0 = G.
 // The state's value columns evolve independently in both directions (the forward
 // update and the G update act column by column), so a CTA owns one 32-column slice
-// of one (sequence, head) chain: it runs the chain forward once, storing its slice
-// of the state every CB tokens, then walks the chunks of CB tokens backwards,
-// recomputing each chunk's states into shared memory and applying the rules above.
-// dv and dh0 columns are complete within a slice; dq, dk, dg and dbeta are sums over
-// all columns, so every slice writes its partial sums and a second kernel adds the
-// slices (in a fixed order: the result does not depend on scheduling).
+// of one (sequence, head) chain.  It runs the chain forward once, storing its slice
+// of the state every CK tokens in HBM; then it walks the CK-token chunks backwards:
+// from a chunk's checkpoint it recomputes the state every CB tokens into a small
+// scratch of its own (L2-resident), and for each CB-token piece, last first, the
+// piece's states into shared memory, to which it applies the rules above.  dv and
+// dh0 columns are complete within a slice; dq, dk, dg and dbeta are sums over all
+// columns: the D/32 slice CTAs of a chain form a thread-block cluster, and after
+// every piece each CTA adds the slices' partial sums for a quarter of the rows
+// through distributed shared memory, in slice order (deterministic).
+// Inside a CTA, warp w owns 4 columns of the slice across all d rows (lane l: rows
+// RPL l .. RPL l + RPL - 1, RPL = d / 32), so the column sums every token needs
+// (u = S'^T k, G^T k) are in-warp butterflies with no CTA barrier; the row sums
+// (dq, dk, dg, dbeta) are only outputs, so each warp's share goes to shared memory
+// and the eight shares are added once per token.
 #pragma once
 
 #include "kda_common.cuh"
@@ -23,8 +31,10 @@
 namespace kda {
 namespace bwd {
 
-constexpr int SLC = 32;   // value columns per CTA
-constexpr int CB = 8;     // tokens per recompute chunk (states of a chunk live in smem)
+constexpr int SLC = 16;   // value columns per CTA
+constexpr int CK = 64;    // tokens per stored checkpoint (HBM)
+constexpr int CB = 8;     // tokens per recompute piece (their states live in smem)
+constexpr int NSUB = CK / CB;
 
 template <typename TIn>
 KDA_DEVINL float ldf(const TIn *p);
@@ -40,98 +50,93 @@ template <>
 KDA_DEVINL void stf<__nv_bfloat16>(__nv_bfloat16 *p, float x) { *p = f2bf(x); }
 
 // Checkpoint slot of chunk j of a sequence starting at token t0 of the flattened
-// token axis, sequence index n: floor(t0 / CB) + n + j.  Distinct sequences get
-// disjoint slot ranges, and slots < T_total / CB + N + 1.
-KDA_DEVINL long long ckpt_slot(int t0, int n, int j) { return (long long)(t0 / CB) + n + j; }
+// token axis, sequence index n: floor(t0 / CK) + n + j.  Distinct sequences get
+// disjoint slot ranges, and slots < T_total / CK + N + 1.
+KDA_DEVINL long long ckpt_slot(int t0, int n, int j) { return (long long)(t0 / CK) + n + j; }
 
-template <int D>
-struct BwdSmem {
-    float st[CB][D][SLC];      // states S_{t-1} of the chunk's tokens (this slice)
-    float q[CB][D], k[CB][D], a[CB][D];   // a = exp(g)
-    float v[CB][SLC], dO[CB][SLC], delta[CB][SLC];
-    float b[CB];
-    float part[D / 16][SLC];   // column-reduction partials, one row per warp
-    float vec[SLC];            // column-reduction result
-    float red[D / 16];         // dbeta partials, one per warp
-};
+// Distributed shared memory: the shared-memory address of `p` in CTA `rank` of the
+// cluster, and a load from it.
+KDA_DEVINL uint32_t dsmem_addr(const void *p, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    return a;
+}
+KDA_DEVINL float dsmem_ld(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+KDA_DEVINL void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
 
-// Column sum over the D rows of x (thread: row tid/2, columns 16 (tid & 1) .. +15 of
-// the slice).  Within a warp (16 rows x 2 column halves) a reduce-scatter over the
-// four row bits of the lane leaves lane l with one column summed over the warp's
-// rows; the warps' partials are added through shared memory.  The result for this
-// thread's 16 columns is returned in out; the CTA synchronises twice.
+constexpr int NWB = SLC / 4;   // warps per CTA (4 columns each)
+constexpr int NTB = 32 * NWB;   // threads per CTA
+
+// Row-sum slots of one token (dq, dk, dg rows, then dbeta), padded to 16 bytes.
 template <int D>
-KDA_DEVINL void col_sum(BwdSmem<D> &sm, const float (&x)[16], float (&out)[16]) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, ch = tid & 1;
-    float c8[8], c4[4], c2[2];
-    {
-        const bool up = lane & 2;
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            const float send = up ? x[p] : x[p + 8];
-            c8[p] = (up ? x[p + 8] : x[p]) + __shfl_xor_sync(0xffffffffu, send, 2);
-        }
+constexpr int psw() { return 3 * D + 4; }
+
+// RPL consecutive fp32 values from shared memory (16-byte aligned for RPL = 4), as
+// one vector access.
+template <int RPL>
+KDA_DEVINL void ld_rows(const float *p, float (&x)[RPL]) {
+    if constexpr (RPL == 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(p);
+        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    } else if constexpr (RPL == 2) {
+        const float2 v = *reinterpret_cast<const float2 *>(p);
+        x[0] = v.x; x[1] = v.y;
+    } else {
+        x[0] = *p;
     }
-    {
-        const bool up = lane & 4;
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float send = up ? c8[p] : c8[p + 4];
-            c4[p] = (up ? c8[p + 4] : c8[p]) + __shfl_xor_sync(0xffffffffu, send, 4);
-        }
-    }
-    {
-        const bool up = lane & 8;
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const float send = up ? c4[p] : c4[p + 2];
-            c2[p] = (up ? c4[p + 2] : c4[p]) + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-    }
-    float c1;
-    {
-        const bool up = lane & 16;
-        const float send = up ? c2[0] : c2[1];
-        c1 = (up ? c2[1] : c2[0]) + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-    // lane bits 1..4 chose the halves 8, 4, 2, 1: the column within this half
-    const int col = ((lane >> 1) & 1) * 8 + ((lane >> 2) & 1) * 4 + ((lane >> 3) & 1) * 2 +
-                    ((lane >> 4) & 1);
-    sm.part[warp][ch * 16 + col] = c1;
-    __syncthreads();
-    if (tid < SLC) {
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < D / 16; ++w) s += sm.part[w][tid];
-        sm.vec[tid] = s;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int c = 0; c < 16; c += 4) {
-        const float4 t = *reinterpret_cast<const float4 *>(&sm.vec[ch * 16 + c]);
-        out[c] = t.x;
-        out[c + 1] = t.y;
-        out[c + 2] = t.z;
-        out[c + 3] = t.w;
+}
+template <int RPL>
+KDA_DEVINL void st_rows(float *p, const float (&x)[RPL]) {
+    if constexpr (RPL == 4) {
+        *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    } else if constexpr (RPL == 2) {
+        *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+    } else {
+        *p = x[0];
     }
 }
 
+template <int D>
+struct BwdSmem {
+    float st[CB][D][SLC];      // states S_{t-1} of the piece's tokens (this slice)
+    float q[CB][D], k[CB][D], a[CB][D];   // a = exp(g)
+    float v[CB][SLC], dO[CB][SLC];
+    float b[CB];
+    float pw[2][NWB][psw<D>()];   // each warp's share of a token's dq, dk, dg, dbeta
+    float ps[CB][psw<D>()];       // this slice's partial dq, dk, dg rows and dbeta per token
+};
+
+// Sum of x over the 32 lanes of the warp, left in every lane.
+KDA_DEVINL float warp_sum(float x) {
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
 template <int D, typename TIn>
-__global__ void __launch_bounds__(2 * D, 1)
+__global__ void __launch_bounds__(NTB, 1)
 kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                      const TIn *__restrict__ v, const float *__restrict__ g,
                      const float *__restrict__ beta, const float *__restrict__ h0,
                      const int *__restrict__ cu, const int *__restrict__ hdr,
                      const TIn *__restrict__ dO, const float *__restrict__ dhT, int T, int H,
-                     float *__restrict__ ckpt, float *__restrict__ part, TIn *__restrict__ dv,
-                     float *__restrict__ dh0, long long ntok, int *err_word) {
-    constexpr int NS = D / SLC, NT = 2 * D;
+                     float *__restrict__ ckpt, float *__restrict__ sub, TIn *__restrict__ dq,
+                     TIn *__restrict__ dk, TIn *__restrict__ dv, float *__restrict__ dg,
+                     float *__restrict__ dbeta, float *__restrict__ dh0, long long ntok,
+                     int *err_word) {
+    constexpr int NS = D / SLC, NT = NTB, RPL = D / 32;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     BwdSmem<D> &sm = *reinterpret_cast<BwdSmem<D> *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int r = tid >> 1, ch = tid & 1;
+    const int r0 = RPL * lane, c4 = 4 * warp;        // this thread: rows r0.., slice columns c4..
     const int slice = blockIdx.x % NS, chain = blockIdx.x / NS, n = chain / H, h = chain % H;
-    const int cs = slice * SLC, cc = cs + ch * 16;   // slice's first column, this thread's
+    const int cs = slice * SLC;                      // the slice's first column
     int t0, len;
     if (cu) {
         if (!hdr[0]) return;
@@ -147,11 +152,28 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
             return;
         }
     }
-    const int nch = (len + CB - 1) / CB;
-    const size_t sstate = (size_t)chain * D * D + (size_t)r * D + cc;   // h0 / dhT / dh0 offset
-    // a chunk's inputs into shared memory: q, k, exp(g) rows; this slice's v, dO columns
-    auto stage = [&](int j, bool with_q) {
-        const int c0 = t0 + j * CB, cl = min(CB, len - j * CB);
+    const int nck = (len + CK - 1) / CK;
+    // this thread's RPL x 4 block of a [D][D] state (h0, dhT, dh0, checkpoints) and of
+    // the CTA's [D][SLC] scratch
+    const size_t sbase = (size_t)chain * D * D + cs + c4;
+    float *mysub = sub + (size_t)blockIdx.x * NSUB * D * SLC + c4;
+    auto ldS = [&](float (&S)[RPL][4], const float *base, int ld) {
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            const float4 x = *reinterpret_cast<const float4 *>(base + (size_t)(r0 + i) * ld);
+            S[i][0] = x.x; S[i][1] = x.y; S[i][2] = x.z; S[i][3] = x.w;
+        }
+    };
+    auto stS = [&](float *base, int ld, const float (&S)[RPL][4]) {
+#pragma unroll
+        for (int i = 0; i < RPL; ++i)
+            *reinterpret_cast<float4 *>(base + (size_t)(r0 + i) * ld) =
+                make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
+    };
+    // a piece's inputs into shared memory (tokens p0 .. p0 + cl - 1 of the sequence):
+    // q, k, exp(g) rows; this slice's v, dO columns; beta
+    auto stage = [&](int p0, int cl, bool with_q) {
+        const int c0 = t0 + p0;
         for (int e = tid; e < CB * D; e += NT) {
             const int i = e / D, c = e % D;
             const bool in = i < cl;
@@ -170,163 +192,177 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         if (tid < CB) sm.b[tid] = tid < cl ? __ldg(beta + (size_t)(c0 + tid) * H + h) : 0.f;
         __syncthreads();
     };
-    // one token of the recurrence on this thread's part of the state; delta to smem
-    auto step = [&](float (&S)[16], int i, bool keep_delta) {
-        const float a = sm.a[i][r], kr = sm.k[i][r], b = sm.b[i];
-        float x[16], u[16];
+    // one token of the recurrence on this thread's block; returns delta = v - u for the
+    // warp's 4 columns (the same in every lane)
+    auto step = [&](float (&S)[RPL][4], int i, float (&dl)[4]) {
+        float u[4] = {0.f, 0.f, 0.f, 0.f}, av[RPL], kv[RPL];
+        ld_rows<RPL>(&sm.a[i][r0], av);
+        ld_rows<RPL>(&sm.k[i][r0], kv);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            S[c] *= a;
-            x[c] = kr * S[c];
+        for (int ri = 0; ri < RPL; ++ri) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                S[ri][c] *= av[ri];
+                u[c] = fmaf(kv[ri], S[ri][c], u[c]);
+            }
         }
-        col_sum<D>(sm, x, u);
+        const float b = sm.b[i];
+        const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][c4]);
+        dl[0] = vv.x - warp_sum(u[0]);
+        dl[1] = vv.y - warp_sum(u[1]);
+        dl[2] = vv.z - warp_sum(u[2]);
+        dl[3] = vv.w - warp_sum(u[3]);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const float dl = sm.v[i][ch * 16 + c] - u[c];
-            S[c] = fmaf(b * kr, dl, S[c]);
-            if (keep_delta && r == 0) sm.delta[i][ch * 16 + c] = dl;
+        for (int ri = 0; ri < RPL; ++ri) {
+            const float bk = b * kv[ri];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) S[ri][c] = fmaf(bk, dl[c], S[ri][c]);
         }
     };
+    // run the tokens p0 .. p0 + cl - 1 forward from S (inputs staged here)
+    auto run = [&](float (&S)[RPL][4], int p0, int cl) {
+        stage(p0, cl, false);
+        float dl[4];
+        for (int i = 0; i < cl; ++i) step(S, i, dl);
+        __syncthreads();   // the next staging overwrites the inputs
+    };
 
-    // ---- forward: the slice's state at the start of every chunk ----
-    float S[16];
+    // ---- forward: the slice's state at the start of every CK-token chunk, to HBM ----
+    float S[RPL][4];
+    if (h0) ldS(S, h0 + sbase, D);
+    else
 #pragma unroll
-    for (int c = 0; c < 16; c += 4) {
-        const float4 x = h0 ? *reinterpret_cast<const float4 *>(h0 + sstate + c)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-        S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
-    }
-    for (int j = 0; j < nch; ++j) {
-        float *cp = ckpt + ((ckpt_slot(t0, n, j) * H + h) * D + r) * D + cc;
-#pragma unroll
-        for (int c = 0; c < 16; c += 4)
-            *reinterpret_cast<float4 *>(cp + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
-        stage(j, false);
-        const int cl = min(CB, len - j * CB);
-        for (int i = 0; i < cl; ++i) step(S, i, false);
-        __syncthreads();   // the next chunk's staging overwrites the inputs
+        for (int i = 0; i < RPL; ++i) S[i][0] = S[i][1] = S[i][2] = S[i][3] = 0.f;
+    for (int j = 0; j < nck; ++j) {
+        stS(ckpt + (ckpt_slot(t0, n, j) * H + h) * D * D + cs + c4, D, S);
+        const int lenj = min(CK, len - j * CK);
+        for (int p = 0; p < lenj; p += CB) run(S, j * CK + p, min(CB, lenj - p));
     }
 
     // ---- backward ----
-    float G[16];
+    float G[RPL][4];
+    if (dhT) ldS(G, dhT + sbase, D);
+    else
 #pragma unroll
-    for (int c = 0; c < 16; c += 4) {
-        const float4 x = dhT ? *reinterpret_cast<const float4 *>(dhT + sstate + c)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        G[c] = x.x; G[c + 1] = x.y; G[c + 2] = x.z; G[c + 3] = x.w;
-    }
-    const size_t pstride = (size_t)ntok * H;   // partial sums: [NS][ntok * H][3 D + 1]
-    for (int j = nch - 1; j >= 0; --j) {
-        const int cl = min(CB, len - j * CB);
-        stage(j, true);
-        const float *cp = ckpt + ((ckpt_slot(t0, n, j) * H + h) * D + r) * D + cc;
-#pragma unroll
-        for (int c = 0; c < 16; c += 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(cp + c);
-            S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
+        for (int i = 0; i < RPL; ++i) G[i][0] = G[i][1] = G[i][2] = G[i][3] = 0.f;
+    const uint32_t cl_rank = (uint32_t)slice;   // the cluster holds the chain's NS slices
+    int tok = 0;                                // tokens done: parity of the pw buffer
+    for (int j = nck - 1; j >= 0; --j) {
+        const int lenj = min(CK, len - j * CK), npc = (lenj + CB - 1) / CB;
+        // the state every CB tokens of the chunk, from its checkpoint, to this CTA's scratch
+        ldS(S, ckpt + (ckpt_slot(t0, n, j) * H + h) * D * D + cs + c4, D);
+        for (int pc = 0; pc < npc; ++pc) {
+            stS(mysub + (size_t)pc * D * SLC, SLC, S);
+            if (pc + 1 < npc) run(S, j * CK + pc * CB, min(CB, lenj - pc * CB));
         }
-        for (int i = 0; i < cl; ++i) {   // recompute: S_{t-1} of every token to smem
+        for (int pc = npc - 1; pc >= 0; --pc) {
+            const int p0 = j * CK + pc * CB, cl = min(CB, lenj - pc * CB);
+            stage(p0, cl, true);
+            ldS(S, mysub + (size_t)pc * D * SLC, SLC);
+            float dls[CB][4];   // delta of every token of the piece (this warp's columns)
 #pragma unroll
-            for (int c = 0; c < 16; c += 4)
-                *reinterpret_cast<float4 *>(&sm.st[i][r][ch * 16 + c]) =
-                    make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
-            step(S, i, true);
+            for (int i = 0; i < CB; ++i) {   // recompute: S_{t-1} of every token to smem
+                if (i < cl) {
+                    stS(&sm.st[i][0][c4], SLC, S);
+                    step(S, i, dls[i]);
+                }
+            }
+#pragma unroll
+            for (int i = CB - 1; i >= 0; --i) {
+                if (i >= cl) continue;
+                const float b = sm.b[i];
+                float Sp[RPL][4], dov[4], av[RPL], kv[RPL], qv[RPL];
+                {
+                    const float4 d4 = *reinterpret_cast<const float4 *>(&sm.dO[i][c4]);
+                    dov[0] = d4.x; dov[1] = d4.y; dov[2] = d4.z; dov[3] = d4.w;
+                }
+                ld_rows<RPL>(&sm.a[i][r0], av);
+                ld_rows<RPL>(&sm.k[i][r0], kv);
+                ld_rows<RPL>(&sm.q[i][r0], qv);
+                // G += q do^T; dq = S_t do with S_t = S' + b k delta^T; w = G delta
+                float pq[RPL], pwr[RPL], xk[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ri = 0; ri < RPL; ++ri) {
+                    const int r = r0 + ri;
+                    const float a = av[ri], kr = kv[ri], qr = qv[ri];
+                    const float4 sv = *reinterpret_cast<const float4 *>(&sm.st[i][r][c4]);
+                    Sp[ri][0] = a * sv.x; Sp[ri][1] = a * sv.y; Sp[ri][2] = a * sv.z; Sp[ri][3] = a * sv.w;
+                    pq[ri] = 0.f;
+                    pwr[ri] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        G[ri][c] = fmaf(qr, dov[c], G[ri][c]);
+                        pq[ri] = fmaf(fmaf(b * kr, dls[i][c], Sp[ri][c]), dov[c], pq[ri]);
+                        pwr[ri] = fmaf(G[ri][c], dls[i][c], pwr[ri]);
+                        xk[c] = fmaf(kr, G[ri][c], xk[c]);
+                    }
+                }
+                // dd = b G^T k for the warp's columns (complete: this CTA owns them)
+                float dd[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) dd[c] = b * warp_sum(xk[c]);
+                if (lane < 4)
+                    stf<TIn>(dv + ((size_t)(t0 + p0 + i) * H + h) * D + cs + c4 + lane,
+                             lane == 0 ? dd[0] : lane == 1 ? dd[1] : lane == 2 ? dd[2] : dd[3]);
+                float pbeta = 0.f, pk[RPL], pgs[RPL];
+                float *pwb = sm.pw[tok & 1][warp];
+#pragma unroll
+                for (int ri = 0; ri < RPL; ++ri) {
+                    const float a = av[ri], kr = kv[ri];
+                    float px = 0.f, pg = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        px = fmaf(Sp[ri][c], dd[c], px);
+                        const float gp = G[ri][c] - kr * dd[c];
+                        pg = fmaf(Sp[ri][c], gp, pg);
+                        G[ri][c] = a * gp;
+                    }
+                    pk[ri] = b * pwr[ri] - px;
+                    pgs[ri] = pg;
+                    pbeta = fmaf(kr, pwr[ri], pbeta);
+                }
+                st_rows<RPL>(pwb + r0, pq);
+                st_rows<RPL>(pwb + D + r0, pk);
+                st_rows<RPL>(pwb + 2 * D + r0, pgs);
+                pbeta = warp_sum(pbeta);
+                if (lane == 0) pwb[3 * D] = pbeta;
+                __syncthreads();
+                // the warps' shares, added in warp order, into the piece's partial sums
+                for (int e = tid; e < 3 * D + 1; e += NT) {
+                    float sum = 0.f;
+#pragma unroll
+                    for (int w = 0; w < NWB; ++w) sum += sm.pw[tok & 1][w][e];
+                    sm.ps[i][e] = sum;
+                }
+                ++tok;
+            }
+            // the slices' partial sums of the piece: every CTA of the cluster adds them for
+            // D / NS rows (and CTA 0 for dbeta), in slice order
+            cluster_sync();
+            {
+                constexpr int RPC = D / NS;                   // rows per CTA
+                for (int e = tid; e < cl * (3 * RPC + 1); e += NT) {
+                    const int i = e / (3 * RPC + 1), f = e % (3 * RPC + 1);
+                    if (f == 3 * RPC && cl_rank != 0) continue;
+                    const int col = f == 3 * RPC ? 3 * D : (f / RPC) * D + cl_rank * RPC + f % RPC;
+                    float sum = 0.f;
+#pragma unroll
+                    for (int sl = 0; sl < NS; ++sl) sum += dsmem_ld(dsmem_addr(&sm.ps[i][col], sl));
+                    const size_t u = (size_t)(t0 + p0 + i) * H + h;
+                    if (f == 3 * RPC) {
+                        dbeta[u] = sum;
+                    } else {
+                        const int kind = f / RPC, row = cl_rank * RPC + f % RPC;
+                        if (kind == 0) stf<TIn>(dq + u * D + row, sum);
+                        else if (kind == 1) stf<TIn>(dk + u * D + row, sum);
+                        else dg[u * D + row] = sum;
+                    }
+                }
+            }
+            cluster_sync();   // the partial sums may be overwritten by the next piece
         }
-        __syncthreads();   // delta visible
-        for (int i = cl - 1; i >= 0; --i) {
-            const int t = t0 + j * CB + i;
-            const float a = sm.a[i][r], kr = sm.k[i][r], qr = sm.q[i][r], b = sm.b[i];
-            float Sp[16], dl[16], dov[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                Sp[c] = a * sm.st[i][r][ch * 16 + c];
-                dl[c] = sm.delta[i][ch * 16 + c];
-                dov[c] = sm.dO[i][ch * 16 + c];
-            }
-            // G += q do^T; dq = S_t do with S_t = S' + b k delta^T; w = G delta
-            float pq = 0.f, pw = 0.f, x[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                G[c] = fmaf(qr, dov[c], G[c]);
-                pq = fmaf(fmaf(b * kr, dl[c], Sp[c]), dov[c], pq);
-                pw = fmaf(G[c], dl[c], pw);
-                x[c] = kr * G[c];
-            }
-            pq += __shfl_xor_sync(0xffffffffu, pq, 1);
-            pw += __shfl_xor_sync(0xffffffffu, pw, 1);
-            // dd = b G^T k: the column sum (complete: this CTA owns the columns)
-            float dd[16];
-            col_sum<D>(sm, x, dd);
-            if (tid < SLC) stf<TIn>(dv + ((size_t)t * H + h) * D + cs + tid, b * sm.vec[tid]);
-            float px = 0.f, pg = 0.f;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                dd[c] *= b;
-                px = fmaf(Sp[c], dd[c], px);
-                const float gp = G[c] - kr * dd[c];
-                pg = fmaf(Sp[c], gp, pg);
-                G[c] = a * gp;
-            }
-            px += __shfl_xor_sync(0xffffffffu, px, 1);
-            pg += __shfl_xor_sync(0xffffffffu, pg, 1);
-            // dbeta partial = sum over rows of k_r w_r (rows of this warp, then warps)
-            float pb = ch == 0 ? kr * pw : 0.f;
-#pragma unroll
-            for (int m = 16; m > 0; m >>= 1) pb += __shfl_xor_sync(0xffffffffu, pb, m);
-            if (lane == 0) sm.red[warp] = pb;
-            float *pp = part + ((size_t)slice * pstride + (size_t)t * H + h) * (3 * D + 1);
-            if (ch == 0) {
-                pp[r] = pq;
-                pp[D + r] = b * pw - px;
-                pp[2 * D + r] = pg;
-            }
-            __syncthreads();
-            if (tid == 0) {
-                float s = 0.f;
-#pragma unroll
-                for (int w = 0; w < D / 16; ++w) s += sm.red[w];
-                pp[3 * D] = s;
-            }
-        }
-        __syncthreads();   // the next chunk's staging overwrites the inputs and states
     }
-    if (dh0) {
-#pragma unroll
-        for (int c = 0; c < 16; c += 4)
-            *reinterpret_cast<float4 *>(dh0 + sstate + c) = make_float4(G[c], G[c + 1], G[c + 2], G[c + 3]);
-    }
-}
-
-// Sum of the slices' partials: dq, dk (input dtype), dg and dbeta (fp32).  One thread
-// per (token, head, row); the slices are added in index order.
-template <int D, typename TIn>
-__global__ void __launch_bounds__(256)
-kda_bwd_reduce_kernel(const float *__restrict__ part, long long ntok, int H,
-                      TIn *__restrict__ dq, TIn *__restrict__ dk, float *__restrict__ dg,
-                      float *__restrict__ dbeta) {
-    constexpr int NS = D / SLC;
-    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long units = ntok * H;
-    if (e >= units * (D + 1)) return;
-    const long long u = e / (D + 1);
-    const int r = (int)(e % (D + 1));
-    const size_t pstride = (size_t)units * (3 * D + 1);
-    if (r == D) {
-        float s = 0.f;
-        for (int sl = 0; sl < NS; ++sl) s += part[sl * pstride + (size_t)u * (3 * D + 1) + 3 * D];
-        dbeta[u] = s;
-        return;
-    }
-    float a = 0.f, b = 0.f, c = 0.f;
-    for (int sl = 0; sl < NS; ++sl) {
-        const float *pp = part + sl * pstride + (size_t)u * (3 * D + 1);
-        a += pp[r];
-        b += pp[D + r];
-        c += pp[2 * D + r];
-    }
-    stf<TIn>(dq + (size_t)u * D + r, a);
-    stf<TIn>(dk + (size_t)u * D + r, b);
-    dg[(size_t)u * D + r] = c;
+    if (dh0) stS(dh0 + sbase, D, G);
 }
 
 }  // namespace bwd

@@ -159,6 +159,54 @@ KDA_DEVINL bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
         if (global_timer_ns() - t0 > kWaitLimitNs) return false;
     return true;
 }
+
+// ---- named CTA barriers (a group of `n` threads, a multiple of 32, on barrier `id`) ----
+// With id 0 and n = the block size these are __syncthreads and its reductions; other
+// ids let independent thread groups of one CTA synchronise among themselves.
+KDA_DEVINL void bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+KDA_DEVINL bool bar_and(int id, int n, bool p) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+                 " bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+                 : "=r"(r) : "r"((uint32_t)p), "r"(id), "r"(n) : "memory");
+    return r != 0;
+}
+KDA_DEVINL bool bar_or(int id, int n, bool p) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+                 " bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+                 : "=r"(r) : "r"((uint32_t)p), "r"(id), "r"(n) : "memory");
+    return r != 0;
+}
+
+// ---- flags between CTAs of one launch (GPU scope) ----
+// Generic-proxy accesses of global memory before this fence are ordered with this
+// thread's later asynchronous-proxy (bulk copy) accesses, and the other way round.
+KDA_DEVINL void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;\n" ::: "memory"); }
+KDA_DEVINL void flag_release(int *f, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(f), "r"(v) : "memory");
+}
+// A counter another CTA only reads as a hint (no ordering with other accesses).
+KDA_DEVINL void store_relaxed(int *f, int v) {
+    asm volatile("st.relaxed.gpu.global.b32 [%0], %1;\n" ::"l"(f), "r"(v) : "memory");
+}
+KDA_DEVINL int flag_acquire(const int *f) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+// Wait until *f != 0, with the same wall-clock limit as the barrier waits.
+KDA_DEVINL bool flag_wait_bounded(const int *f) {
+    if (flag_acquire(f)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!flag_acquire(f)) {
+        __nanosleep(64);
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
 // Tiled 4-D tensor copy global -> this CTA's shared memory by the tensor-memory-access
 // engine, completing on `bar`: the box of the tensor map `tm` at coordinates
 // (c0, c1, c2, c3), innermost first.  Coordinates past the tensor's extent read zeros.

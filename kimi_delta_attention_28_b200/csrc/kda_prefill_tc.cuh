@@ -195,33 +195,89 @@ struct PrepSmem {
     uint32_t tmem_slot;            // tensor-memory base address (written by tcgen05.alloc)
 };
 
-__global__ void __launch_bounds__(256, 2)
-kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                   const float *__restrict__ beta, int T, int H, int cps, int slots,
-                   const int *__restrict__ hdr, const ChunkLoc *__restrict__ chunks,
-                   uint8_t *__restrict__ recs, int *err_word) {
-    extern __shared__ uint8_t smem_raw[];
-    // 1024-byte alignment: the swizzled operand tiles are read by the tensor core
-    PrepSmem &sm = *reinterpret_cast<PrepSmem *>(
-        smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
-    uint32_t *tmem_slot = &sm.tmem_slot;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// Arguments of kernel 1 besides the tensor maps.
+struct PrepArgs {
+    const float *beta;
+    int T, H, cps, slots;
+    const int *hdr;
+    const ChunkLoc *chunks;
+    uint8_t *recs;
+    int *err_word;
+    // Overlapped schedule (one launch with the state pass, fixed-length input only):
+    // items in time order -- chunk j of every (sequence, head) before chunk j + 1 --
+    // and a flag per record, ready[chunk * H + head], set (release, GPU scope) once
+    // the record is complete.  Null: items in sequence order, no flags.
+    int *ready;
+    int nseq;
+    // Overlapped schedule: chunks each state CTA has started copying in (2 CTAs per
+    // chain, column tile fastest); a worker starts the item of chunk j of a chain only
+    // once both of the chain's CTAs have reached chunk j - window, so the records in
+    // flight between the two roles stay within L2.  Null: no limit.
+    const int *progress;
+    int window;
+};
+constexpr int kPrepThreads = 256;   // one prep worker: 8 warps
+
+// Progress counters of the state CTAs: one per 128-byte line, so that pollers of
+// one chain do not contend with the stores of another.
+constexpr int kProgStride = 32;
+// Wait until both state CTAs of a chain have started chunk `need` (bounded; polled
+// about once a microsecond: the counters advance once per chunk period).
+KDA_DEVINL bool progress_wait_bounded(const int *prog2, int need) {
+    auto reached = [&]() {
+        int a, b;
+        asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];\n" : "=r"(a) : "l"(prog2) : "memory");
+        asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];\n"
+                     : "=r"(b) : "l"(prog2 + kProgStride) : "memory");
+        return a >= need && b >= need;
+    };
+    if (reached()) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!reached()) {
+        __nanosleep(1000);
+        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// One prep worker: `kPrepThreads` threads (tid 0..255) with their own PrepSmem, the
+// 2D tensor-memory columns at `tmem` (allocated by the caller) and named barrier
+// `bar`, walking items worker, worker + nworkers, ...
+KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                            const CUtensorMap &tm_v, const CUtensorMap &tm_g, const PrepArgs &p,
+                            PrepSmem &sm, const uint32_t tmem, const int tid, const int bar,
+                            const int worker, const int nworkers) {
+    const float *__restrict__ beta = p.beta;
+    const int T = p.T, H = p.H, cps = p.cps, slots = p.slots;
+    const int *__restrict__ hdr = p.hdr;
+    const ChunkLoc *__restrict__ chunks = p.chunks;
+    uint8_t *__restrict__ recs = p.recs;
+    int *err_word = p.err_word;
+    const int lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
     if (chunks && !hdr[0]) return;
     const int items = (chunks ? min(hdr[1], slots) : slots) * H;
-    if ((int)blockIdx.x >= items) return;
+    if (worker >= items) return;
     const uint32_t s_ka = smem_u32(sm.ka), s_qa = smem_u32(sm.qa), s_kb = smem_u32(sm.kb);
 
     struct Item {
         int t0, len, h;
         int tl, b;         // the chunk's token and batch coordinates in the tensor maps
+        int idx;           // record index: chunk * H + head
         uint8_t *rec;
     };
+    const bool time_order = p.ready && !chunks;
     auto locate = [&](int item) {
         Item it;
-        const int cid = item / H;
-        it.h = item % H;
+        int cid;
+        if (time_order) {
+            const int per = p.nseq * H, j = item / per, r = item % per;
+            cid = (r / H) * cps + j;
+            it.h = r % H;
+        } else {
+            cid = item / H;
+            it.h = item % H;
+        }
         if (chunks) {
             it.t0 = chunks[cid].t0;
             it.len = chunks[cid].len;
@@ -234,7 +290,8 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             it.tl = j * C;
             it.b = n;
         }
-        it.rec = recs + ((size_t)cid * H + it.h) * REC_BYTES;
+        it.idx = cid * H + it.h;
+        it.rec = recs + (size_t)it.idx * REC_BYTES;
         return it;
     };
     // Input loads by the tensor-memory-access engine (one thread issues them), in four
@@ -288,19 +345,15 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if constexpr (KDA_DEBUG) {   // every item this CTA will take: a chunk of 1..C tokens
         const long long ntok = chunks ? (long long)T : (long long)(slots / max(cps, 1)) * T;
         bool bad = false;
-        for (int item = blockIdx.x + tid * gridDim.x; item < items; item += 256 * gridDim.x) {
+        for (int item = worker + tid * nworkers; item < items; item += kPrepThreads * nworkers) {
             const Item it = locate(item);
             bad |= it.len < 1 || it.len > C || it.t0 < 0 || (long long)it.t0 + it.len > ntok ||
                    item / H >= slots;
         }
-        if (__syncthreads_or(bad)) {
+        if (bar_or(bar, kPrepThreads, bad)) {
             if (tid == 0) atomicOr(err_word, ERR_BOUNDS_BIT);
             return;
         }
-    }
-    if (warp == 0) {   // 256 tensor-memory columns, reused by the three products
-        t5::alloc(tmem_slot, 2 * D);
-        t5::relinquish();
     }
     if (tid == 0) {
         mbar_init(&sm.mma_bar, 1);
@@ -317,15 +370,22 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     uint32_t mma_phase = 0;   // completions of mma_bar so far
     uint32_t ld_phase = 0;    // items whose loads have been consumed
     bool ok = true;
-    __syncthreads();          // barrier initialisation is visible to every thread
+    bar_sync(bar, kPrepThreads);   // barrier initialisation is visible to every thread
 
-    Item cur = locate(blockIdx.x);
+    Item cur = locate(worker);
     for (int grp = 0; grp < 4; ++grp) issue(grp, cur, 0);
 
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
-    const int nxt_item = item + gridDim.x;
+    for (int item = worker; item < items && ok; item += nworkers) {
+    const int nxt_item = item + nworkers;
     const bool has_next = nxt_item < items;
     uint8_t *rec = cur.rec;
+    // overlapped schedule: no more than `window` chunks ahead of this chain's state pass
+    // (the item's first global writes, in P1, come after the barrier below)
+    if (p.progress && tid == 0) {
+        const int need = cur.tl / C - p.window;
+        if (need > 0)
+            ok = progress_wait_bounded(p.progress + 2 * kProgStride * (cur.b * H + cur.h), need) && ok;
+    }
     // g, k, q (tensor loads) and beta (cp.async); V may still be in flight.  One warp
     // polls the load barriers and the CTA barrier passes the loads' completion (and
     // their data) on to the rest, instead of 256 threads polling the same words.
@@ -337,7 +397,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         pend &= ~7u;
     }
     cp_async_wait<0>();
-    ok = __syncthreads_and(ok) != 0;
+    ok = bar_and(bar, kPrepThreads, ok) != 0;
     if (!ok) break;
 
     // ---- P1: cumulative decay and the scaled operands ----
@@ -366,7 +426,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // for every r, i, and the key-key and query-key blocks are two whole 64 x 64
         // products on the tensor core.  Otherwise (decays near the -5 bound) the
         // 16-token sub-tile references are used.
-        dense = __syncthreads_and(run.x >= -0.25f * kDenseSpan && run.y >= -0.25f * kDenseSpan) != 0;
+        dense = bar_and(bar, kPrepThreads, run.x >= -0.25f * kDenseSpan && run.y >= -0.25f * kDenseSpan) != 0;
     }
     // (the barrier above: every g value is in registers; ka and xk may be overwritten)
     // pair factors exp(G_ref(a) - G_ref(b)) <= 1 for the off-diagonal sub-tile blocks
@@ -436,7 +496,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     fence_proxy_async_smem();   // the dense path's products read ka, qa, kb
     t5::fence_before_sync();
-    __syncthreads();
+    bar_sync(bar, kPrepThreads);
 
     // ---- P2: key-key and query-key blocks ----
     // (I + A_aa)^-1 of diagonal sub-tile blocks: lane -> (block a0 + lane/16, column j)
@@ -460,7 +520,6 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // memory columns 0-63 and 64-127; then every thread takes its rows of one block
         // (warps 0-3: A_kk, 4-7: A_qk) to the masked, beta-scaled forms the
         // substitution and the record products use.
-        const uint32_t tmem = *tmem_slot;
         if (warp == 0) {
             if (t5::elect_one()) {
                 t5::fence_after_sync();
@@ -599,7 +658,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
     }
     }
-    __syncthreads();
+    bar_sync(bar, kPrepThreads);
 
     // ---- P3: T' = (I + A)^-1 Diag(b) by blocked forward substitution, transposed ----
     // (I + A) T' = Diag(b), solved per 16-row block a:
@@ -670,8 +729,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         else pend &= ~8u;
         fence_proxy_async_smem();   // T' (generic stores) -> tensor core
         t5::fence_before_sync();
-        ok = __syncthreads_and(ok) != 0;
-        const uint32_t tmem = *tmem_slot;
+        ok = bar_and(bar, kPrepThreads, ok) != 0;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         if (ok && warp == 0) {
             if (t5::elect_one()) {
@@ -720,7 +778,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         cp_async_wait<0>();         // Kt and Qg
         fence_proxy_async_smem();   // [W|U] (generic stores), Kt (cp.async) -> tensor core
         t5::fence_before_sync();
-        ok = __syncthreads_and(ok) != 0;
+        ok = bar_and(bar, kPrepThreads, ok) != 0;
         const uint64_t ydesc = t5::smem_desc(s_qa, C * 128, 1024, t5::kSwz128);   // [W|U], N-major
         if (ok && warp == 0) {
             if (t5::elect_one()) {
@@ -759,7 +817,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
         }
         t5::fence_before_sync();
-        ok = __syncthreads_and(ok) != 0;
+        ok = bar_and(bar, kPrepThreads, ok) != 0;
         if (ok && warp == 0) {
             if (t5::elect_one()) {
                 t5::fence_after_sync();
@@ -801,9 +859,18 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
             }
         }
+        // the record's generic stores, ordered before the state pass's bulk copies of it
+        if (p.ready) fence_proxy_async_global();
         t5::fence_before_sync();
-        ok = __syncthreads_and(ok) != 0;   // Qg in xv is consumed
+        ok = bar_and(bar, kPrepThreads, ok) != 0;   // Qg in xv is consumed; the record is whole
         t5::fence_after_sync();
+        // publish the record (the barrier ordered every thread's stores before this
+        // thread's release); not thread 0, which issues the loads: its fence would wait
+        // for them
+        if (p.ready && ok && tid == 32) {
+            __threadfence();
+            flag_release(p.ready + cur.idx, 1);
+        }
         if (has_next) issue(3, nxt, ld_phase + 1);
     }
     cur = nxt;
@@ -816,10 +883,29 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     for (int grp = 0; grp < 4; ++grp)
         if (pend & (1u << grp)) wait_ld(grp);
     cp_async_wait<0>();
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 2)
+kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                   const PrepArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment: the swizzled operand tiles are read by the tensor core
+    PrepSmem &sm = *reinterpret_cast<PrepSmem *>(
+        smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    if (threadIdx.x < 32) {   // 2D tensor-memory columns, reused by the three products
+        t5::alloc(&sm.tmem_slot, 2 * D);
+        t5::relinquish();
+    }
     t5::fence_before_sync();
     __syncthreads();
     t5::fence_after_sync();
-    if (warp == 0) t5::dealloc(*tmem_slot, 2 * D);
+    prep_worker(tm_q, tm_k, tm_v, tm_g, p, sm, sm.tmem_slot, threadIdx.x, 0, blockIdx.x,
+                gridDim.x);
+    t5::fence_before_sync();
+    __syncthreads();
+    t5::fence_after_sync();
+    if (threadIdx.x < 32) t5::dealloc(sm.tmem_slot, 2 * D);
 }
 
 // ---------------------------------------------------------------------------
@@ -882,6 +968,11 @@ struct StateArgs {
     // extents for the debug bounds checks: tokens in o (all sequences) and chunk slots
     long long ntok;
     int max_chunks;
+    // overlapped schedule: the prep's per-record ready flags (chunk * H + head), waited
+    // for before each record is copied in; null when the records are all written
+    const int *ready;
+    // overlapped schedule: this CTA's count of chunks whose copies have started
+    int *progress;
 };
 template <int DVT>
 struct T5Layout {
@@ -928,8 +1019,10 @@ struct StateRoles {
     static constexpr int THREADS = 32 * (NSW + 6);
 };
 
+// One state-pass CTA: `cta` indexes (unit, column tile), column tile fastest.  Warps
+// past the roles (when the block is larger) only take part in the CTA barriers.
 template <int DVT>
-__global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kernel(const StateArgs a) {
+KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
     using L = T5Layout<DVT>;
     using RL = StateRoles<DVT>;
     const uint8_t *__restrict__ recs = a.recs;
@@ -950,11 +1043,13 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 4);
     int *cnt = reinterpret_cast<int *>(sm + L::OFF_MISC + 8);   // [0] ring A issued, [1] ring B issued, [2] MMA issued
+    // overlapped schedule: records known to be published, [0, *rdy) (the poller warp's count)
+    volatile int *rdy = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 20);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // 1-D grid, column tile fastest so the tiles of one unit run side by side
     // and share the chunk records through L2.
     const int tiles = (map_mode ? 2 * D : D) / DVT;
-    const int tile = blockIdx.x % tiles, unit = blockIdx.x / tiles;
+    const int tile = cta % tiles, unit = cta / tiles;
     const int chain = unit / a.nseg, seg = unit % a.nseg, n = chain / H, h = chain % H;
     const bool p_half = map_mode && tile >= D / DVT;   // linear part of the map: no R
     const int col0 = (tile % (D / DVT)) * DVT;
@@ -1005,6 +1100,7 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
         mbar_init(&do_free[1], 128);
         *abort_flag = 0;
         cnt[0] = cnt[1] = cnt[2] = 0;
+        *rdy = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -1234,12 +1330,39 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
             }
             mbar_arrive(&b_free[sbb]);
         }
-    } else {
+    } else if (warp == RL::PROD_WARP + 1) {
+        // ---------------- poller (overlapped schedule only; the fused block's spare warp) ----------------
+        // walks the chain's records in order, waiting (acquire, GPU scope) for each ready
+        // flag the prep sets, and counts the published ones in shared memory, so the
+        // producer's copies never wait on a global-memory round trip
+        if (a.ready && lane == 0) {
+            for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+                if (!flag_wait_bounded(a.ready + (size_t)(c_begin + c) * H + h)) { fail(); break; }
+                __threadfence_block();   // the acquired state first, then the count (CTA scope)
+                *rdy = c + 1;
+            }
+        }
+        __syncwarp();
+    } else if (warp == RL::PROD_WARP) {
         // ---------------- producer warp: lane 0 feeds ring A, lane 1 ring B ----------------
+        // overlapped schedule: a record is copied in only once the poller has seen it published
+        auto ready = [&](int c) {
+            if (!a.ready) return true;
+            if (*rdy <= c) {
+                const uint64_t t0 = global_timer_ns();
+                while (*rdy <= c) {
+                    if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) return false;
+                }
+            }
+            __threadfence_block();
+            fence_proxy_async_global();   // the prep's generic stores -> these bulk copies
+            return true;
+        };
         if (lane == 0) {
             for (int c = 0; c < nchunks && !*abort_flag; ++c) {
                 const int s = c % NA;
                 if (c >= NA && !mbar_wait_bounded(&a_free[s], ((c - NA) / NA) & 1)) { fail(); break; }
+                if (!ready(c)) { fail(); break; }
                 fence_proxy_async_smem();
                 uint64_t *bar = &full_a[s];
                 uint8_t *dst = sm + s * L::A_BYTES;
@@ -1251,11 +1374,15 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
                 bulk_g2s(dst + L::A_GC, rec + REC_GC, D * 4, bar);
                 if (!p_half)
                     bulk_g2s(dst + L::A_R, rec + REC_R + core_off(D, 0, col0), L::R_BYTES, bar);
+                // a hint for the prep's throttle: a relaxed store, no fence (a release
+                // here would hold this lane until its earlier copies are done)
+                if (a.progress) store_relaxed(a.progress + kProgStride * cta, c + 1);
             }
         } else if (lane == 1) {
             for (int c = 0; c < (map_mode ? 0 : nchunks) && !*abort_flag; ++c) {
                 const int s = c % NB;
                 if (c >= NB && !mbar_wait_bounded(&b_free[s], ((c - NB) / NB) & 1)) { fail(); break; }
+                if (!ready(c)) { fail(); break; }
                 fence_proxy_async_smem();
                 uint64_t *bar = &full_b[s];
                 uint8_t *dst = sm + L::OFF_B + s * L::B_BYTES;
@@ -1287,6 +1414,60 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
     __syncthreads();
     t5::fence_after_sync();
     if (warp == 0) t5::dealloc(tmem, L::TMEM_COLS);
+}
+
+template <int DVT>
+__global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kernel(const StateArgs a) {
+    state_cta<DVT>(a, blockIdx.x);
+}
+
+// ---------------------------------------------------------------------------
+// Overlapped schedule: kernels 1 and 2 as one launch (fixed-length input).
+// The first `nstate` CTAs run the state pass on 64-column slices (one per SM), the
+// others each run two prep workers (the two CTAs of kernel 1's usual two per SM, as
+// one block, with their own shared memory, tensor-memory columns and named barriers)
+// over the records in time order.  A state CTA waits for a record's ready flag
+// before copying it in, so the state chain starts after the first records instead
+// of after all of them, and the prep runs on the SMs the chain leaves idle.  The
+// wait is one-way (the prep never waits for the state pass) and bounded, and the
+// grid is one block per SM, launched cooperatively so all blocks are resident.
+// ---------------------------------------------------------------------------
+constexpr int kFusedThreads = 2 * kPrepThreads;
+constexpr int kFusedPrepStride = (int)((sizeof(PrepSmem) + 1023) / 1024 * 1024);
+constexpr int kFusedSmem = (2 * kFusedPrepStride + 1024 > T5Layout<64>::BYTES)
+                               ? 2 * kFusedPrepStride + 1024 : T5Layout<64>::BYTES;
+// the state roles and the ready-flag poller (one more warp) fit the fused block
+static_assert(StateRoles<64>::THREADS + 32 <= kFusedThreads, "state roles fit the fused block");
+static_assert(kFusedSmem <= 232448, "shared memory budget");
+
+__global__ void __launch_bounds__(kFusedThreads, 1)
+kda_tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                    const PrepArgs p, const StateArgs a, const int nstate) {
+    if ((int)blockIdx.x < nstate) {
+        state_cta<64>(a, blockIdx.x);
+        return;
+    }
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    PrepSmem &s0 = *reinterpret_cast<PrepSmem *>(base);
+    const int w = threadIdx.x / kPrepThreads;
+    PrepSmem &sm = *reinterpret_cast<PrepSmem *>(base + w * kFusedPrepStride);
+    if (threadIdx.x < 32) {   // both workers' columns at once: one allocation per CTA
+        t5::alloc(&s0.tmem_slot, 4 * D);
+        t5::relinquish();
+    }
+    t5::fence_before_sync();
+    __syncthreads();
+    t5::fence_after_sync();
+    const uint32_t tmem = s0.tmem_slot + (uint32_t)(w * 2 * D);
+    const int nprep = 2 * ((int)gridDim.x - nstate);
+    prep_worker(tm_q, tm_k, tm_v, tm_g, p, sm, tmem, threadIdx.x % kPrepThreads, 1 + w,
+                2 * ((int)blockIdx.x - nstate) + w, nprep);
+    t5::fence_before_sync();
+    __syncthreads();
+    t5::fence_after_sync();
+    if (threadIdx.x < 32) t5::dealloc(s0.tmem_slot, 4 * D);
 }
 
 // ---------------------------------------------------------------------------

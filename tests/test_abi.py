@@ -56,10 +56,11 @@ def test_version_and_status_strings(lib):
 
 def test_workspace_size(lib):
     ws = lib.kda_fwd_workspace_size
-    # tensor-core path stores one 98,816-byte record per (64-token chunk, head)
+    # tensor-core path stores one 98,816-byte record and one 4-byte ready flag (the
+    # overlapped schedule's) per (64-token chunk, head)
     a = ws(2, 4096, 8, 128, 128, 0, BF16)
     b = ws(2, 4096 + 64, 8, 128, 128, 0, BF16)
-    assert b - a == 2 * 8 * 98816
+    assert b - a == 2 * 8 * (98816 + 4)
     assert ws(1, 100, 4, 128, 128, 3, BF16) > 0          # packed varlen
     assert ws(2, 100, 4, 128, 128, 3, BF16) == 0         # packed needs B == 1
     assert ws(1, 64, 4, 128, 64, 0, BF16) == 0           # d_k != d_v
@@ -74,6 +75,30 @@ def test_plan_segments_validates(lib):
     assert plan(2, 4096, 8, 64, 64, 0, F32) == 1           # CUDA-core path never splits
     assert plan(2, 100, 4, 128, 64, 0, BF16) == 0          # d_k != d_v
     assert plan(2, 100, 4, 128, 128, 3, BF16) == 0         # packed needs B == 1
+
+
+def test_plan_overlap_and_overlapped_validation(lib):
+    plan = lib.kda_fwd_plan_overlap
+    assert plan(2, 4096, 8, 128, 128, 0, BF16) == 0       # no device here
+    assert plan(1, 4096, 8, 128, 128, 3, BF16) == 0       # packed input: never
+    assert plan(2, 4096, 8, 64, 64, 0, F32) == 0          # CUDA-core path: never
+    ov = lib.kda_fwd_overlapped
+    p = 0x10000
+
+    def call(**over):
+        a = dict(q=p, k=p, v=p, g=p, beta=p, h0=None, B=2, T=128, H=2, dk=128, dv=128,
+                 dtype=BF16, o=p + 0x100000, hT=None, work=p, ws=1 << 40, stream=None)
+        a.update(over)
+        return ov(a["q"], a["k"], a["v"], a["g"], a["beta"], a["h0"], a["B"], a["T"], a["H"],
+                  a["dk"], a["dv"], a["dtype"], a["o"], a["hT"], a["work"], a["ws"],
+                  a["stream"])
+    assert call(dk=64, dv=64) == UNSUPPORTED              # tensor-core path only
+    assert call(dtype=F32) == UNSUPPORTED
+    assert call(q=None) == INVALID
+    assert call(B=-1) == INVALID
+    assert call(q=p + 2) == MISALIGNED
+    assert call(ws=1000) == WS_SMALL
+    assert call() == 5                                    # KDA_ERR_CUDA: no device here
 
 
 def test_segmented_workspace_size(lib):

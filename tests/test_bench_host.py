@@ -13,10 +13,11 @@ BF16 = torch.bfloat16
 
 
 def test_record_bytes_match_the_library_workspace():
-    # one more chunk per sequence adds one record per (sequence, head)
+    # one more chunk per sequence adds one record and one 4-byte ready flag per
+    # (sequence, head)
     grow = kda.workspace_size(2, 4096 + 64, 8, 128, 128, 0, BF16) - \
         kda.workspace_size(2, 4096, 8, 128, 128, 0, BF16)
-    assert grow == 2 * 8 * bench.record_bytes()
+    assert grow == 2 * 8 * (bench.record_bytes() + 4)
 
 
 def _tree(root, code):
