@@ -250,8 +250,10 @@ def _input_bytes(inp):
 
 
 def measure_prefill(name, steps, warmup, world=1, rank=0, local=0, e2e=True, cpu=True,
-                    cpu_seconds=10.0, ckpt_every=0):
-    """Time `steps` kda_fwd calls on workload `name`; returns the JSON object (rank 0)."""
+                    cpu_seconds=10.0, ckpt_every=0, two_launch=False):
+    """Time `steps` kda_fwd calls on workload `name`; returns the JSON object (rank 0).
+    two_launch: time kda_fwd_segmented with one segment instead (the prep kernel, then
+    the state pass) whatever schedule kda_fwd would pick."""
     import torch
     import kimi_delta_attention_28_b200 as kda
     dev = torch.device("cuda", local)
@@ -283,6 +285,9 @@ def measure_prefill(name, steps, warmup, world=1, rank=0, local=0, e2e=True, cpu
             kda.kda_fwd_checkpointed(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
                                      inp["h0"], cu, ckpt_every=ckpt_every, ckpts=ck, o=o,
                                      hT=hT, workspace=ws)
+        elif two_launch:
+            kda.kda_fwd_segmented(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                  inp["h0"], cu, num_segments=1, o=o, hT=hT, workspace=ws)
         else:
             kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], cu, o=o,
                         hT=hT, workspace=ws)
@@ -335,7 +340,9 @@ def measure_prefill(name, steps, warmup, world=1, rank=0, local=0, e2e=True, cpu
     inter_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in split)
     nseg = kda.plan_segments(B, T, H, dk, dv, nseq, w.dtype)
     # kda_fwd's schedule: one overlapped launch, or the prep kernel then the state pass
-    overlap = kda.plan_overlap(B, T, H, dk, dv, nseq, w.dtype)
+    overlap = kda.plan_overlap(B, T, H, dk, dv, nseq, w.dtype) and not two_launch
+    if two_launch:
+        nseg = 1
     launches_per_step = 1 if overlap else (2 if cu is not None else 1) + (1 if nseg <= 1 else 3)
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / steps
@@ -421,6 +428,9 @@ def measure_prefill(name, steps, warmup, world=1, rank=0, local=0, e2e=True, cpu
         "clocks": clocks.summary(t_wall0, t_wall1),
         "e2e": e2e_obj,
     }
+    out["config"]["schedule"] = ("one overlapped launch (kda_tc_fused_kernel)" if overlap else
+                                 "two launches (prep kernel, then state pass)" +
+                                 (" (forced)" if two_launch else ""))
     if ck is not None:
         out["config"]["ckpt_every"] = ckpt_every
         out["config"]["checkpoints_per_head"] = int(ck.shape[0])
@@ -787,7 +797,9 @@ def measure_speculative(steps, warmup, K=4, cpu=True):
                    "H": w.H, "K": K, "accepted": "uniform in [0, K] per sequence (seeded)"},
         "roofline": {"bound": "hbm", "kernel": "kda_decode_multi_kernel (verify + commit)",
                      "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
-                     "traffic": None, "algorithmic_bytes_per_launch": bytes_step / 2,
+                     # mean DRAM bytes of a verify and a commit launch (ncu capture)
+                     "traffic": load_traffic("kda_decode_multi_kernel", units),
+                     "algorithmic_bytes_per_launch": bytes_step / 2,
                      "algorithmic_bytes_rule": "per (sequence, head): state read (verify) + read "
                                                "and write (commit), drafted inputs and outputs",
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)"},
@@ -855,7 +867,8 @@ def measure_backward(name, steps, warmup, cpu=True, cpu_seconds=10.0):
            "warmup": warmup, "config": prefill_config(w, inp, 1),
            "roofline": {"bound": "alu", "kernel": "kda_bwd_slice_kernel",
                         "achieved": tf, "peak": peak_fp32, "unit": "TFLOP/s",
-                        "frac": tf / peak_fp32, "traffic": None,
+                        "frac": tf / peak_fp32,
+                        "traffic": load_traffic("kda_bwd_slice_kernel", units),
                         "algorithmic_flops_per_launch": flops,
                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz "
                                        "(CUDA-core fp32, nominal clock)",
@@ -1022,6 +1035,9 @@ def main():
     ap.add_argument("--ckpt-every", type=int, default=0,
                     help="prefill workloads: also store the state every N tokens (multiple of 64)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--two-launch", action="store_true",
+                    help="prefill workloads: time the two-launch schedule (prep kernel, then "
+                         "state pass) even where kda_fwd would overlap them in one launch")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     args = ap.parse_args()
@@ -1052,7 +1068,7 @@ def main():
         else:
             out = measure_prefill(args.workload, args.steps, args.warmup, world, rank, local,
                                   e2e=not args.no_e2e, cpu=cpu, cpu_seconds=args.cpu_seconds,
-                                  ckpt_every=args.ckpt_every)
+                                  ckpt_every=args.ckpt_every, two_launch=args.two_launch)
         if world == 1 and not args.no_nested and args.workload == HEADLINE and out is not None:
             # the other workloads, each with its own roofline and parity sample
             nested = {}
