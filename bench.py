@@ -200,13 +200,14 @@ def _strip_comments(text):
 
 
 def kernel_source_sha(src=None):
-    """sha256 over the CUDA sources of the library with comments removed (identifies
-    the kernel code; an edit of comments alone keeps it)."""
+    """sha256 over the device-code headers of the library (csrc/*.cuh, where every
+    kernel lives) with comments removed: it identifies the kernel code.  An edit of
+    comments alone, or of the host-side launch and policy code (csrc/*.cu), keeps it."""
     import hashlib
     src = src or os.path.join(ROOT, "kimi_delta_attention_28_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(src)):
-        if f.endswith((".cu", ".cuh")):
+        if f.endswith(".cuh"):
             with open(os.path.join(src, f), encoding="utf-8") as fh:
                 h.update(f.encode() + b"\0" + _strip_comments(fh.read()).encode())
     return h.hexdigest()

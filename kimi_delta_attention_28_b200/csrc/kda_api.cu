@@ -517,11 +517,14 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
 //     the 32-column state pass takes 0.79 us per chunk per wave of 4 CTAs per chain;
 //   one launch: a prep item takes 14.5 us (it shares the GPU with the state pass), a
 //     64-column chunk 1.19 us, and the chain starts about 5 us after the launch.
-// (B=1, H=16, T=1M: 19.7 against 23.8 ms; B=2, H=8, T=4,096: 0.139 against 0.140 ms.)
+// Below 128 chunks per chain the two were measured equal or the single launch slower
+// (B=2, H=8, T=4,096: 0.110 against 0.107 ms), so the single launch needs at least that
+// many (B=1, H=16, T=16,384: 0.380 against 0.416 ms; T=1M: 19.5 against 23.8 ms).
 constexpr double kPrepUsTwo = 12.2, kState32Us = 0.79;
 constexpr double kPrepUsOne = 14.5, kState64OneUs = 1.19, kRampUs = 5.0;
+constexpr long long kMinOverlapChunks = 128;
 static bool overlap_schedule(long long chains, long long cps, int sms) {
-    if (chains <= 0 || cps <= 0 || sms <= 0) return false;
+    if (chains <= 0 || cps < kMinOverlapChunks || sms <= 0) return false;
     const long long nstate = 2 * chains;
     if (nstate > sms / 2) return false;
     const double c = (double)chains, n = (double)cps;

@@ -20,10 +20,10 @@ def test_record_bytes_match_the_library_workspace():
     assert grow == 2 * 8 * (bench.record_bytes() + 4)
 
 
-def _tree(root, code):
+def _tree(root, code, name="k.cuh"):
     src = os.path.join(root, "kimi_delta_attention_28_b200", "csrc")
     os.makedirs(src, exist_ok=True)
-    with open(os.path.join(src, "k.cu"), "w") as f:
+    with open(os.path.join(src, name), "w") as f:
         f.write(code)
     return src
 
@@ -42,7 +42,10 @@ def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monk
     _tree(root, "/* the same kernel */\n__global__ void k(int *p) { p[0] = 1; }  // store\n")
     assert bench.kernel_source_sha() == sha
     assert bench.load_traffic("prep", 2) == 3.0
-    # ... a code edit drops it
+    # ... so does host-side code (launch policy) beside the kernels ...
+    _tree(root, "int policy() { return 2; }\n", name="api.cu")
+    assert bench.kernel_source_sha() == sha
+    # ... a kernel code edit drops it
     _tree(root, "__global__ void k(int *p) { p[0] = 2; }\n")
     assert bench.kernel_source_sha() != sha
     assert bench.load_traffic("prep", 2) is None

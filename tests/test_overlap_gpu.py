@@ -90,9 +90,10 @@ def test_policy_and_kda_fwd_dispatch():
     assert not kda.plan_overlap(2, 4096, 8, 64, 64, 0, torch.float32)
     if sms < 128:
         pytest.skip("policy thresholds are for B200-sized GPUs")
-    assert kda.plan_overlap(2, 4096, 8, 128, 128, 0, bf)
+    assert not kda.plan_overlap(2, 4096, 8, 128, 128, 0, bf)      # 64 chunks: too short
+    assert kda.plan_overlap(2, 8192, 8, 128, 128, 0, bf)
     assert kda.plan_overlap(1, 1 << 20, 16, 128, 128, 0, bf)
-    inp = W.make_prefill_inputs(2, 4096, 8, 128, 128, bf, True, seed=131, device=DEV)
+    inp = W.make_prefill_inputs(2, 8192, 8, 128, 128, bf, True, seed=131, device=DEV)
     a = kda.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
     b = kda.kda_fwd_overlapped(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
     c = kda.kda_fwd_overlapped(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
@@ -110,7 +111,7 @@ def test_checkpoints_on_the_overlapped_schedule():
     """kda_fwd_checkpointed where kda_fwd overlaps: o and hT equal kda_fwd's, and
     every stored state matches the oracle's state after that prefix."""
     bf = torch.bfloat16
-    B, T, H, every = 2, 4096, 8, 1024
+    B, T, H, every = 2, 8192, 8, 2048
     if not kda.plan_overlap(B, T, H, 128, 128, 0, bf):
         pytest.skip("kda_fwd does not overlap at these sizes on this GPU")
     inp = W.make_prefill_inputs(B, T, H, 128, 128, bf, True, seed=132, device=DEV)
