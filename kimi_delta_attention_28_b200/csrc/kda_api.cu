@@ -574,6 +574,7 @@ static kda_status tc_fused(const void *q, const void *k, const void *v, const fl
     p.err_word = err;
     p.ready = ready;
     p.nseq = N;
+    p.nstate = (int)nstate;
     p.progress = prog;
     // records in flight between the roles: about 48 MiB, well inside L2
     const long long win = (48LL << 20) / (chains * (long long)REC_BYTES);

@@ -209,6 +209,7 @@ struct PrepArgs {
     // the record is complete.  Null: items in sequence order, no flags.
     int *ready;
     int nseq;
+    int nstate;   // overlapped schedule: state blocks before the prep blocks
     // Overlapped schedule: chunks each state CTA has started copying in (2 CTAs per
     // chain, column tile fastest); a worker starts the item of chunk j of a chain only
     // once both of the chain's CTAs have reached chunk j - window, so the records in
@@ -240,13 +241,38 @@ KDA_DEVINL bool progress_wait_bounded(const int *prog2, int need) {
     return true;
 }
 
-// One prep worker: `kPrepThreads` threads (tid 0..255) with their own PrepSmem, the
-// 2D tensor-memory columns at `tmem` (allocated by the caller) and named barrier
-// `bar`, walking items worker, worker + nworkers, ...
+// One prep worker: `kPrepThreads` threads with their own PrepSmem, whose tmem_slot
+// holds the worker's 2D tensor-memory columns (allocated by the caller), walking
+// items worker, worker + nworkers, ...
+// OVERLAP = false: the standalone kernel, one worker per block (barrier 0).
+// OVERLAP = true: two workers per block of the fused kernel after its p.nstate state
+// blocks (worker w = threadIdx.x / 256 on named barrier 1 + w), with the overlapped
+// schedule's item order, flags and window.  The indices are derived from the special
+// registers where they are used rather than held in registers through the item loop
+// (the standalone kernel's register budget is exactly full).
+template <bool OVERLAP>
 KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                             const CUtensorMap &tm_v, const CUtensorMap &tm_g, const PrepArgs &p,
-                            PrepSmem &sm, const uint32_t tmem, const int tid, const int bar,
-                            const int worker, const int nworkers) {
+                            PrepSmem &sm) {
+    const int tid = OVERLAP ? (int)(threadIdx.x % kPrepThreads) : (int)threadIdx.x;
+    const int bar = OVERLAP ? 1 + (int)(threadIdx.x / kPrepThreads) : 0;
+    const int worker = OVERLAP ? 2 * ((int)blockIdx.x - p.nstate) + (int)(threadIdx.x / kPrepThreads)
+                               : (int)blockIdx.x;
+    const int nworkers = OVERLAP ? 2 * ((int)gridDim.x - p.nstate) : (int)gridDim.x;
+    // the worker's barriers: the block's own (barrier 0, immediate forms) when it is
+    // alone in its block, else its named barrier
+    auto cta_sync = [&]() {
+        if constexpr (OVERLAP) bar_sync(bar, kPrepThreads);
+        else __syncthreads();
+    };
+    auto cta_and = [&](bool x) {
+        if constexpr (OVERLAP) return bar_and(bar, kPrepThreads, x);
+        else return __syncthreads_and(x) != 0;
+    };
+    auto cta_or = [&](bool x) {
+        if constexpr (OVERLAP) return bar_or(bar, kPrepThreads, x);
+        else return __syncthreads_or(x) != 0;
+    };
     const float *__restrict__ beta = p.beta;
     const int T = p.T, H = p.H, cps = p.cps, slots = p.slots;
     const int *__restrict__ hdr = p.hdr;
@@ -266,7 +292,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
         int idx;           // record index: chunk * H + head
         uint8_t *rec;
     };
-    const bool time_order = p.ready && !chunks;
+    const bool time_order = OVERLAP && !chunks;
     auto locate = [&](int item) {
         Item it;
         int cid;
@@ -350,7 +376,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
             bad |= it.len < 1 || it.len > C || it.t0 < 0 || (long long)it.t0 + it.len > ntok ||
                    item / H >= slots;
         }
-        if (bar_or(bar, kPrepThreads, bad)) {
+        if (cta_or(bad)) {
             if (tid == 0) atomicOr(err_word, ERR_BOUNDS_BIT);
             return;
         }
@@ -370,7 +396,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
     uint32_t mma_phase = 0;   // completions of mma_bar so far
     uint32_t ld_phase = 0;    // items whose loads have been consumed
     bool ok = true;
-    bar_sync(bar, kPrepThreads);   // barrier initialisation is visible to every thread
+    cta_sync();   // barrier initialisation is visible to every thread
 
     Item cur = locate(worker);
     for (int grp = 0; grp < 4; ++grp) issue(grp, cur, 0);
@@ -381,7 +407,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
     uint8_t *rec = cur.rec;
     // overlapped schedule: no more than `window` chunks ahead of this chain's state pass
     // (the item's first global writes, in P1, come after the barrier below)
-    if (p.progress && tid == 0) {
+    if (OVERLAP && p.progress && tid == 0) {
         const int need = cur.tl / C - p.window;
         if (need > 0)
             ok = progress_wait_bounded(p.progress + 2 * kProgStride * (cur.b * H + cur.h), need) && ok;
@@ -397,7 +423,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
         pend &= ~7u;
     }
     cp_async_wait<0>();
-    ok = bar_and(bar, kPrepThreads, ok) != 0;
+    ok = cta_and(ok) != 0;
     if (!ok) break;
 
     // ---- P1: cumulative decay and the scaled operands ----
@@ -426,7 +452,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
         // for every r, i, and the key-key and query-key blocks are two whole 64 x 64
         // products on the tensor core.  Otherwise (decays near the -5 bound) the
         // 16-token sub-tile references are used.
-        dense = bar_and(bar, kPrepThreads, run.x >= -0.25f * kDenseSpan && run.y >= -0.25f * kDenseSpan) != 0;
+        dense = cta_and(run.x >= -0.25f * kDenseSpan && run.y >= -0.25f * kDenseSpan) != 0;
     }
     // (the barrier above: every g value is in registers; ka and xk may be overwritten)
     // pair factors exp(G_ref(a) - G_ref(b)) <= 1 for the off-diagonal sub-tile blocks
@@ -496,7 +522,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
     }
     fence_proxy_async_smem();   // the dense path's products read ka, qa, kb
     t5::fence_before_sync();
-    bar_sync(bar, kPrepThreads);
+    cta_sync();
 
     // ---- P2: key-key and query-key blocks ----
     // (I + A_aa)^-1 of diagonal sub-tile blocks: lane -> (block a0 + lane/16, column j)
@@ -515,6 +541,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
         for (int r = 0; r < ST; ++r) sm.taa[a][r * (ST + 8) + j] = f2bf(x[r]);
     };
     if (dense) {
+        const uint32_t tmem = sm.tmem_slot;
         // Two tcgen05 products with the row-31 reference: A_kk = Kl Kr^T and
         // A_qk = Ql Kr^T (M = 64, N = 64, K = 128; ka, qa, kb all K-major), into tensor
         // memory columns 0-63 and 64-127; then every thread takes its rows of one block
@@ -658,7 +685,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                 }
     }
     }
-    bar_sync(bar, kPrepThreads);
+    cta_sync();
 
     // ---- P3: T' = (I + A)^-1 Diag(b) by blocked forward substitution, transposed ----
     // (I + A) T' = Diag(b), solved per 16-row block a:
@@ -725,11 +752,12 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
     //   D1 = Kt^T [W|U]        (M = 128 key rows):         M' = -D1[:, :128], R = D1[:, 128:]
     //   D2 = Aqk  [W|U]        (M = 64 chunk rows):        Q' = Qg - D2[:, :128], O0 = D2[:, 128:]
     {
+        const uint32_t tmem = sm.tmem_slot;
         if (warp == 0) ok = wait_ld(3) && ok;   // V (read by the tensor core only)
         else pend &= ~8u;
         fence_proxy_async_smem();   // T' (generic stores) -> tensor core
         t5::fence_before_sync();
-        ok = bar_and(bar, kPrepThreads, ok) != 0;
+        ok = cta_and(ok) != 0;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         if (ok && warp == 0) {
             if (t5::elect_one()) {
@@ -778,7 +806,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
         cp_async_wait<0>();         // Kt and Qg
         fence_proxy_async_smem();   // [W|U] (generic stores), Kt (cp.async) -> tensor core
         t5::fence_before_sync();
-        ok = bar_and(bar, kPrepThreads, ok) != 0;
+        ok = cta_and(ok) != 0;
         const uint64_t ydesc = t5::smem_desc(s_qa, C * 128, 1024, t5::kSwz128);   // [W|U], N-major
         if (ok && warp == 0) {
             if (t5::elect_one()) {
@@ -817,7 +845,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
             }
         }
         t5::fence_before_sync();
-        ok = bar_and(bar, kPrepThreads, ok) != 0;
+        ok = cta_and(ok) != 0;
         if (ok && warp == 0) {
             if (t5::elect_one()) {
                 t5::fence_after_sync();
@@ -860,14 +888,14 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
             }
         }
         // the record's generic stores, ordered before the state pass's bulk copies of it
-        if (p.ready) fence_proxy_async_global();
+        if (OVERLAP) fence_proxy_async_global();
         t5::fence_before_sync();
-        ok = bar_and(bar, kPrepThreads, ok) != 0;   // Qg in xv is consumed; the record is whole
+        ok = cta_and(ok) != 0;   // Qg in xv is consumed; the record is whole
         t5::fence_after_sync();
         // publish the record (the barrier ordered every thread's stores before this
         // thread's release); not thread 0, which issues the loads: its fence would wait
         // for them
-        if (p.ready && ok && tid == 32) {
+        if (OVERLAP && ok && tid == 32) {
             __threadfence();
             flag_release(p.ready + cur.idx, 1);
         }
@@ -888,7 +916,7 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
 __global__ void __launch_bounds__(kPrepThreads, 2)
 kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                   const PrepArgs p) {
+                   const __grid_constant__ PrepArgs p) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment: the swizzled operand tiles are read by the tensor core
     PrepSmem &sm = *reinterpret_cast<PrepSmem *>(
@@ -900,8 +928,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     t5::fence_before_sync();
     __syncthreads();
     t5::fence_after_sync();
-    prep_worker(tm_q, tm_k, tm_v, tm_g, p, sm, sm.tmem_slot, threadIdx.x, 0, blockIdx.x,
-                gridDim.x);
+    prep_worker<false>(tm_q, tm_k, tm_v, tm_g, p, sm);
     t5::fence_before_sync();
     __syncthreads();
     t5::fence_after_sync();
@@ -1021,7 +1048,10 @@ struct StateRoles {
 
 // One state-pass CTA: `cta` indexes (unit, column tile), column tile fastest.  Warps
 // past the roles (when the block is larger) only take part in the CTA barriers.
-template <int DVT>
+// OVERLAP: the poller warp, the wait for published records and the progress counter
+// of the overlapped schedule (compiled out of the standalone kernel: their mere
+// presence in the producer's loop cost it 13% in time).
+template <int DVT, bool OVERLAP>
 KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
     using L = T5Layout<DVT>;
     using RL = StateRoles<DVT>;
@@ -1330,12 +1360,12 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
             }
             mbar_arrive(&b_free[sbb]);
         }
-    } else if (warp == RL::PROD_WARP + 1) {
+    } else if (OVERLAP && warp == RL::PROD_WARP + 1) {
         // ---------------- poller (overlapped schedule only; the fused block's spare warp) ----------------
         // walks the chain's records in order, waiting (acquire, GPU scope) for each ready
         // flag the prep sets, and counts the published ones in shared memory, so the
         // producer's copies never wait on a global-memory round trip
-        if (a.ready && lane == 0) {
+        if (lane == 0) {
             for (int c = 0; c < nchunks && !*abort_flag; ++c) {
                 if (!flag_wait_bounded(a.ready + (size_t)(c_begin + c) * H + h)) { fail(); break; }
                 __threadfence_block();   // the acquired state first, then the count (CTA scope)
@@ -1347,7 +1377,7 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
         // ---------------- producer warp: lane 0 feeds ring A, lane 1 ring B ----------------
         // overlapped schedule: a record is copied in only once the poller has seen it published
         auto ready = [&](int c) {
-            if (!a.ready) return true;
+            if constexpr (!OVERLAP) return true;
             if (*rdy <= c) {
                 const uint64_t t0 = global_timer_ns();
                 while (*rdy <= c) {
@@ -1376,7 +1406,7 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
                     bulk_g2s(dst + L::A_R, rec + REC_R + core_off(D, 0, col0), L::R_BYTES, bar);
                 // a hint for the prep's throttle: a relaxed store, no fence (a release
                 // here would hold this lane until its earlier copies are done)
-                if (a.progress) store_relaxed(a.progress + kProgStride * cta, c + 1);
+                if constexpr (OVERLAP) store_relaxed(a.progress + kProgStride * cta, c + 1);
             }
         } else if (lane == 1) {
             for (int c = 0; c < (map_mode ? 0 : nchunks) && !*abort_flag; ++c) {
@@ -1417,8 +1447,8 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
 }
 
 template <int DVT>
-__global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kernel(const StateArgs a) {
-    state_cta<DVT>(a, blockIdx.x);
+__global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kernel(const __grid_constant__ StateArgs a) {
+    state_cta<DVT, false>(a, blockIdx.x);
 }
 
 // ---------------------------------------------------------------------------
@@ -1443,9 +1473,10 @@ static_assert(kFusedSmem <= 232448, "shared memory budget");
 __global__ void __launch_bounds__(kFusedThreads, 1)
 kda_tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                    const PrepArgs p, const StateArgs a, const int nstate) {
+                    const __grid_constant__ PrepArgs p, const __grid_constant__ StateArgs a,
+                    const int nstate) {
     if ((int)blockIdx.x < nstate) {
-        state_cta<64>(a, blockIdx.x);
+        state_cta<64, true>(a, blockIdx.x);
         return;
     }
     extern __shared__ uint8_t smem_raw[];
@@ -1460,10 +1491,10 @@ kda_tc_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     t5::fence_before_sync();
     __syncthreads();
     t5::fence_after_sync();
-    const uint32_t tmem = s0.tmem_slot + (uint32_t)(w * 2 * D);
-    const int nprep = 2 * ((int)gridDim.x - nstate);
-    prep_worker(tm_q, tm_k, tm_v, tm_g, p, sm, tmem, threadIdx.x % kPrepThreads, 1 + w,
-                2 * ((int)blockIdx.x - nstate) + w, nprep);
+    // worker 1's columns follow worker 0's; each worker reads its own slot
+    if (w == 1 && threadIdx.x == kPrepThreads) sm.tmem_slot = s0.tmem_slot + 2 * D;
+    __syncthreads();
+    prep_worker<true>(tm_q, tm_k, tm_v, tm_g, p, sm);
     t5::fence_before_sync();
     __syncthreads();
     t5::fence_after_sync();
