@@ -104,7 +104,10 @@ KDA_DEVINL void st_rows(float *p, const float (&x)[RPL]) {
 
 template <int D>
 struct BwdSmem {
-    float st[CB][D][SLC];      // states S_{t-1} of the piece's tokens (this slice)
+    // states S_{t-1} of the piece's tokens: each thread's own RPL x 4 block, stored
+    // thread-minor (the 16-byte vectors of consecutive threads are adjacent, so a warp's
+    // access is conflict-free; the data never leaves the thread that wrote it)
+    float4 st[CB][D / 32][NTB];
     float q[CB][D], k[CB][D], a[CB][D];   // a = exp(g)
     float v[CB][SLC], dO[CB][SLC];
     float b[CB];
@@ -263,7 +266,9 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 #pragma unroll
             for (int i = 0; i < CB; ++i) {   // recompute: S_{t-1} of every token to smem
                 if (i < cl) {
-                    stS(&sm.st[i][0][c4], SLC, S);
+#pragma unroll
+                    for (int ri = 0; ri < RPL; ++ri)
+                        sm.st[i][ri][tid] = make_float4(S[ri][0], S[ri][1], S[ri][2], S[ri][3]);
                     step(S, i, dls[i]);
                 }
             }
@@ -283,9 +288,8 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                 float pq[RPL], pwr[RPL], xk[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ri = 0; ri < RPL; ++ri) {
-                    const int r = r0 + ri;
                     const float a = av[ri], kr = kv[ri], qr = qv[ri];
-                    const float4 sv = *reinterpret_cast<const float4 *>(&sm.st[i][r][c4]);
+                    const float4 sv = sm.st[i][ri][tid];
                     Sp[ri][0] = a * sv.x; Sp[ri][1] = a * sv.y; Sp[ri][2] = a * sv.z; Sp[ri][3] = a * sv.w;
                     pq[ri] = 0.f;
                     pwr[ri] = 0.f;
