@@ -200,9 +200,12 @@ kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const 
  * (sequence, head) state) and every other block runs two workers of the record
  * kernel, which write the records in time order (chunk j of every chain before
  * chunk j + 1) and publish each through a flag in the workspace; a state block
- * waits (bounded, 1 s) for a record's flag before copying it in.  The record
- * kernel never waits for the state pass, so the blocks cannot deadlock, and the
- * launch is cooperative so that every block is resident.  Results equal those of
+ * waits (bounded, 1 s) for a record's flag before copying it in, and a record
+ * worker starts a chunk only within a window of chunks (about 48 MiB of records)
+ * ahead of that chain's state blocks, so the records are read back from L2.  Each
+ * waits only for work that comes earlier in time order than what it holds, so the
+ * blocks cannot deadlock; the launch is cooperative so that every block is
+ * resident.  Results equal those of
  * kda_fwd_segmented with one segment up to the state pass's bf16 rounding (the two
  * schedules slice the state differently), and are checked against the oracle at
  * the same tolerance.

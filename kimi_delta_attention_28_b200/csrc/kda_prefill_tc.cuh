@@ -26,6 +26,8 @@
 // update, tcgen05 issue, output, bulk-copy producer) and hand off through
 // mbarriers, so the loop-carried path per chunk is one tcgen05 product plus the
 // register update of the state; the outputs and copies run beside it.
+// kda_tc_fused_kernel runs both in one cooperative launch for few long chains: state
+// blocks consume each record as soon as prep workers in the other blocks publish it.
 #pragma once
 
 #include "kda_common.cuh"
@@ -1458,9 +1460,11 @@ __global__ void __launch_bounds__(StateRoles<DVT>::THREADS, 1) kda_tc_state_kern
 // one block, with their own shared memory, tensor-memory columns and named barriers)
 // over the records in time order.  A state CTA waits for a record's ready flag
 // before copying it in, so the state chain starts after the first records instead
-// of after all of them, and the prep runs on the SMs the chain leaves idle.  The
-// wait is one-way (the prep never waits for the state pass) and bounded, and the
-// grid is one block per SM, launched cooperatively so all blocks are resident.
+// of after all of them, and the prep runs on the SMs the chain leaves idle; a prep
+// worker stays within a window of chunks ahead of its chain's state CTAs.  Every
+// wait is for work earlier in time order than what the waiter holds (no cycle) and
+// bounded, and the grid is one block per SM, launched cooperatively so all blocks
+// are resident.
 // ---------------------------------------------------------------------------
 constexpr int kFusedThreads = 2 * kPrepThreads;
 constexpr int kFusedPrepStride = (int)((sizeof(PrepSmem) + 1023) / 1024 * 1024);
