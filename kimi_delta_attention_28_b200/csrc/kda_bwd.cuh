@@ -16,14 +16,16 @@
 // scratch of its own (L2-resident), and for each CB-token piece, last first, the
 // piece's states into shared memory, to which it applies the rules above.  dv and
 // dh0 columns are complete within a slice; dq, dk, dg and dbeta are sums over all
-// columns: the D/32 slice CTAs of a chain form a thread-block cluster, and after
-// every piece each CTA adds the slices' partial sums for a quarter of the rows
+// columns: the D/16 slice CTAs of a chain form a thread-block cluster, and after
+// every piece each CTA adds the slices' partial sums for D/(D/16) of the rows
 // through distributed shared memory, in slice order (deterministic).
 // Inside a CTA, warp w owns 4 columns of the slice across all d rows (lane l: rows
 // RPL l .. RPL l + RPL - 1, RPL = d / 32), so the column sums every token needs
 // (u = S'^T k, G^T k) are in-warp butterflies with no CTA barrier; the row sums
 // (dq, dk, dg, dbeta) are only outputs, so each warp's share goes to shared memory
-// and the eight shares are added once per token.
+// and the four shares are added once per token.  (Keeping every token's shares of a
+// piece and adding them once per piece needs 37 KiB more shared memory, one CTA per
+// SM instead of two, and the 8-CTA clusters then no longer fit the GPU at once.)
 #pragma once
 
 #include "kda_common.cuh"

@@ -24,6 +24,22 @@ KDA_DEVINL float ld1<float>(const float *p) { return __ldg(p); }
 template <>
 KDA_DEVINL float ld1<__nv_bfloat16>(const __nv_bfloat16 *p) { return bf2f(*p); }
 
+// RPT consecutive fp32 values of a shared-memory row (16-byte aligned when RPT is a
+// multiple of 4), as few vector loads as possible.
+template <int RPT>
+KDA_DEVINL void ld_rows(const float *p, float (&x)[RPT]) {
+    if constexpr (RPT % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < RPT; i += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(p + i);
+            x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) x[i] = p[i];
+    }
+}
+
 template <int D, typename TIn>
 __global__ void __launch_bounds__(NT, 2)
 kda_decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
@@ -48,7 +64,7 @@ kda_decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     // Issue every state load first: RPT independent 16-byte loads per thread.
     float4 s[RPT];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(Sp + (rs + i * RS) * CG + cg);
+    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(Sp + (rs * RPT + i) * CG + cg);
 
     if (tid < D) {
         s_k[tid] = ld1<TIn>(k + unit * D + tid);
@@ -65,10 +81,13 @@ kda_decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     }
     // decay, then partial column sums of k^T S' and q^T S' over this thread's rows
     float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+    float av[RPT], kv[RPT], qv[RPT];   // this thread's rows rs RPT .. rs RPT + RPT - 1
+    ld_rows<RPT>(&s_a[rs * RPT], av);
+    ld_rows<RPT>(&s_k[rs * RPT], kv);
+    ld_rows<RPT>(&s_q[rs * RPT], qv);
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
-        const int row = rs + i * RS;
-        const float a = s_a[row], kr = s_k[row], qr = s_q[row];
+        const float a = av[i], kr = kv[i], qr = qv[i];
         s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
         pk.x += kr * s[i].x; pk.y += kr * s[i].y; pk.z += kr * s[i].z; pk.w += kr * s[i].w;
         pq.x += qr * s[i].x; pq.y += qr * s[i].y; pq.z += qr * s[i].z; pq.w += qr * s[i].w;
@@ -96,10 +115,9 @@ kda_decode_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     const float4 dl = *reinterpret_cast<const float4 *>(&s_delta[cg * 4]);
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
-        const int row = rs + i * RS;
-        const float kr = s_k[row];
+        const float kr = kv[i];
         s[i].x += kr * dl.x; s[i].y += kr * dl.y; s[i].z += kr * dl.z; s[i].w += kr * dl.w;
-        __stcs(Sp + row * CG + cg, s[i]);
+        __stcs(Sp + (rs * RPT + i) * CG + cg, s[i]);
     }
 }
 
@@ -155,7 +173,7 @@ kda_decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     float4 *Sp = reinterpret_cast<float4 *>(S + unit * D * D);
     float4 s[RPT];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(Sp + (rs + i * RS) * CG + cg);
+    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(Sp + (rs * RPT + i) * CG + cg);
 
     // stage the tokens' inputs: token t of (n, h) sits at row (n K + t) H + h
     for (int e = tid; e < ntok * D; e += NT) {
@@ -180,14 +198,17 @@ kda_decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     for (int t = 0; t < ntok; ++t) {
         // decay, then partial column sums of k^T S' (and q^T S') over this thread's rows
         float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+        float av[RPT], kv[RPT], qv[COMMIT ? 1 : RPT];   // rows rs RPT .. rs RPT + RPT - 1
+        ld_rows<RPT>(&s_a[t][rs * RPT], av);
+        ld_rows<RPT>(&s_k[t][rs * RPT], kv);
+        if constexpr (!COMMIT) ld_rows<RPT>(&s_q[t][rs * RPT], qv);
 #pragma unroll
         for (int i = 0; i < RPT; ++i) {
-            const int row = rs + i * RS;
-            const float a = s_a[t][row], kr = s_k[t][row];
+            const float a = av[i], kr = kv[i];
             s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
             pk.x += kr * s[i].x; pk.y += kr * s[i].y; pk.z += kr * s[i].z; pk.w += kr * s[i].w;
             if constexpr (!COMMIT) {
-                const float qr = s_q[t][row];
+                const float qr = qv[i];
                 pq.x += qr * s[i].x; pq.y += qr * s[i].y; pq.z += qr * s[i].z; pq.w += qr * s[i].w;
             }
         }
@@ -216,13 +237,13 @@ kda_decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         const float4 dl = *reinterpret_cast<const float4 *>(&s_delta[cg * 4]);
 #pragma unroll
         for (int i = 0; i < RPT; ++i) {
-            const float kr = s_k[t][rs + i * RS];
+            const float kr = kv[i];
             s[i].x += kr * dl.x; s[i].y += kr * dl.y; s[i].z += kr * dl.z; s[i].w += kr * dl.w;
         }
     }
     if constexpr (COMMIT) {
 #pragma unroll
-        for (int i = 0; i < RPT; ++i) __stcs(Sp + (rs + i * RS) * CG + cg, s[i]);
+        for (int i = 0; i < RPT; ++i) __stcs(Sp + (rs * RPT + i) * CG + cg, s[i]);
     }
 }
 
