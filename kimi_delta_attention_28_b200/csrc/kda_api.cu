@@ -235,7 +235,7 @@ kda_status launch_bwd(const void *q, const void *k, const void *v, const float *
                       long long chains, float *ckpt, float *sub, void *dq, void *dkk, void *dvv,
                       float *dg, float *db, float *dh0, int *err, cudaStream_t s) {
     using namespace kda::bwd;
-    const size_t smem = sizeof(BwdSmem<D>);
+    const size_t smem = sizeof(BwdSmem<D, TIn>);
     auto kern = kda_bwd_slice_kernel<D, TIn>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)

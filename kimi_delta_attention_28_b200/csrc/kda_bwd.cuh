@@ -44,6 +44,8 @@ template <>
 KDA_DEVINL float ldf<float>(const float *p) { return __ldg(p); }
 template <>
 KDA_DEVINL float ldf<__nv_bfloat16>(const __nv_bfloat16 *p) { return bf2f(*p); }
+KDA_DEVINL float to_f(float x) { return x; }
+KDA_DEVINL float to_f(__nv_bfloat16 x) { return bf2f(x); }
 template <typename TIn>
 KDA_DEVINL void stf(TIn *p, float x);
 template <>
@@ -104,7 +106,7 @@ KDA_DEVINL void st_rows(float *p, const float (&x)[RPL]) {
     }
 }
 
-template <int D>
+template <int D, typename TIn>
 struct BwdSmem {
     // states S_{t-1} of the piece's tokens: each thread's own RPL x 4 block, stored
     // thread-minor (the 16-byte vectors of consecutive threads are adjacent, so a warp's
@@ -115,6 +117,13 @@ struct BwdSmem {
     float b[CB];
     float pw[2][NWB][psw<D>()];   // each warp's share of a token's dq, dk, dg, dbeta
     float ps[CB][psw<D>()];       // this slice's partial dq, dk, dg rows and dbeta per token
+    // the next piece's inputs as they arrive (asynchronous copies, input dtype)
+    __align__(16) TIn xk[CB][D];
+    __align__(16) TIn xq[CB][D];
+    __align__(16) float xg[CB][D];
+    __align__(16) TIn xv[CB][SLC];
+    __align__(16) TIn xdo[CB][SLC];
+    __align__(16) float xb[CB];
 };
 
 // Sum of x over the 32 lanes of the warp, left in every lane.
@@ -137,7 +146,7 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                      int *err_word) {
     constexpr int NS = D / SLC, NT = NTB, RPL = D / 32;
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    BwdSmem<D> &sm = *reinterpret_cast<BwdSmem<D> *>(smem_raw);
+    BwdSmem<D, TIn> &sm = *reinterpret_cast<BwdSmem<D, TIn> *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r0 = RPL * lane, c4 = 4 * warp;        // this thread: rows r0.., slice columns c4..
     const int slice = blockIdx.x % NS, chain = blockIdx.x / NS, n = chain / H, h = chain % H;
@@ -175,27 +184,98 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
             *reinterpret_cast<float4 *>(base + (size_t)(r0 + i) * ld) =
                 make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
     };
-    // a piece's inputs into shared memory (tokens p0 .. p0 + cl - 1 of the sequence):
-    // q, k, exp(g) rows; this slice's v, dO columns; beta
-    auto stage = [&](int p0, int cl, bool with_q) {
-        const int c0 = t0 + p0;
+    // A piece's inputs in shared memory (tokens p0 .. p0 + cl - 1 of the sequence): q,
+    // k, exp(g) rows; this slice's v, dO columns; beta.  They arrive one piece ahead by
+    // asynchronous copies (rows past the piece zero-filled) into a staging area: when
+    // a piece is due, its copies are awaited, converted to fp32 in place for the
+    // steps, and the copies of the next piece in the kernel's order are issued, so
+    // their latency hides behind the current piece's work (CTA barriers do not wait
+    // for them).  The order: the forward walk's pieces (phase 1), then per chunk from
+    // the last, its recompute walk (phase 2, pieces 0 .. npc - 2) and its backward
+    // pieces (phase 3, npc - 1 .. 0, which also need q and dO).
+    struct Ev {
+        int ph, j, pc;   // ph 0: none
+    };
+    auto npc_of = [&](int j) { return (min(CK, len - j * CK) + CB - 1) / CB; };
+    auto first_back = [&](int j) -> Ev {
+        const int npc = npc_of(j);
+        return npc >= 2 ? Ev{2, j, 0} : Ev{3, j, npc - 1};
+    };
+    auto next_ev = [&](Ev e) -> Ev {
+        if (e.ph == 1) {
+            if (e.pc + 1 < npc_of(e.j)) return Ev{1, e.j, e.pc + 1};
+            if (e.j + 1 < nck) return Ev{1, e.j + 1, 0};
+            return first_back(nck - 1);
+        }
+        if (e.ph == 2) {
+            if (e.pc + 1 <= npc_of(e.j) - 2) return Ev{2, e.j, e.pc + 1};
+            return Ev{3, e.j, npc_of(e.j) - 1};
+        }
+        if (e.ph == 3) {
+            if (e.pc > 0) return Ev{3, e.j, e.pc - 1};
+            if (e.j > 0) return first_back(e.j - 1);
+        }
+        return Ev{0, 0, 0};
+    };
+    auto issue_stage = [&](Ev e) {
+        if (e.ph == 0) return;
+        const int p0 = e.j * CK + e.pc * CB, cl = min(CB, len - p0), c0 = t0 + p0;
+        const bool with_q = e.ph == 3;
+        constexpr int RC = D * (int)sizeof(TIn) / 16;   // 16-byte pieces of a q / k row
+        constexpr int GC = D * 4 / 16;                   // ... of a g row
+        constexpr int VC = SLC * (int)sizeof(TIn) / 16;  // ... of the slice of a v / dO row
+        for (int x = tid; x < CB * RC; x += NT) {
+            const int i = x / RC, ch = x % RC, ii = min(i, cl - 1);   // a valid source row
+            const size_t row = ((size_t)(c0 + ii) * H + h) * D;
+            const int nb = i < cl ? 16 : 0;
+            cp_async16(reinterpret_cast<uint8_t *>(sm.xk[i]) + 16 * ch,
+                       reinterpret_cast<const uint8_t *>(k + row) + 16 * ch, nb);
+            if (with_q)
+                cp_async16(reinterpret_cast<uint8_t *>(sm.xq[i]) + 16 * ch,
+                           reinterpret_cast<const uint8_t *>(q + row) + 16 * ch, nb);
+        }
+        for (int x = tid; x < CB * GC; x += NT) {
+            const int i = x / GC, ch = x % GC, ii = min(i, cl - 1);
+            cp_async16(reinterpret_cast<uint8_t *>(sm.xg[i]) + 16 * ch,
+                       reinterpret_cast<const uint8_t *>(g + ((size_t)(c0 + ii) * H + h) * D) +
+                           16 * ch,
+                       i < cl ? 16 : 0);
+        }
+        for (int x = tid; x < CB * VC; x += NT) {
+            const int i = x / VC, ch = x % VC, ii = min(i, cl - 1);
+            const size_t row = ((size_t)(c0 + ii) * H + h) * D + cs;
+            const int nb = i < cl ? 16 : 0;
+            cp_async16(reinterpret_cast<uint8_t *>(sm.xv[i]) + 16 * ch,
+                       reinterpret_cast<const uint8_t *>(v + row) + 16 * ch, nb);
+            if (with_q)
+                cp_async16(reinterpret_cast<uint8_t *>(sm.xdo[i]) + 16 * ch,
+                           reinterpret_cast<const uint8_t *>(dO + row) + 16 * ch, nb);
+        }
+        if (tid < CB)
+            cp_async4(&sm.xb[tid], beta + (size_t)(c0 + min(tid, cl - 1)) * H + h, tid < cl ? 4 : 0);
+        cp_async_commit();
+    };
+    Ev cur = Ev{nck > 0 ? 1 : 0, 0, 0};
+    issue_stage(cur);
+    auto stage = [&]() {
+        const bool with_q = cur.ph == 3;
+        cp_async_wait<0>();
+        __syncthreads();   // every thread's copies of the piece have landed
         for (int e = tid; e < CB * D; e += NT) {
             const int i = e / D, c = e % D;
-            const bool in = i < cl;
-            const size_t row = ((size_t)(c0 + i) * H + h) * D + c;
-            sm.k[i][c] = in ? ldf<TIn>(k + row) : 0.f;
-            sm.a[i][c] = in ? expf(__ldg(g + row)) : 1.f;
-            if (with_q) sm.q[i][c] = in ? ldf<TIn>(q + row) : 0.f;
+            sm.k[i][c] = to_f(sm.xk[i][c]);
+            sm.a[i][c] = expf(sm.xg[i][c]);   // exp(0) = 1 past the piece
+            if (with_q) sm.q[i][c] = to_f(sm.xq[i][c]);
         }
         for (int e = tid; e < CB * SLC; e += NT) {
             const int i = e / SLC, c = e % SLC;
-            const bool in = i < cl;
-            const size_t row = ((size_t)(c0 + i) * H + h) * D + cs + c;
-            sm.v[i][c] = in ? ldf<TIn>(v + row) : 0.f;
-            if (with_q) sm.dO[i][c] = in ? ldf<TIn>(dO + row) : 0.f;
+            sm.v[i][c] = to_f(sm.xv[i][c]);
+            if (with_q) sm.dO[i][c] = to_f(sm.xdo[i][c]);
         }
-        if (tid < CB) sm.b[tid] = tid < cl ? __ldg(beta + (size_t)(c0 + tid) * H + h) : 0.f;
-        __syncthreads();
+        if (tid < CB) sm.b[tid] = sm.xb[tid];
+        __syncthreads();   // converted; the staging area is free for the next piece
+        cur = next_ev(cur);
+        issue_stage(cur);
     };
     // one token of the recurrence on this thread's block; returns delta = v - u for the
     // warp's 4 columns (the same in every lane)
@@ -226,7 +306,8 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     };
     // run the tokens p0 .. p0 + cl - 1 forward from S (inputs staged here)
     auto run = [&](float (&S)[RPL][4], int p0, int cl) {
-        stage(p0, cl, false);
+        (void)p0;   // staged in order (see stage)
+        stage();
         float dl[4];
         for (int i = 0; i < cl; ++i) step(S, i, dl);
         __syncthreads();   // the next staging overwrites the inputs
@@ -262,7 +343,7 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         }
         for (int pc = npc - 1; pc >= 0; --pc) {
             const int p0 = j * CK + pc * CB, cl = min(CB, lenj - pc * CB);
-            stage(p0, cl, true);
+            stage();
             ldS(S, mysub + (size_t)pc * D * SLC, SLC);
             float dls[CB][4];   // delta of every token of the piece (this warp's columns)
 #pragma unroll
