@@ -65,9 +65,11 @@ KDA_DEVINL uint32_t dsmem_addr(const void *p, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
     return a;
 }
+// (No memory clobber: a run of these loads may be issued back to back; the cluster
+// barriers around them, which do clobber memory, keep them in place.)
 KDA_DEVINL float dsmem_ld(uint32_t addr) {
     float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr));
     return v;
 }
 KDA_DEVINL void cluster_sync() {
@@ -432,9 +434,12 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                     const int i = e / (3 * RPC + 1), f = e % (3 * RPC + 1);
                     if (f == 3 * RPC && cl_rank != 0) continue;
                     const int col = f == 3 * RPC ? 3 * D : (f / RPC) * D + cl_rank * RPC + f % RPC;
+                    float part[NS];   // all the slices' loads in flight at once, then added in order
+#pragma unroll
+                    for (int sl = 0; sl < NS; ++sl) part[sl] = dsmem_ld(dsmem_addr(&sm.ps[i][col], sl));
                     float sum = 0.f;
 #pragma unroll
-                    for (int sl = 0; sl < NS; ++sl) sum += dsmem_ld(dsmem_addr(&sm.ps[i][col], sl));
+                    for (int sl = 0; sl < NS; ++sl) sum += part[sl];
                     const size_t u = (size_t)(t0 + p0 + i) * H + h;
                     if (f == 3 * RPC) {
                         dbeta[u] = sum;
