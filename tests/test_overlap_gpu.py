@@ -132,6 +132,19 @@ def test_checkpoints_on_the_overlapped_schedule():
             _close(ck[b * per + c], s_ref[b], f"checkpoint {c} of sequence {b}")
 
 
+def test_in_place_state_update():
+    """hT == h0 (the one allowed overlap): every state block reads its slice of h0
+    before it writes hT."""
+    inp = W.make_prefill_inputs(2, 700, 3, 128, 128, torch.bfloat16, True, seed=135, device=DEV)
+    o_ref, hT_ref = _oracle(inp)
+    S = inp["h0"].clone()
+    o, hT = kda.kda_fwd_overlapped(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S, hT=S)
+    torch.cuda.synchronize()
+    assert hT.data_ptr() == S.data_ptr()
+    _close(o, o_ref, "o")
+    _close(S, hT_ref, "hT in place")
+
+
 def test_rejects_too_many_chains():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     H = sms // 2 + 1   # 2 * B * H >= SMs with B = 1
