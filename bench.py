@@ -199,15 +199,28 @@ def _strip_comments(text):
     return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
 
 
-def kernel_source_sha(src=None):
-    """sha256 over the device-code headers of the library (csrc/*.cuh, where every
-    kernel lives) with comments removed: it identifies the kernel code.  An edit of
-    comments alone, or of the host-side launch and policy code (csrc/*.cu), keeps it."""
+# The device-code headers each kernel is compiled from (its own and the shared one).
+KERNEL_SOURCES = {
+    "kda_tc_fused_kernel": ("kda_prefill_tc.cuh", "kda_common.cuh"),
+    "kda_tc_prep_kernel": ("kda_prefill_tc.cuh", "kda_common.cuh"),
+    "kda_tc_state_kernel": ("kda_prefill_tc.cuh", "kda_common.cuh"),
+    "kda_decode_kernel": ("kda_decode.cuh", "kda_common.cuh"),
+    "kda_decode_multi_kernel": ("kda_decode.cuh", "kda_common.cuh"),
+    "kda_bwd_slice_kernel": ("kda_bwd.cuh", "kda_common.cuh"),
+}
+
+
+def kernel_source_sha(kernel=None, src=None):
+    """sha256 over the device-code headers `kernel` is compiled from (all of csrc/*.cuh
+    when kernel is None or unknown) with comments removed: it identifies that kernel's
+    code.  An edit of comments alone, of the host-side launch and policy code
+    (csrc/*.cu), or of another kernel's header keeps it."""
     import hashlib
     src = src or os.path.join(ROOT, "kimi_delta_attention_28_b200", "csrc")
+    files = KERNEL_SOURCES.get(kernel)
     h = hashlib.sha256()
     for f in sorted(os.listdir(src)):
-        if f.endswith(".cuh"):
+        if f.endswith(".cuh") and (files is None or f in files):
             with open(os.path.join(src, f), encoding="utf-8") as fh:
                 h.update(f.encode() + b"\0" + _strip_comments(fh.read()).encode())
     return h.hexdigest()
@@ -217,12 +230,13 @@ def load_traffic(kernel, units):
     """DRAM bytes (read + write) of `kernel` for `units` units (token-heads for the
     prefill kernels, (sequence, head) chains for decode): the per-unit figure of the
     committed ncu summary profiles/traffic.json scaled by the units -- only if that
-    summary was taken on the current kernel sources (same sha256), else None."""
+    figure was taken on the kernel's current code (same sha256 of its headers), else
+    None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        if d.get("kernel_source_sha256") != kernel_source_sha():
+        if d.get("source_sha256", {}).get(kernel) != kernel_source_sha(kernel):
             return None
         per = d["dram_bytes_per_unit"].get(kernel)
         return None if per is None else float(per) * units

@@ -31,24 +31,34 @@ def _tree(root, code, name="k.cuh"):
 def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
     root = str(tmp_path)
     monkeypatch.setattr(bench, "ROOT", root)
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", {"prep": ("k.cuh", "c.cuh"),
+                                                  "decode": ("d.cuh", "c.cuh")})
     src = _tree(root, "// a kernel\n__global__ void k(int *p) { p[0] = 1; }\n")
-    sha = bench.kernel_source_sha()
+    _tree(root, "__device__ int c() { return 0; }\n", name="c.cuh")
+    _tree(root, "__global__ void d(int *p) { p[0] = 3; }\n", name="d.cuh")
+    sha, sha_d = bench.kernel_source_sha("prep"), bench.kernel_source_sha("decode")
     os.makedirs(os.path.join(root, "profiles"))
     with open(os.path.join(root, "profiles", "traffic.json"), "w") as f:
-        json.dump({"kernel_source_sha256": sha, "dram_bytes_per_unit": {"prep": 1.5}}, f)
+        json.dump({"source_sha256": {"prep": sha, "decode": sha_d},
+                   "dram_bytes_per_unit": {"prep": 1.5, "decode": 4.0}}, f)
     assert bench.load_traffic("prep", 100) == 150.0      # per-unit figure x units
-    assert bench.load_traffic("decode", 100) is None
+    assert bench.load_traffic("decode", 10) == 40.0
+    assert bench.load_traffic("other", 100) is None
     # a comment-only edit keeps the figure ...
     _tree(root, "/* the same kernel */\n__global__ void k(int *p) { p[0] = 1; }  // store\n")
-    assert bench.kernel_source_sha() == sha
+    assert bench.kernel_source_sha("prep") == sha
     assert bench.load_traffic("prep", 2) == 3.0
     # ... so does host-side code (launch policy) beside the kernels ...
     _tree(root, "int policy() { return 2; }\n", name="api.cu")
-    assert bench.kernel_source_sha() == sha
-    # ... a kernel code edit drops it
+    assert bench.kernel_source_sha("prep") == sha
+    # ... a code edit of one kernel's header drops its figure, not the other's ...
     _tree(root, "__global__ void k(int *p) { p[0] = 2; }\n")
-    assert bench.kernel_source_sha() != sha
+    assert bench.kernel_source_sha("prep") != sha
     assert bench.load_traffic("prep", 2) is None
+    assert bench.load_traffic("decode", 10) == 40.0
+    # ... and an edit of the shared header drops both
+    _tree(root, "__device__ int c() { return 1; }\n", name="c.cuh")
+    assert bench.load_traffic("decode", 10) is None
     assert os.path.isdir(src)
 
 
