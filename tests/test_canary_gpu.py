@@ -99,6 +99,21 @@ def test_fwd_writes_every_output(kind):
     _check(hT, hT_ref, inp["q"].dtype, f"{kind} hT")
 
 
+def test_overlapped_writes_every_output():
+    """The single-launch schedule, with NaN in o, hT and the whole workspace (its ready
+    flags and progress counters included: the call clears them itself)."""
+    inp = W.make_prefill_inputs(3, 64 * 5 + 9, 2, 128, 128, BF16, True, seed=37, device=DEV)
+    o, hT = _outs(inp)
+    B, T, H, dk = inp["q"].shape
+    ws = _nan_workspace(kda.workspace_size(B, T, H, dk, dk, 0, BF16))
+    kda.kda_fwd_overlapped(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], o=o,
+                           hT=hT, workspace=ws)
+    assert kda.device_error() == 0
+    o_ref, hT_ref = _ref(inp)
+    _check(o, o_ref, BF16, "overlapped o")
+    _check(hT, hT_ref, BF16, "overlapped hT")
+
+
 @pytest.mark.parametrize("kind", ["fixed", "packed"])
 def test_time_split_writes_every_output(kind):
     inp = W.make_prefill_inputs(1, 64 * 40 + 17, 2, 128, 128, BF16, True, seed=34, device=DEV) \
@@ -192,6 +207,12 @@ DEBUG_CHILD = textwrap.dedent("""
                                        inp["h0"], inp["cu_seqlens"])
         tol = 1e-2 if inp["q"].dtype == torch.bfloat16 else 1e-4
         worst = max(worst, err(o, o_ref) / tol, err(hT, hT_ref) / tol)
+    # the overlapped single launch (its prep workers' and state blocks' checks)
+    inp = cases[3]
+    o, hT = kda.kda_fwd_overlapped(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
+    assert kda.device_error() == 0
+    o_ref, hT_ref = oracle.kda_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"])
+    worst = max(worst, err(o, o_ref) / 1e-2, err(hT, hT_ref) / 1e-2)
     inp = W.make_prefill_inputs(1, 64 * 30, 1, 128, 128, torch.bfloat16, True, seed=7, device=dev)
     o, hT = kda.kda_fwd_segmented(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"],
                                   num_segments=4)
