@@ -124,7 +124,8 @@ size_t kda_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
  * the number of time segments of the state pass (kda_fwd_segmented: split only
  * when N * H chains are too few to fill the GPU), and, for fixed-length input
  * without a split, whether both phases run as one overlapped launch
- * (kda_fwd_overlapped) or as two (kda_fwd_segmented with one segment).
+ * (kda_fwd_overlapped) or as two (kda_fwd_segmented with one segment; also taken
+ * when the device refuses the overlapped launch).
  */
 kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
                    const float *beta, const float *h0, const int32_t *cu_seqlens,

@@ -535,8 +535,10 @@ static bool overlap_schedule(long long chains, long long cps, int sms) {
     return one < 0.95 * two;
 }
 
-// Both phases as one launch (fixed-length input, no T-split).
-static kda_status tc_fused(const void *q, const void *k, const void *v, const float *g,
+// Both phases as one launch (fixed-length input, no T-split).  *refused is set when
+// the launch itself was refused (e.g. the device cannot hold one such block per SM
+// at once), with nothing started, so the caller may take the two launches instead.
+static kda_status tc_fused(bool *refused, const void *q, const void *k, const void *v, const float *g,
                            const float *beta, const float *h0, int N, int T, int H,
                            const WsLayout &L, void *o, float *hT, void *workspace,
                            cudaStream_t s, float *ckpt = nullptr, int ckpt_chunks = 0,
@@ -587,6 +589,7 @@ static kda_status tc_fused(const void *q, const void *k, const void *v, const fl
     if (cudaFuncSetAttribute(kda_tc_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kFusedSmem) != cudaSuccess) {
         cudaGetLastError();
+        if (refused) *refused = true;
         return KDA_ERR_CUDA;
     }
     // every block must be resident at once (state blocks wait for prep blocks): one
@@ -604,6 +607,7 @@ static kda_status tc_fused(const void *q, const void *k, const void *v, const fl
     if (cudaLaunchKernelEx(&cfg, kda_tc_fused_kernel, tq, tk, tv, tg, p, a, (int)nstate) !=
         cudaSuccess) {
         cudaGetLastError();
+        if (refused) *refused = true;
         return KDA_ERR_CUDA;
     }
     return launch_status();
@@ -658,8 +662,11 @@ kda_status kda_fwd(const void *q, const void *k, const void *v, const float *g,
     if (N == 0) return KDA_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (is_tc_path(dtype, dk)) {
-        if (use_overlap(cu_seqlens, N, T, H, L))
-            return tc_fused(q, k, v, g, beta, h0, N, T, H, L, o, hT, workspace, s);
+        if (use_overlap(cu_seqlens, N, T, H, L)) {
+            bool refused = false;
+            st = tc_fused(&refused, q, k, v, g, beta, h0, N, T, H, L, o, hT, workspace, s);
+            if (!refused) return st;   // else: the two launches below
+        }
         if ((st = tc_intra(q, k, v, g, beta, cu_seqlens, N, T, H, L, workspace, s)) != KDA_OK)
             return st;
         return tc_inter(h0, cu_seqlens, N, T, H, L, o, hT, workspace, s);
@@ -704,9 +711,12 @@ kda_status kda_fwd_checkpointed(const void *q, const void *k, const void *v, con
     if (!cu_seqlens && (long long)B * (T / ckpt_every) > ckpt_capacity) return KDA_ERR_INVALID_ARG;
     if (N == 0) return KDA_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (use_overlap(cu_seqlens, N, T, H, L))
-        return tc_fused(q, k, v, g, beta, h0, N, T, H, L, o, hT, workspace, s, ckpts,
-                        ckpt_every / kda::tc::C, ckpt_capacity);
+    if (use_overlap(cu_seqlens, N, T, H, L)) {
+        bool refused = false;
+        st = tc_fused(&refused, q, k, v, g, beta, h0, N, T, H, L, o, hT, workspace, s, ckpts,
+                      ckpt_every / kda::tc::C, ckpt_capacity);
+        if (!refused) return st;   // else: the two launches below
+    }
     if ((st = tc_intra(q, k, v, g, beta, cu_seqlens, N, T, H, L, workspace, s)) != KDA_OK)
         return st;
     return tc_inter(h0, cu_seqlens, N, T, H, L, o, hT, workspace, s, ckpts,
@@ -736,7 +746,7 @@ kda_status kda_fwd_overlapped(const void *q, const void *k, const void *v, const
     if (N == 0) return KDA_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0) return tc_inter(h0, nullptr, N, T, H, L, o, hT, workspace, s);   // hT = h0
-    return tc_fused(q, k, v, g, beta, h0, N, T, H, L, o, hT, workspace, s);
+    return tc_fused(nullptr, q, k, v, g, beta, h0, N, T, H, L, o, hT, workspace, s);
 }
 
 int kda_fwd_plan_segments(int B, int T, int H, int dk, int dv, int num_seqs, int dtype) {
