@@ -4,8 +4,9 @@
 Default (headline) workload: the 1M-token prefill -- bf16 q/k/v, fp32 g/beta/state,
 B=1, H=16, T=1,048,576, d_k = d_v = 128, zero initial state, seeded synthetic
 inputs (about 26 GB of inputs and outputs, far larger than L2).  A step is one
-full ``kda_fwd`` call (the intra-chunk kernel, then the state pass) over the whole
-batch.  On one GPU the same JSON line also carries, under ``workloads``, the other
+full ``kda_fwd`` call over the whole batch: for this shape one overlapped launch in
+which the state pass consumes the intra-chunk records as they are written
+(``--two-launch`` times the intra-chunk kernel, then the state pass, instead).  On one GPU the same JSON line also carries, under ``workloads``, the other
 measured workloads with their own roofline and sampled parity: the B=2, H=8,
 T=4,096 prefill, the packed varlen prefill (16 sequences, H=32) and the decode
 step (256 sequences x 96 heads, fp32 state in place).
