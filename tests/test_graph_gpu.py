@@ -24,9 +24,13 @@ def _cuda():
     kda.load_library()
 
 
-@pytest.mark.parametrize("shape", [(2, 1000, 4), (1, 20000, 1)])   # plain; time-split policy
+# two launches; time-split policy; the overlapped single launch (ready flags cleared by a
+# captured memset, the cooperative kernel captured as a graph node)
+@pytest.mark.parametrize("shape", [(2, 1000, 4), (1, 20000, 1), (2, 8192, 8)])
 def test_prefill_graph_replays_on_new_inputs(shape):
     B, T, H = shape
+    if shape == (2, 8192, 8) and not kda.plan_overlap(B, T, H, 128, 128, 0, BF16):
+        pytest.skip("kda_fwd does not overlap at these sizes on this GPU")
     bufs = W.make_prefill_inputs(B, T, H, 128, 128, BF16, True, seed=90, device=DEV)
     ws = torch.empty(kda.workspace_size(B, T, H, 128, 128, 0, BF16), dtype=torch.uint8,
                      device=DEV)
