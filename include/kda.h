@@ -82,7 +82,9 @@ int kda_build_flags(void);
  * Bytes of device workspace that kda_fwd needs for these sizes.  The
  * tensor-core path stores, per 64-token chunk and head, the chunk's affine map
  * on the state (98,816 bytes: the state transition and offset, the output
- * read-out and offset, and the chunk's total decay) that the state pass consumes.
+ * read-out and offset, and the chunk's total decay) that the state pass consumes,
+ * plus a 4-byte ready flag per record and a few KiB of progress counters for the
+ * overlapped single-launch schedule.
  * When few (sequence, head) chains would leave most SMs idle, kda_fwd splits
  * each chain in time (see kda_fwd_segmented); the size returned here includes
  * room for the largest split the library would choose on a GPU of up to 192
