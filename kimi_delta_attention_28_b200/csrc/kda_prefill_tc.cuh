@@ -39,6 +39,25 @@ constexpr int D = 128;          // head size (d_k = d_v)
 constexpr int C = 64;           // chunk length
 constexpr int ST = 16;          // sub-tile length for the decay reference rows
 constexpr int NST = C / ST;     // sub-tiles per chunk
+// A 4-D tensor copy (tma_load_4d) with an L2 eviction-priority hint (`policy`, from
+// l2_evict_first): for data read exactly once, so that it does not displace data
+// still to be read.
+KDA_DEVINL void tma_load_4d_hint(void *smem_dst, const CUtensorMap *tm, int c0, int c1, int c2,
+                                 int c3, uint64_t *bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;\n"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1),
+          "r"(c2), "r"(c3), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+// An L2 cache policy that marks every access it is given as evict-first.
+KDA_DEVINL uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+    return p;
+}
+
 // Largest total decay of a chunk (log2 units, per channel) for which the prep uses
 // one reference row and whole-chunk tensor-core products: factors up to 2^120 stay
 // inside the bf16 / fp32 range (2^127) with room for |k| <= 1.
@@ -332,25 +351,31 @@ KDA_DEVINL void prep_worker(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
     // neutralised in P1: their g counts as zero and their beta is zero, so they neither
     // decay nor write the state.  beta comes by 4-byte cp.async beside k and q.
     uint32_t pend = 0, pend_par = 0;   // load groups in flight and the parity each completes
+    // overlapped schedule: the inputs are read once, so they go through L2 as
+    // evict-first and leave it to the records in flight between the two roles
+    auto load = [&](void *dst, const CUtensorMap *tm, int c0, int c1, int c2, int c3, uint64_t *b) {
+        if constexpr (OVERLAP) tma_load_4d_hint(dst, tm, c0, c1, c2, c3, b, l2_evict_first());
+        else tma_load_4d(dst, tm, c0, c1, c2, c3, b);
+    };
     auto issue = [&](int grp, const Item &it, uint32_t par) {
         if (tid == 0) {
             uint64_t *bar = &sm.ld_bar[grp];
             fence_proxy_async_smem();   // earlier generic accesses of the tile come first
             if (grp < 2) {
                 mbar_arrive_expect_tx(bar, 32 * D * 4);
-                tma_load_4d(grp ? sm.xk : sm.ka, &tm_g, 0, it.h, it.tl + 32 * grp, it.b, bar);
+                load(grp ? sm.xk : sm.ka, &tm_g, 0, it.h, it.tl + 32 * grp, it.b, bar);
             } else if (grp == 2) {
                 mbar_arrive_expect_tx(bar, 2 * C * D * 2);
 #pragma unroll
                 for (int pl = 0; pl < 2; ++pl) {
-                    tma_load_4d(sm.qa + pl * C * 128, &tm_k, 64 * pl, it.h, it.tl, it.b, bar);
-                    tma_load_4d(sm.kb + pl * C * 128, &tm_q, 64 * pl, it.h, it.tl, it.b, bar);
+                    load(sm.qa + pl * C * 128, &tm_k, 64 * pl, it.h, it.tl, it.b, bar);
+                    load(sm.kb + pl * C * 128, &tm_q, 64 * pl, it.h, it.tl, it.b, bar);
                 }
             } else {
                 mbar_arrive_expect_tx(bar, C * D * 2);
 #pragma unroll
                 for (int pl = 0; pl < 2; ++pl)
-                    tma_load_4d(sm.xv + pl * C * 128, &tm_v, 64 * pl, it.h, it.tl, it.b, bar);
+                    load(sm.xv + pl * C * 128, &tm_v, 64 * pl, it.h, it.tl, it.b, bar);
             }
         }
         if (grp == 2) {
