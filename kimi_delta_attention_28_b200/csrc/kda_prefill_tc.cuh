@@ -964,7 +964,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 // ---------------------------------------------------------------------------
 // Kernel 2: inter-chunk state pass on tcgen05, warp-specialised.
-// grid = units * tiles CTAs of 32 (NSW + 6) threads.  A unit is one (sequence,
+// grid = units * tiles CTAs of 32 (NSW + 7) threads.  A unit is one (sequence,
 // head) chain, or with a T-split one of its nseg consecutive segments (equal
 // numbers of chunks, the last may be shorter or empty); tiles = D / DVT column
 // slices of the state.  Roles:
@@ -981,9 +981,11 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 //                        waits for D_O's ring slot and accumulator;
 //   4 output warps:      O = D_O + O0 for the chunk's rows (warp w reads tensor-memory
 //                        lane quarter w % 4), stored as bf16;
-//   1 producer warp:     bulk copies of the chunk records into two rings, the state
+//   2 producer warps:    bulk copies of the chunk records into two rings, the state
 //                        ring (M', exp(G_C), R slice) and the output ring (Q', O0 slice),
-//                        refilling a slot once its consumers release it.
+//                        one warp each, refilling a slot once its consumers release it
+//                        (one lane of each warp: two divergent lanes of one warp delayed
+//                        the state ring's copies while the other lane spun on its wait).
 // The roles hand off through mbarriers only, so the loop-carried path per chunk is
 // M' S on the tensor core -> state update -> bf16 copy -> next M' S.  Every wait is
 // bounded; a wait that runs out sets the shared abort flag and the timeout bit, all
@@ -1065,12 +1067,14 @@ struct T5Layout {
 
 // Warp roles of the state pass: NSW = 4 DVT/32 state warps (warp w: key row
 // 32 (w % 4) + lane, columns 32 (w / 4) .. + 31 of the slice), then the MMA warp, four
-// output warps and the producer warp.
+// output warps and the producer warps of the state ring and the output ring; in the
+// overlapped schedule one more warp polls the records' ready flags.
 template <int DVT>
 struct StateRoles {
     static constexpr int NSW = 4 * (DVT / 32);
-    static constexpr int MMA_WARP = NSW, OUT_WARP0 = NSW + 1, PROD_WARP = NSW + 5;
-    static constexpr int THREADS = 32 * (NSW + 6);
+    static constexpr int MMA_WARP = NSW, OUT_WARP0 = NSW + 1, PROD_WARP = NSW + 5,
+                         PROD_B_WARP = NSW + 6, POLL_WARP = NSW + 7;
+    static constexpr int THREADS = 32 * (NSW + 7);
 };
 
 // One state-pass CTA: `cta` indexes (unit, column tile), column tile fastest.  Warps
@@ -1147,14 +1151,15 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
     int *err_word = a.err_word;
 
     if (tid == 0) {
-        for (int s = 0; s < NA; ++s) { mbar_init(&full_a[s], 1); mbar_init(&a_free[s], 32 * RL::NSW); }
-        for (int s = 0; s < NB; ++s) { mbar_init(&full_b[s], 1); mbar_init(&b_free[s], 128); }
+        // consumers release and hand over once per warp (lane 0, after __syncwarp)
+        for (int s = 0; s < NA; ++s) { mbar_init(&full_a[s], 1); mbar_init(&a_free[s], RL::NSW); }
+        for (int s = 0; s < NB; ++s) { mbar_init(&full_b[s], 1); mbar_init(&b_free[s], 4); }
         mbar_init(done_s, 1);
         mbar_init(&done_o[0], 1);
         mbar_init(&done_o[1], 1);
-        for (int w = 0; w < 4; ++w) mbar_init(&sb_full[w], 32 * (DVT / 32));
-        mbar_init(&do_free[0], 128);
-        mbar_init(&do_free[1], 128);
+        for (int w = 0; w < 4; ++w) mbar_init(&sb_full[w], DVT / 32);
+        mbar_init(&do_free[0], 4);
+        mbar_init(&do_free[1], 4);
         *abort_flag = 0;
         cnt[0] = cnt[1] = cnt[2] = 0;
         *rdy = 0;
@@ -1228,7 +1233,8 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
                 *reinterpret_cast<uint4 *>(sb + L::sb_off(row, cb + c8)) = pk;
             }
             fence_proxy_async_smem();   // generic writes -> tensor-core reads
-            mbar_arrive(&sb_full[warp & 3]);   // key rows 32(w%4).. : K slab w%4 of the next products
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sb_full[warp & 3]);   // key rows 32(w%4).. : K slab w%4 of the next products
         };
         write_sb(0);
         int j = 0;
@@ -1249,7 +1255,8 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
             float v[32];
             t5::ld32(tmem + lane_base + L::ds_col(j & 1) + cb, v);
             t5::fence_before_sync();
-            mbar_arrive(&a_free[sa]);   // this thread is done with the slot and with D_S
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_free[sa]);   // the warp is done with the slot and with D_S
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const uint32_t u[4] = {rv[i].x, rv[i].y, rv[i].z, rv[i].w};
@@ -1365,7 +1372,8 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
             float w[DVT];
             t5::ld_cols<DVT>(tmem + lane_base + DVT + (j & 1) * DVT, w);
             t5::fence_before_sync();
-            mbar_arrive(&do_free[j & 1]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&do_free[j & 1]);
             const int t0 = seq_t0 + j * C;
             const int len = min(C, seq_len - j * C);
             if (lane < 16 && orow < len) {
@@ -1385,9 +1393,10 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
                     *reinterpret_cast<uint4 *>(op + i * 8) = res;
                 }
             }
-            mbar_arrive(&b_free[sbb]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&b_free[sbb]);
         }
-    } else if (OVERLAP && warp == RL::PROD_WARP + 1) {
+    } else if (OVERLAP && warp == RL::POLL_WARP) {
         // ---------------- poller (overlapped schedule only; the fused block's spare warp) ----------------
         // walks the chain's records in order, waiting (acquire, GPU scope) for each ready
         // flag the prep sets, and counts the published ones in shared memory, so the
@@ -1400,8 +1409,8 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
             }
         }
         __syncwarp();
-    } else if (warp == RL::PROD_WARP) {
-        // ---------------- producer warp: lane 0 feeds ring A, lane 1 ring B ----------------
+    } else if (warp == RL::PROD_WARP || warp == RL::PROD_B_WARP) {
+        // ---------------- producer warps: lane 0 of each feeds ring A, ring B ----------------
         // overlapped schedule: a record is copied in only once the poller has seen it published
         auto ready = [&](int c) {
             if constexpr (!OVERLAP) return true;
@@ -1415,7 +1424,7 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
             fence_proxy_async_global();   // the prep's generic stores -> these bulk copies
             return true;
         };
-        if (lane == 0) {
+        if (lane == 0 && warp == RL::PROD_WARP) {
             for (int c = 0; c < nchunks && !*abort_flag; ++c) {
                 const int s = c % NA;
                 if (c >= NA && !mbar_wait_bounded(&a_free[s], ((c - NA) / NA) & 1)) { fail(); break; }
@@ -1435,7 +1444,7 @@ KDA_DEVINL void state_cta(const StateArgs &a, const int cta) {
                 // here would hold this lane until its earlier copies are done)
                 if constexpr (OVERLAP) store_relaxed(a.progress + kProgStride * cta, c + 1);
             }
-        } else if (lane == 1) {
+        } else if (lane == 0) {
             for (int c = 0; c < (map_mode ? 0 : nchunks) && !*abort_flag; ++c) {
                 const int s = c % NB;
                 if (c >= NB && !mbar_wait_bounded(&b_free[s], ((c - NB) / NB) & 1)) { fail(); break; }
