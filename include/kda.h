@@ -318,9 +318,7 @@ kda_status kda_cp_finish(const float *maps, int rank, int world, const float *h0
  * dL/dg, dL/dbeta (fp32) and dL/dh0 (fp32, NULL to skip).  Same inputs, layouts,
  * packed-sequence rules and alignment as kda_fwd; grad_o [B, T, H, d_v] has the
  * dtype of q; grad_hT, grad_h0 [N, H, d_k, d_v].  No gradient buffer may alias an
- * input.  The workspace must hold kda_bwd_workspace_size(...) bytes: the state every
- * 64 tokens of every (sequence, head) (d_k d_v / 16 bytes per token-head, 1 KiB at
- * d = 128) plus 8 states of scratch per (sequence, head).
+ * input.  The workspace must hold kda_bwd_workspace_size(...) bytes.
  *
  * What it computes is the chain rule through the recurrence (panel "KDA 单头递归"),
  * token by token from the last to the first, with G = dL/dS_t, S' = Diag(exp g_t)
@@ -329,10 +327,29 @@ kda_status kda_cp_finish(const float *maps, int rank, int world, const float *h0
  *     dk = beta w - S' dv;  G' = G - k dv^T;  dg_i = sum_j S'_ij G'_ij;
  *     G = Diag(exp g) G';  and dh0 = G after the first token.
  * The source pages name the training kernel ("FlashKDA / FLA" panel) but give no
- * formulas for it; this is the gradient of the recurrence they print, in fp32 on
- * CUDA cores (one CTA per (sequence, head) and 32 value columns, the slices of a
- * chain one thread-block cluster; states recomputed from stored checkpoints).  All
- * head sizes and dtypes of kda_fwd are supported.
+ * formulas for it; this is the gradient of the recurrence they print, applied in fp32
+ * on CUDA cores per (sequence, head) and 16 value columns, the slices of a chain (or of
+ * a segment of it) one thread-block cluster, states recomputed from checkpoints.
+ *
+ * Two schedules (kda_bwd_segmented chooses explicitly):
+ *   per chain:  each chain walked whole, from h0 and dL/dhT; every dtype, head size
+ *               and the packed layout.  Workspace: the state every 64 tokens of every
+ *               (sequence, head) (d_k d_v / 16 bytes per token-head) plus 8 states per
+ *               (sequence, head).  The gradients stored in fp32 match an fp64
+ *               evaluation to about 1e-7.
+ *   segmented:  (bf16, d_k = d_v = 128, fixed-length input, grad_o, grad_q and grad_k
+ *               16-byte aligned) the chain cut into segments of whole 64-token chunks,
+ *               all run at once.  A segment's starting state comes from the tensor-core
+ *               forward (kda_fwd's records and state pass, with a checkpoint at every
+ *               segment start), its ending gradient from the chunk-level chain
+ *               dL/dS_in = Diag(exp G_C) dL/dS_out + M'^T dL/dS_out + Q'^T dO run by the
+ *               same state pass backwards over the chunks (reversed records); both carry
+ *               the bf16 records' rounding, so every gradient is held to the bf16
+ *               prefill bound (rel-L2 <= 1e-2).  grad_q and grad_k serve as scratch for
+ *               the two state passes' outputs before they receive the gradients.
+ * kda_bwd takes the segmented schedule whenever it applies and some cut leaves at least
+ * two segments: one chunk per segment, or the fewest chunks (a power of two dividing
+ * the chunks per sequence) that keep (sequences x heads x segments) <= 1024.
  */
 size_t kda_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype);
 kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
@@ -341,6 +358,28 @@ kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
                    const float *grad_hT, void *grad_q, void *grad_k, void *grad_v,
                    float *grad_g, float *grad_beta, float *grad_h0, void *workspace,
                    size_t ws_bytes, void *stream);
+
+/*
+ * kda_bwd with the schedule chosen by the caller: num_segments = 0 as kda_bwd, 1 the
+ * per-chain pass (any input kda_bwd takes), n >= 2 the segmented pass with n segments
+ * per sequence (n must divide ceil(T / 64); bf16, d = 128, fixed-length input, else
+ * KDA_ERR_UNSUPPORTED_SHAPE; grad_o, grad_q, grad_k 16-byte aligned, else
+ * KDA_ERR_MISALIGNED).  The workspace must hold
+ * kda_bwd_segmented_workspace_size(..., num_segments) bytes (0 when the request cannot
+ * be met).
+ */
+size_t kda_bwd_segmented_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
+                                        int dtype, int num_segments);
+/* The segments per sequence kda_bwd uses for these sizes (1: the per-chain pass; it
+ * may still take the per-chain pass when the alignment rule above is not met); 0 on
+ * invalid sizes. */
+int kda_bwd_plan_segments(int B, int T, int H, int dk, int dv, int num_seqs, int dtype);
+kda_status kda_bwd_segmented(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *h0, const int32_t *cu_seqlens,
+                             int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
+                             const void *grad_o, const float *grad_hT, void *grad_q, void *grad_k,
+                             void *grad_v, float *grad_g, float *grad_beta, float *grad_h0,
+                             int num_segments, void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * Speculative decoding: verify K drafted tokens per sequence, then commit the

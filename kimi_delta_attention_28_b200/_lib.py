@@ -55,6 +55,10 @@ SIGNATURES = {
     "kda_bwd_workspace_size": ([_I, _I, _I, _I, _I, _I, _I], _SZ),
     "kda_bwd": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP,
                  _VP, _VP, _VP, _VP, _VP, _SZ, _VP], _I),
+    "kda_bwd_segmented_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _I], _SZ),
+    "kda_bwd_plan_segments": ([_I, _I, _I, _I, _I, _I, _I], _I),
+    "kda_bwd_segmented": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP,
+                           _VP, _VP, _VP, _VP, _VP, _VP, _I, _VP, _SZ, _VP], _I),
     "kda_decode_verify": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP], _I),
     "kda_decode_commit": ([_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP], _I),
     "kda_fwd_noalloc": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _VP, _VP,
@@ -497,10 +501,33 @@ def bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
                                                      _dtype_code(dtype)))
 
 
+def bwd_segmented_workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
+                                 dtype: torch.dtype, num_segments: int) -> int:
+    return int(load_library().kda_bwd_segmented_workspace_size(B, T, H, dk, dv, num_seqs,
+                                                               _dtype_code(dtype), num_segments))
+
+
+def bwd_plan_segments(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
+                      dtype: torch.dtype) -> int:
+    """Segments per sequence kda_bwd uses (1: the per-chain pass)."""
+    return int(load_library().kda_bwd_plan_segments(B, T, H, dk, dv, num_seqs, _dtype_code(dtype)))
+
+
 def kda_bwd(q, k, v, g, beta, h0, cu_seqlens, grad_o, grad_hT=None, *, workspace=None):
     """Gradient of a loss through kda_fwd: given grad_o = dL/do [B, T, H, d_v] (dtype of
     q) and grad_hT = dL/dhT [N, H, d_k, d_v] fp32 (None: zero), returns (dq, dk, dv, dg,
     dbeta, dh0): dq, dk, dv in the dtype of q, the rest fp32 (dh0 None when h0 is None)."""
+    return _bwd(q, k, v, g, beta, h0, cu_seqlens, grad_o, grad_hT, None, workspace)
+
+
+def kda_bwd_segmented(q, k, v, g, beta, h0, cu_seqlens, grad_o, grad_hT=None, *,
+                      num_segments: int, workspace=None):
+    """kda_bwd with the schedule given: num_segments 0 as kda_bwd, 1 the per-chain pass,
+    n >= 2 n segments per sequence (n divides ceil(T / 64); bf16, d = 128, fixed length)."""
+    return _bwd(q, k, v, g, beta, h0, cu_seqlens, grad_o, grad_hT, int(num_segments), workspace)
+
+
+def _bwd(q, k, v, g, beta, h0, cu_seqlens, grad_o, grad_hT, num_segments, workspace):
     lib = load_library()
     dev = q.device
     B, T, H, dk, dv, num_seqs, N = _prefill_shapes(q, k, v, g, beta, h0, cu_seqlens,
@@ -518,14 +545,20 @@ def kda_bwd(q, k, v, g, beta, h0, cu_seqlens, grad_o, grad_hT=None, *, workspace
     dq, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dg, db = torch.empty_like(g), torch.empty_like(beta)
     dh0 = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev) if h0 is not None else None
-    need = bwd_workspace_size(B, T, H, dk, dv, num_seqs, q.dtype)
+    if num_segments is None:
+        need = bwd_workspace_size(B, T, H, dk, dv, num_seqs, q.dtype)
+    else:
+        need = bwd_segmented_workspace_size(B, T, H, dk, dv, num_seqs, q.dtype, num_segments)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    _check(lib.kda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                       _ptr(cu_seqlens), num_seqs, B, T, H, dk, dv, _dtype_code(q.dtype),
-                       _ptr(grad_o), _ptr(grad_hT), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg),
-                       _ptr(db), _ptr(dh0), _ptr(workspace), workspace.numel(), _stream(dev)),
-           "kda_bwd")
+    common = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
+              num_seqs, B, T, H, dk, dv, _dtype_code(q.dtype), _ptr(grad_o), _ptr(grad_hT),
+              _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(db), _ptr(dh0))
+    if num_segments is None:
+        _check(lib.kda_bwd(*common, _ptr(workspace), workspace.numel(), _stream(dev)), "kda_bwd")
+    else:
+        _check(lib.kda_bwd_segmented(*common, num_segments, _ptr(workspace), workspace.numel(),
+                                     _stream(dev)), "kda_bwd_segmented")
     return dq, dk_, dv_, dg, db, dh0
 
 

@@ -14,6 +14,7 @@
 
 #include "../../include/kda.h"
 #include "kda_bwd.cuh"
+#include "kda_bwd_chain.cuh"
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
 #include "kda_prefill_simt.cuh"
@@ -228,21 +229,64 @@ BwdLayout bwd_layout(int B, int T, int H, int dk, int num_seqs, int dtype) {
     return L;
 }
 
+// Segmented backward (tensor-core path, fixed-length input): chains cut into segments of
+// sc chunks, sc the smallest power of two dividing the chunks per sequence for which
+// the segments number at most kBwdUnits (each unit holds the per-CTA scratch of
+// NSUB states per slice, 512 KiB at d = 128); 0 when no cut leaves two segments.
+constexpr long long kBwdUnits = 1024;
+int bwd_seg_chunks(long long chains, int cps) {
+    if (chains <= 0 || cps < 2) return 0;
+    for (int sc = 1; sc < cps && cps % sc == 0; sc *= 2)
+        if (chains * (cps / sc) <= kBwdUnits) return sc;
+    return 0;
+}
+// Its workspace: the forward's (records), the reversed records, the states at the
+// segment starts and the state gradients at the segment ends (nfw = floor(T / (sc C))
+// slots per sequence each), then the per-token pass's checkpoints and scratch.
+struct BwdSegLayout {
+    WsLayout F;
+    size_t rrec, fck, rck, ckpt, sub, total;
+    int sc, nseg, nfw, cps;
+};
+// sc chunks per segment (sc divides the chunks per sequence, at least two segments);
+// sc = 0: the policy above.  S.sc == 0 when no such cut exists.
+BwdSegLayout bwd_seg_layout(int B, int T, int H, int dk, int dtype, int sc = 0) {
+    BwdSegLayout S{};
+    if (!is_tc_path(dtype, dk) || B <= 0 || T <= 0) return S;
+    S.cps = (T + kda::tc::C - 1) / kda::tc::C;
+    S.sc = sc > 0 ? (sc < S.cps && S.cps % sc == 0 ? sc : 0) : bwd_seg_chunks((long long)B * H, S.cps);
+    if (!S.sc) return S;
+    S.nseg = S.cps / S.sc;
+    S.nfw = T / (S.sc * kda::tc::C);
+    S.F = ws_layout(B, T, H, dk, 0, dtype, 1);
+    S.rrec = round_up(S.F.total, 256);
+    S.fck = round_up(S.rrec + (size_t)S.F.max_chunks * H * kda::tc::REC_BYTES, 256);
+    const size_t states = (size_t)B * S.nfw * H * dk * dk * sizeof(float);
+    S.rck = round_up(S.fck + states, 256);
+    const long long slots = (long long)B * T / kda::bwd::CK + B + 1;
+    S.ckpt = round_up(S.rck + states, 256);
+    S.sub = round_up(S.ckpt + (size_t)slots * H * dk * dk * sizeof(float), 256);
+    S.total = S.sub + (size_t)B * H * S.nseg * kda::bwd::NSUB * dk * dk * sizeof(float);
+    return S;
+}
+
 template <int D, typename TIn>
 kda_status launch_bwd(const void *q, const void *k, const void *v, const float *g,
                       const float *beta, const float *h0, const int32_t *cu, const int *hdr,
                       const void *dO, const float *dhT, int T, int H, long long ntok,
                       long long chains, float *ckpt, float *sub, void *dq, void *dkk, void *dvv,
-                      float *dg, float *db, float *dh0, int *err, cudaStream_t s) {
+                      float *dg, float *db, float *dh0, int *err, cudaStream_t s, int nseg = 1,
+                      int seg_chunks = 1, const float *s_start = nullptr,
+                      const float *g_end = nullptr, int nfw = 0, int cps = 0) {
     using namespace kda::bwd;
     const size_t smem = sizeof(BwdSmem<D, TIn>);
     auto kern = kda_bwd_slice_kernel<D, TIn>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return KDA_ERR_CUDA;
-    const long long grid = chains * (D / SLC);
+    const long long grid = chains * nseg * (D / SLC);
     if (grid > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
-    // the D / 32 column slices of a chain are one thread-block cluster
+    // the D / SLC column slices of a chain (or of a segment of it) are one thread-block cluster
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(NTB);
@@ -259,7 +303,8 @@ kda_status launch_bwd(const void *q, const void *k, const void *v, const float *
                            static_cast<const TIn *>(v), g, beta, h0, (const int *)cu, hdr,
                            static_cast<const TIn *>(dO), dhT, T, H, ckpt, sub,
                            static_cast<TIn *>(dq), static_cast<TIn *>(dkk),
-                           static_cast<TIn *>(dvv), dg, db, dh0, ntok, err) != cudaSuccess) {
+                           static_cast<TIn *>(dvv), dg, db, dh0, ntok, err, nseg, seg_chunks,
+                           s_start, g_end, nfw, cps) != cudaSuccess) {
         cudaGetLastError();
         return KDA_ERR_CUDA;
     }
@@ -903,18 +948,42 @@ kda_status kda_decode_commit(const void *k, const void *v, const float *g, const
 }
 
 size_t kda_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int dtype) {
-    if (B < 0 || T < 0 || num_seqs < 0) return 0;
-    if (check_shape(H, dk, dv, dtype) != KDA_OK) return 0;
-    if (num_seqs > 0 && B != 1) return 0;
-    return bwd_layout(B, T, H, dk, num_seqs, dtype).total;
+    return kda_bwd_segmented_workspace_size(B, T, H, dk, dv, num_seqs, dtype, 0);
 }
 
-kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
-                   const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
-                   int B, int T, int H, int dk, int dv, int dtype, const void *grad_o,
-                   const float *grad_hT, void *grad_q, void *grad_k, void *grad_v,
-                   float *grad_g, float *grad_beta, float *grad_h0, void *workspace,
-                   size_t ws_bytes, void *stream) {
+int kda_bwd_plan_segments(int B, int T, int H, int dk, int dv, int num_seqs, int dtype) {
+    if (B < 0 || T < 0 || num_seqs < 0 || check_shape(H, dk, dv, dtype) != KDA_OK) return 0;
+    if (num_seqs > 0) return 1;
+    const BwdSegLayout S = bwd_seg_layout(B, T, H, dk, dtype);
+    return S.sc ? S.nseg : 1;
+}
+
+// num_segments == 0: kda_bwd's choice; 1: the per-chain pass; n >= 2: n segments.
+size_t kda_bwd_segmented_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
+                                        int dtype, int num_segments) {
+    if (B < 0 || T < 0 || num_seqs < 0 || num_segments < 0) return 0;
+    if (check_shape(H, dk, dv, dtype) != KDA_OK) return 0;
+    if (num_seqs > 0 && B != 1) return 0;
+    const size_t old = bwd_layout(B, T, H, dk, num_seqs, dtype).total;
+    if (num_segments == 1) return old;
+    if (num_segments >= 2) {
+        if (num_seqs > 0 || T <= 0) return 0;
+        const int cps = (T + kda::tc::C - 1) / kda::tc::C;
+        if (cps % num_segments) return 0;
+        return bwd_seg_layout(B, T, H, dk, dtype, cps / num_segments).total;
+    }
+    const size_t seg = num_seqs > 0 ? 0 : bwd_seg_layout(B, T, H, dk, dtype).total;
+    return old > seg ? old : seg;
+}
+
+// nseg_req: 0 the policy, 1 the per-chain pass, n >= 2 n segments.
+static kda_status bwd_impl(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, const float *h0, const int32_t *cu_seqlens,
+                           int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
+                           const void *grad_o, const float *grad_hT, void *grad_q, void *grad_k,
+                           void *grad_v, float *grad_g, float *grad_beta, float *grad_h0,
+                           void *workspace, size_t ws_bytes, void *stream, int nseg_req) {
+    if (nseg_req < 0) return KDA_ERR_INVALID_ARG;
     int N;
     WsLayout F;
     // the forward's checks cover the inputs; the outputs are checked here
@@ -936,7 +1005,19 @@ kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
         for (const void *i : ins)
             if (o && o == i) return KDA_ERR_INVALID_ARG;
     const BwdLayout L = bwd_layout(B, T, H, dk, cu_seqlens ? num_seqs : 0, dtype);
-    if (!workspace || ws_bytes < L.total) return KDA_ERR_WORKSPACE_TOO_SMALL;
+    BwdSegLayout SL{};
+    if (nseg_req >= 2) {   // explicit segments: tensor-core path, fixed length, n | chunks
+        const int cps = (T + kda::tc::C - 1) / kda::tc::C;
+        if (!cu_seqlens && T > 0 && cps % nseg_req == 0)
+            SL = bwd_seg_layout(B, T, H, dk, dtype, cps / nseg_req);
+        if (!SL.sc) return KDA_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned_to(grad_o, 16) || !aligned_to(grad_q, 16) || !aligned_to(grad_k, 16))
+            return KDA_ERR_MISALIGNED;
+    } else if (nseg_req == 0 && !cu_seqlens) {
+        SL = bwd_seg_layout(B, T, H, dk, dtype);
+    }
+    if (!workspace || ws_bytes < (L.total > SL.total ? L.total : SL.total))
+        return KDA_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned_to(workspace, 16)) return KDA_ERR_MISALIGNED;
     if (N == 0 || ntok == 0 && !grad_h0) return KDA_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -951,9 +1032,46 @@ kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
             ERRBIT_SEQLENS);
         if ((st = launch_status()) != KDA_OK) return st;
     }
+    const long long chains = (long long)N * H;
+    // Segmented: the tensor-core forward with the state at every segment start (its o
+    // goes to grad_q), the reversed records, the chunk-level gradient chain over them
+    // from dL/dhT with dL/dS at every segment end (its o goes to grad_k), then the
+    // per-token backward on all segments at once, which overwrites grad_q and grad_k.
+    // 16-byte vector accesses of grad_o, grad_q and grad_k; else the per-chain pass.
+    if (SL.sc && aligned_to(grad_o, 16) && aligned_to(grad_q, 16) && aligned_to(grad_k, 16)) {
+        using namespace kda::bwd;
+        float *fck = reinterpret_cast<float *>(ws + SL.fck);
+        float *rck = reinterpret_cast<float *>(ws + SL.rck);
+        const long long nck_slots = (long long)N * SL.nfw;
+        if ((st = tc_intra(q, k, v, g, beta, nullptr, N, T, H, SL.F, workspace, s)) != KDA_OK)
+            return st;
+        if ((st = tc_inter(h0, nullptr, N, T, H, SL.F, grad_q, nullptr, workspace, s, fck, SL.sc,
+                           nck_slots)) != KDA_OK)
+            return st;
+        const size_t rsmem = sizeof(RevSmem);
+        if (cudaFuncSetAttribute(kda_bwd_rev_records_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        const long long items = SL.F.max_chunks * H;
+        const int sms = device_sms();
+        const long long cap = 3LL * (sms > 0 ? sms : 148);
+        kda_bwd_rev_records_kernel<<<(unsigned)(items < cap ? items : cap), kRevThreads, rsmem, s>>>(
+            ws + SL.F.recs, static_cast<const __nv_bfloat16 *>(grad_o), ws + SL.rrec, T, H, SL.cps,
+            items);
+        if ((st = launch_status()) != KDA_OK) return st;
+        WsLayout R = SL.F;
+        R.recs = SL.rrec;
+        if ((st = tc_inter(grad_hT, nullptr, N, T, H, R, grad_k, nullptr, workspace, s, rck, SL.sc,
+                           nck_slots)) != KDA_OK)
+            return st;
+        return launch_bwd<128, __nv_bfloat16>(
+            q, k, v, g, beta, h0, nullptr, hdr, grad_o, grad_hT, T, H, ntok, chains,
+            reinterpret_cast<float *>(ws + SL.ckpt), reinterpret_cast<float *>(ws + SL.sub), grad_q,
+            grad_k, grad_v, grad_g, grad_beta, grad_h0, err, s, SL.nseg, SL.sc, fck, rck, SL.nfw,
+            SL.cps);
+    }
     float *ckpt = reinterpret_cast<float *>(ws + L.ckpt);
     float *sub = reinterpret_cast<float *>(ws + L.sub);
-    const long long chains = (long long)N * H;
 #define KDA_BWD(DD, TT)                                                                    \
     return launch_bwd<DD, TT>(q, k, v, g, beta, h0, cu_seqlens, hdr, grad_o, grad_hT, T, H, \
                               ntok, chains, ckpt, sub, grad_q, grad_k, grad_v, grad_g,      \
@@ -967,6 +1085,28 @@ kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
     if (dk == 64) KDA_BWD(64, float);
     KDA_BWD(128, float);
 #undef KDA_BWD
+}
+
+kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
+                   int B, int T, int H, int dk, int dv, int dtype, const void *grad_o,
+                   const float *grad_hT, void *grad_q, void *grad_k, void *grad_v,
+                   float *grad_g, float *grad_beta, float *grad_h0, void *workspace,
+                   size_t ws_bytes, void *stream) {
+    return bwd_impl(q, k, v, g, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv, dtype, grad_o,
+                    grad_hT, grad_q, grad_k, grad_v, grad_g, grad_beta, grad_h0, workspace,
+                    ws_bytes, stream, 0);
+}
+
+kda_status kda_bwd_segmented(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *h0, const int32_t *cu_seqlens,
+                             int num_seqs, int B, int T, int H, int dk, int dv, int dtype,
+                             const void *grad_o, const float *grad_hT, void *grad_q, void *grad_k,
+                             void *grad_v, float *grad_g, float *grad_beta, float *grad_h0,
+                             int num_segments, void *workspace, size_t ws_bytes, void *stream) {
+    return bwd_impl(q, k, v, g, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv, dtype, grad_o,
+                    grad_hT, grad_q, grad_k, grad_v, grad_g, grad_beta, grad_h0, workspace,
+                    ws_bytes, stream, num_segments);
 }
 
 // ---------------------------------------------------------------------------

@@ -19,6 +19,12 @@
 // columns: the D/16 slice CTAs of a chain form a thread-block cluster, and after
 // every piece each CTA adds the slices' partial sums for D/(D/16) of the rows
 // through distributed shared memory, in slice order (deterministic).
+// Segments: with nseg > 1 (fixed-length input) a chain is cut into nseg segments of
+// seg_chunks chunks, one cluster each, all running at once.  A segment starts from the
+// state at its first token (h0 for the first segment, else s_start) and its reverse
+// pass from dL/dS at its last token (dL/dhT for the last segment, else g_end); both
+// come from the tensor-core forward and the chunk-level gradient chain
+// (kda_bwd_chain.cuh), whose checkpoints every seg_chunks chunks they are.
 // Inside a CTA, warp w owns 4 columns of the slice across all d rows (lane l: rows
 // RPL l .. RPL l + RPL - 1, RPL = d / 32), so the column sums every token needs
 // (u = S'^T k, G^T k) are in-warp butterflies with no CTA barrier; the row sums
@@ -145,13 +151,15 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                      float *__restrict__ ckpt, float *__restrict__ sub, TIn *__restrict__ dq,
                      TIn *__restrict__ dk, TIn *__restrict__ dv, float *__restrict__ dg,
                      float *__restrict__ dbeta, float *__restrict__ dh0, long long ntok,
-                     int *err_word) {
+                     int *err_word, int nseg, int seg_chunks, const float *__restrict__ s_start,
+                     const float *__restrict__ g_end, int nfw, int cps) {
     constexpr int NS = D / SLC, NT = NTB, RPL = D / 32;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     BwdSmem<D, TIn> &sm = *reinterpret_cast<BwdSmem<D, TIn> *>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r0 = RPL * lane, c4 = 4 * warp;        // this thread: rows r0.., slice columns c4..
-    const int slice = blockIdx.x % NS, chain = blockIdx.x / NS, n = chain / H, h = chain % H;
+    const int slice = blockIdx.x % NS, unit = blockIdx.x / NS;
+    const int chain = unit / nseg, seg = unit % nseg, n = chain / H, h = chain % H;
     const int cs = slice * SLC;                      // the slice's first column
     int t0, len;
     if (cu) {
@@ -161,6 +169,11 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     } else {
         t0 = n * T;
         len = T;
+    }
+    if (nseg > 1) {   // this unit's tokens: seg_chunks chunks from the segment's start
+        const int lo = seg * seg_chunks * CK;
+        t0 += lo;
+        len = min(len - lo, seg_chunks * CK);
     }
     if constexpr (KDA_DEBUG) {
         if (len < 0 || t0 < 0 || (long long)t0 + len > ntok) {
@@ -192,9 +205,9 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     // a piece is due, its copies are awaited, converted to fp32 in place for the
     // steps, and the copies of the next piece in the kernel's order are issued, so
     // their latency hides behind the current piece's work (CTA barriers do not wait
-    // for them).  The order: the forward walk's pieces (phase 1), then per chunk from
-    // the last, its recompute walk (phase 2, pieces 0 .. npc - 2) and its backward
-    // pieces (phase 3, npc - 1 .. 0, which also need q and dO).
+    // for them).  The order: the forward walk's pieces (phase 1, chunks 0 .. nck - 2),
+    // then per chunk from the last, its recompute walk (phase 2, pieces 0 .. npc - 2)
+    // and its backward pieces (phase 3, npc - 1 .. 0, which also need q and dO).
     struct Ev {
         int ph, j, pc;   // ph 0: none
     };
@@ -206,7 +219,7 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     auto next_ev = [&](Ev e) -> Ev {
         if (e.ph == 1) {
             if (e.pc + 1 < npc_of(e.j)) return Ev{1, e.j, e.pc + 1};
-            if (e.j + 1 < nck) return Ev{1, e.j + 1, 0};
+            if (e.j + 2 < nck) return Ev{1, e.j + 1, 0};
             return first_back(nck - 1);
         }
         if (e.ph == 2) {
@@ -257,7 +270,7 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
             cp_async4(&sm.xb[tid], beta + (size_t)(c0 + min(tid, cl - 1)) * H + h, tid < cl ? 4 : 0);
         cp_async_commit();
     };
-    Ev cur = Ev{nck > 0 ? 1 : 0, 0, 0};
+    Ev cur = nck > 1 ? Ev{1, 0, 0} : (nck == 1 ? first_back(0) : Ev{0, 0, 0});
     issue_stage(cur);
     auto stage = [&]() {
         const bool with_q = cur.ph == 3;
@@ -316,20 +329,30 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     };
 
     // ---- forward: the slice's state at the start of every CK-token chunk, to HBM ----
+    // (the state after the last chunk is not needed: the walk stops before it)
     float S[RPL][4];
-    if (h0) ldS(S, h0 + sbase, D);
+    const float *s_init = seg == 0 ? (h0 ? h0 + sbase : nullptr)
+                                   : s_start + ((size_t)(n * nfw + seg - 1) * H + h) * D * D + cs + c4;
+    if (s_init) ldS(S, s_init, D);
     else
 #pragma unroll
         for (int i = 0; i < RPL; ++i) S[i][0] = S[i][1] = S[i][2] = S[i][3] = 0.f;
     for (int j = 0; j < nck; ++j) {
         stS(ckpt + (ckpt_slot(t0, n, j) * H + h) * D * D + cs + c4, D, S);
         const int lenj = min(CK, len - j * CK);
-        for (int p = 0; p < lenj; p += CB) run(S, j * CK + p, min(CB, lenj - p));
+        if (j + 1 < nck)
+            for (int p = 0; p < lenj; p += CB) run(S, j * CK + p, min(CB, lenj - p));
     }
 
     // ---- backward ----
+    // dL/dS after the unit's last token: dL/dhT, or the chain's checkpoint at the
+    // boundary (seg + 1) seg_chunks chunks, which it stored after cps - (seg + 1)
+    // seg_chunks of its (reversed) steps
     float G[RPL][4];
-    if (dhT) ldS(G, dhT + sbase, D);
+    const float *g_init = seg == nseg - 1
+                              ? (dhT ? dhT + sbase : nullptr)
+                              : g_end + ((size_t)(n * nfw + cps / seg_chunks - seg - 2) * H + h) * D * D + cs + c4;
+    if (g_init) ldS(G, g_init, D);
     else
 #pragma unroll
         for (int i = 0; i < RPL; ++i) G[i][0] = G[i][1] = G[i][2] = G[i][3] = 0.f;
@@ -454,7 +477,7 @@ kda_bwd_slice_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
             cluster_sync();   // the partial sums may be overwritten by the next piece
         }
     }
-    if (dh0) stS(dh0 + sbase, D, G);
+    if (dh0 && seg == 0) stS(dh0 + sbase, D, G);
 }
 
 }  // namespace bwd

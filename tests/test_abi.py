@@ -122,6 +122,63 @@ def test_segmented_workspace_size(lib):
     assert seg(1, 100, 1, 64, 64, 0, F32, 1) == ws(1, 100, 1, 64, 64, 0, F32)
 
 
+def test_bwd_workspace_and_plan(lib):
+    """kda_bwd's schedule: segments of whole chunks for bf16, d = 128, fixed-length
+    input (one chunk each while (sequences x heads x segments) <= 1024, else the fewest
+    power-of-two chunks that keep it so), the per-chain pass otherwise."""
+    ws, seg, plan = (lib.kda_bwd_workspace_size, lib.kda_bwd_segmented_workspace_size,
+                     lib.kda_bwd_plan_segments)
+    assert plan(2, 4096, 8, 128, 128, 0, BF16) == 64        # 16 chains x 64 chunks
+    assert plan(2, 8192, 8, 128, 128, 0, BF16) == 64        # 2 chunks per segment
+    assert plan(1, 1 << 20, 16, 128, 128, 0, BF16) == 64    # 256 chunks per segment
+    assert plan(3, 1000, 3, 128, 128, 0, BF16) == 16
+    assert plan(1, 64, 2, 128, 128, 0, BF16) == 1           # one chunk: nothing to cut
+    assert plan(2, 4096, 8, 64, 64, 0, F32) == 1            # CUDA-core path
+    assert plan(1, 300, 2, 128, 128, 2, BF16) == 1          # packed
+    assert plan(1, 100, 2, 128, 96, 0, BF16) == 0           # invalid sizes
+    # the policy's workspace is the larger of the two schedules'
+    assert ws(2, 4096, 8, 128, 128, 0, BF16) == seg(2, 4096, 8, 128, 128, 0, BF16, 64)
+    assert seg(2, 4096, 8, 128, 128, 0, BF16, 0) == ws(2, 4096, 8, 128, 128, 0, BF16)
+    one = seg(2, 4096, 8, 128, 128, 0, BF16, 1)
+    assert 0 < one < seg(2, 4096, 8, 128, 128, 0, BF16, 2) < seg(2, 4096, 8, 128, 128, 0, BF16, 64)
+    # per-unit scratch: 8 states of 128 x 128 fp32 per (sequence, head, segment)
+    unit = 8 * 128 * 128 * 4
+    d = seg(2, 4096, 8, 128, 128, 0, BF16, 64) - seg(2, 4096, 8, 128, 128, 0, BF16, 32)
+    states = 2 * 2 * 32 * 8 * 128 * 128 * 4                 # start states and end gradients
+    assert unit * 16 * 32 + states <= d < unit * 16 * 32 + states + 1024
+    for n in (3, 128, -1):                                  # n must divide the 64 chunks
+        assert seg(2, 4096, 8, 128, 128, 0, BF16, n) == 0
+    assert seg(2, 4096, 8, 64, 64, 0, F32, 2) == 0
+    assert seg(2, 4096, 8, 64, 64, 0, F32, 1) == ws(2, 4096, 8, 64, 64, 0, F32)
+    assert seg(1, 300, 2, 128, 128, 2, BF16, 2) == 0        # packed: per-chain only
+
+
+def _bwd(lib, nseg, ptr=0x10000, ws=1 << 40, **over):
+    a = dict(q=ptr, k=ptr, v=ptr, g=ptr, beta=ptr, h0=None, cu=None, num_seqs=0, B=1, T=512,
+             H=2, dk=128, dv=128, dtype=BF16, do=ptr, dhT=None, dq=0x200000, dk_=0x300000,
+             dv_=0x400000, dg=0x500000, db=0x600000, dh0=None, work=0x700000, ws=ws,
+             stream=None)
+    a.update(over)
+    return lib.kda_bwd_segmented(a["q"], a["k"], a["v"], a["g"], a["beta"], a["h0"], a["cu"],
+                                 a["num_seqs"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                                 a["dtype"], a["do"], a["dhT"], a["dq"], a["dk_"], a["dv_"],
+                                 a["dg"], a["db"], a["dh0"], nseg, a["work"], a["ws"],
+                                 a["stream"])
+
+
+def test_bwd_segmented_validation_before_launch(lib):
+    assert _bwd(lib, -1) == INVALID
+    assert _bwd(lib, 3) == UNSUPPORTED                       # 3 does not divide 8 chunks
+    assert _bwd(lib, 16) == UNSUPPORTED
+    assert _bwd(lib, 2, dk=64, dv=64, dtype=F32) == UNSUPPORTED
+    assert _bwd(lib, 2, cu=0x30000, num_seqs=2, B=1) == UNSUPPORTED
+    assert _bwd(lib, 2, do=0x10002) == MISALIGNED            # 16-byte vector reads of dO
+    assert _bwd(lib, 2, dq=0x200002) == MISALIGNED
+    assert _bwd(lib, 2, dk_=0x300008) == MISALIGNED
+    assert _bwd(lib, 2, ws=1024) == WS_SMALL
+    assert _bwd(lib, 2, dq=0x10000) == INVALID               # a gradient aliases an input
+
+
 def _fwd(lib, ptr=0x10000, ws=1 << 40, **over):
     a = dict(q=ptr, k=ptr, v=ptr, g=ptr, beta=ptr, h0=None, cu=None, num_seqs=0, B=1, T=64,
              H=2, dk=128, dv=128, dtype=BF16, o=ptr + 0x100000, hT=None, work=ptr, ws=ws,

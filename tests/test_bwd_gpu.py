@@ -1,11 +1,15 @@
-"""The backward pass (kda_bwd) through the C ABI against the fp64 oracle gradient.
+"""The backward pass (kda_bwd, kda_bwd_segmented) through the C ABI against the fp64
+oracle gradient.
 
 The loss is L = sum(do * o) + sum(dhT * hT) for seeded upstream gradients do (in
-the dtype of q) and dhT (fp32).  The kernels compute in fp32 from the exact input
-values, so gradients stored in fp32 (dg, dbeta, dh0) must match the fp64 oracle
-to rel-L2 <= 1e-4 whatever the input dtype; gradients stored in the input dtype
-(dq, dk, dv) carry its rounding: rel-L2 <= 1e-4 for fp32 and, for bf16, rel-L2
-<= 1e-2 with max-abs <= 5e-2 of the tensor's largest magnitude (at least 1).
+the dtype of q) and dhT (fp32).  The per-chain pass computes in fp32 from the exact
+input values, so there the gradients stored in fp32 (dg, dbeta, dh0) must match the
+fp64 oracle to rel-L2 <= 1e-4 whatever the input dtype; gradients stored in the input
+dtype (dq, dk, dv) carry its rounding: rel-L2 <= 1e-4 for fp32 and, for bf16, rel-L2
+<= 1e-2 with max-abs <= 5e-2 of the tensor's largest magnitude (at least 1).  The
+segmented pass (bf16, d = 128) starts its segments from states of the bf16 tensor-core
+forward and ends them at gradients carried over the bf16 chunk records, so every one of
+its gradients is held to that bf16 bound, the prefill's own.
 """
 import numpy as np
 import pytest
@@ -40,7 +44,7 @@ def _check(got, ref, stored_dtype, what):
     return r
 
 
-def _run(inp, seed, with_dhT=True):
+def _upstream(inp, seed, with_dhT):
     B, T, H, dk = inp["q"].shape
     dv = inp["v"].shape[-1]
     cu = inp["cu_seqlens"]
@@ -48,17 +52,41 @@ def _run(inp, seed, with_dhT=True):
     gen = torch.Generator(device=DEV).manual_seed(seed)
     do = torch.randn(B, T, H, dv, generator=gen, device=DEV).to(inp["q"].dtype)
     dhT = (0.1 * torch.randn(N, H, dk, dv, generator=gen, device=DEV)) if with_dhT else None
-    got = kda.kda_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], cu, do,
-                      dhT)
+    return do, dhT
+
+
+def _call(inp, do, dhT, num_segments):
+    """kda_bwd (num_segments None) or kda_bwd_segmented; returns the gradients and the
+    segments per sequence the call used."""
+    B, T, H, dk = inp["q"].shape
+    cu = inp["cu_seqlens"]
+    a = (inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], cu, do, dhT)
+    plan = kda.bwd_plan_segments(B, T, H, dk, inp["v"].shape[-1],
+                                 0 if cu is None else cu.numel() - 1, inp["q"].dtype)
+    if num_segments is None:
+        got = kda.kda_bwd(*a)
+    else:
+        got = kda.kda_bwd_segmented(*a, num_segments=num_segments)
+        plan = num_segments or plan
+    torch.cuda.synchronize()
     assert kda.device_error() == 0
-    ref = oracle.kda_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], do,
-                         dhT, cu)
-    dt = inp["q"].dtype
+    return got, plan
+
+
+def _compare(got, ref, dt, segmented):
     for name, a, b in zip(NAMES, got, ref):
         if a is None:
             continue
-        stored = dt if name in ("dq", "dk", "dv") else torch.float32
+        stored = dt if name in ("dq", "dk", "dv") or segmented else torch.float32
         _check(a, b.reshape(a.shape), stored, name)
+
+
+def _run(inp, seed, with_dhT=True, num_segments=None):
+    do, dhT = _upstream(inp, seed, with_dhT)
+    got, nseg = _call(inp, do, dhT, num_segments)
+    ref = oracle.kda_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], do,
+                         dhT, inp["cu_seqlens"])
+    _compare(got, ref, inp["q"].dtype, nseg >= 2)
     return got
 
 
@@ -98,10 +126,64 @@ def test_empty_sequence_passes_the_final_state_gradient_through():
 
 
 def test_prefill_workload_full_size():
-    """The B=2, H=8, T=4,096 workload: every gradient of every token and head."""
-    w = W.PREFILL
-    inp = W.make_workload(w, DEV)
-    _run(inp, seed=60)
+    """The B=2, H=8, T=4,096 workload: every gradient of every token and head, from
+    kda_bwd (64 segments of one chunk per sequence) and from the per-chain pass."""
+    inp = W.make_workload(W.PREFILL, DEV)
+    do, dhT = _upstream(inp, 60, True)
+    seg, nseg = _call(inp, do, dhT, None)
+    assert nseg == 64
+    chain, _ = _call(inp, do, dhT, 1)
+    ref = oracle.kda_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"], do,
+                         dhT, None)
+    _compare(seg, ref, torch.bfloat16, True)
+    _compare(chain, ref, torch.bfloat16, False)
+
+
+@pytest.mark.parametrize("T", [65, 200])
+def test_per_chain_pass_is_exact_for_bf16(T):
+    """num_segments = 1: the per-chain fp32 pass, held to 1e-4 on the fp32 gradients."""
+    inp = W.make_prefill_inputs(2, T, 3, 128, 128, torch.bfloat16, True, seed=T + 70,
+                                device=DEV)
+    _run(inp, seed=T + 1, num_segments=1)
+
+
+@pytest.mark.parametrize("T,nseg,h0,dhT", [(512, 2, True, True), (512, 4, False, True),
+                                           (512, 8, True, False), (500, 2, True, True),
+                                           (500, 8, False, False), (1000, 16, True, True)])
+def test_explicit_segment_counts(T, nseg, h0, dhT):
+    """Segments of 1 to 4 chunks (and a ragged last chunk) against the oracle."""
+    inp = W.make_prefill_inputs(2, T, 3, 128, 128, torch.bfloat16, h0, seed=T + nseg,
+                                device=DEV)
+    _run(inp, seed=T + nseg + 1, with_dhT=dhT, num_segments=nseg)
+
+
+def test_policy_equals_explicit_count():
+    inp = W.make_prefill_inputs(1, 200, 2, 128, 128, torch.bfloat16, True, seed=71, device=DEV)
+    do, dhT = _upstream(inp, 72, True)
+    a, na = _call(inp, do, dhT, None)
+    b, _ = _call(inp, do, dhT, na)
+    c, _ = _call(inp, do, dhT, 0)
+    assert na == 4
+    for x, y, z in zip(a, b, c):
+        assert torch.equal(x, y) and torch.equal(x, z)
+
+
+def test_explicit_segments_rejected():
+    """Counts that do not divide the chunks, other dtypes and head sizes, packed input."""
+    def expect_unsupported(inp, n):
+        do, dhT = _upstream(inp, 73, True)
+        with pytest.raises(kda.KDAError) as e:
+            kda.kda_bwd_segmented(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["h0"],
+                                  inp["cu_seqlens"], do, dhT, num_segments=n)
+        assert e.value.code == 2   # KDA_ERR_UNSUPPORTED_SHAPE
+    expect_unsupported(W.make_prefill_inputs(1, 512, 2, 128, 128, torch.bfloat16, True, seed=74,
+                                             device=DEV), 3)
+    expect_unsupported(W.make_prefill_inputs(1, 512, 2, 128, 128, torch.bfloat16, True, seed=74,
+                                             device=DEV), 16)
+    expect_unsupported(W.make_prefill_inputs(1, 512, 2, 64, 64, torch.float32, True, seed=75,
+                                             device=DEV), 2)
+    expect_unsupported(W.make_prefill_inputs(1, 0, 2, 128, 128, torch.bfloat16, True, seed=76,
+                                             device=DEV, lengths=[128, 128]), 2)
 
 
 def test_deterministic():
