@@ -204,7 +204,7 @@ kda_status kda_fwd_segmented(const void *q, const void *k, const void *v, const 
  * kernel, which write the records in time order (chunk j of every chain before
  * chunk j + 1) and publish each through a flag in the workspace; a state block
  * waits (bounded, 1 s) for a record's flag before copying it in, and a record
- * worker starts a chunk only within a window of chunks (about 48 MiB of records)
+ * worker starts a chunk only within a window of chunks (about 32 MiB of records)
  * ahead of that chain's state blocks, so the records are read back from L2.  Each
  * waits only for work that comes earlier in time order than what it holds, so the
  * blocks cannot deadlock; the launch is cooperative so that every block is
