@@ -130,3 +130,66 @@ def test_sub_tile_reference_factors_stay_in_range_at_the_decay_bound():
     o_ref, S_ref = reference(q, k, v, g, beta, S0)
     assert np.abs(o - o_ref).max() <= 1e-11 * max(1.0, np.abs(o_ref).max())
     assert np.abs(S - S_ref).max() <= 1e-11 * max(1.0, np.abs(S_ref).max())
+
+
+def _bwd(q, k, v, g, beta, S0, do, dhT):
+    """The oracle's gradient on one (sequence, head): (dq, dk, dv, dg, dbeta, dh0)."""
+    r = oracle.kda_bwd(q[None, :, None], k[None, :, None], v[None, :, None], g[None, :, None],
+                       beta[None, :, None], S0[None, None], do[None, :, None], dhT[None, None])
+    return tuple(x[0, :, 0] for x in r[:5]) + (r[5][0, 0],)
+
+
+@pytest.mark.parametrize("T,slow", [(150, False), (256, False), (150, True), (256, True)])
+def test_state_gradient_chain_over_the_chunk_maps(T, slow):
+    """The segmented backward's premise.  With S_out = P S_in + R and O = Q' S_in + O0
+    (P = Diag(exp G_C) + M'), the loss is affine in the state at a chunk boundary and
+    its gradient there obeys dS_in = Diag(exp G_C) dS_out + M'^T dS_out + Q'^T dO,
+    from dS = dL/dhT after the last chunk: the forward update with M'^T for M' and
+    Q'^T dO for R, run over the chunks in reverse.  At every boundary it must equal
+    the oracle's dL/dh0 of the suffix that starts there.  slow: decays of 0.1-1.1% per
+    token, so the state (and its gradient) carries across chunks and the M'^T term
+    weighs as much as the others."""
+    dk, dv = 12, 10
+    q, k, v, g, beta, S0 = inputs(T, dk, dv, seed=T + 5)
+    rng = np.random.default_rng(T + 6)
+    if slow:
+        g = -0.001 - 0.01 * rng.random((T, dk))
+    do = rng.standard_normal((T, dv))
+    dhT = 0.1 * rng.standard_normal((dk, dv))
+    starts = list(range(0, T, C))
+    maps = [chunk_map(q[t:t + C], k[t:t + C], v[t:t + C], g[t:t + C], beta[t:t + C])
+            for t in starts]
+    G = dhT.copy()
+    chain = {}
+    for t, m in zip(reversed(starts), reversed(maps)):
+        G = m["gC"][:, None] * G + m["M"].T @ G + m["Qp"].T @ do[t:t + C]
+        chain[t] = G
+    for t in starts:
+        sl = slice(t, T)
+        dh0 = _bwd(q[sl], k[sl], v[sl], g[sl], beta[sl], np.zeros((dk, dv)), do[sl], dhT)[5]
+        assert np.abs(chain[t] - dh0).max() <= 1e-10 * max(1.0, np.abs(dh0).max()), t
+
+
+def test_segments_from_their_boundary_states_and_gradients():
+    """The per-token backward run on a segment alone, from the forward state at its
+    start and the chain's gradient at its end, gives the whole sequence's gradients
+    for the segment's tokens (and, for the first segment, dL/dh0)."""
+    T, dk, dv = 200, 8, 6
+    q, k, v, g, beta, S0 = inputs(T, dk, dv, seed=31)
+    rng = np.random.default_rng(32)
+    do = rng.standard_normal((T, dv))
+    dhT = 0.1 * rng.standard_normal((dk, dv))
+    full = _bwd(q, k, v, g, beta, S0, do, dhT)
+    bounds = [0, 64, 128, T]          # segments of whole chunks; the last one ragged
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        S_a = S0 if a == 0 else reference(q[:a], k[:a], v[:a], g[:a], beta[:a], S0)[1]
+        if b == T:
+            G_b = dhT
+        else:   # dL/dS_b: the suffix's dL/dh0 (the loss is affine in S_b)
+            G_b = _bwd(q[b:], k[b:], v[b:], g[b:], beta[b:], np.zeros((dk, dv)), do[b:], dhT)[5]
+        part = _bwd(q[a:b], k[a:b], v[a:b], g[a:b], beta[a:b], S_a, do[a:b], G_b)
+        for x, y in zip(part[:5], full[:5]):
+            ref = y[a:b]
+            assert np.abs(x - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max()), (a, b)
+        if a == 0:
+            assert np.abs(part[5] - full[5]).max() <= 1e-10 * max(1.0, np.abs(full[5]).max())
