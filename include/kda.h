@@ -18,8 +18,8 @@
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller, row-major and
  *     contiguous.  Alignment: prefill q, k, v, h0, hT and the workspace 16
- *     bytes, g 8 bytes, o two elements; the decode state S 16 bytes; everything
- *     else its element size.  A violation returns KDA_ERR_MISALIGNED.  The library never
+ *     bytes, g 8 bytes (16 on the tensor-core path, bf16 with d = 128), o two
+ *     elements; the decode state S 16 bytes; everything else its element size.  A violation returns KDA_ERR_MISALIGNED.  The library never
  *     allocates device memory and never synchronises the stream in the compute
  *     entry points.
  *   - q, k, g are [.., H, d_k]; v, o are [.., H, d_v]; beta is [.., H];
@@ -316,7 +316,8 @@ kda_status kda_cp_finish(const float *maps, int rank, int world, const float *h0
  * Backward pass: the gradient of a loss L through kda_fwd.  Given grad_o = dL/do and
  * grad_hT = dL/dhT (NULL: zero), writes dL/dq, dL/dk, dL/dv (dtype of q, k, v),
  * dL/dg, dL/dbeta (fp32) and dL/dh0 (fp32, NULL to skip).  Same inputs, layouts,
- * packed-sequence rules and alignment as kda_fwd; grad_o [B, T, H, d_v] has the
+ * packed-sequence rules and alignment as kda_fwd, except that g and grad_o must be
+ * 16-byte aligned (rows are staged by 16-byte copies); grad_o [B, T, H, d_v] has the
  * dtype of q; grad_hT, grad_h0 [N, H, d_k, d_v].  No gradient buffer may alias an
  * input.  The workspace must hold kda_bwd_workspace_size(...) bytes.
  *
@@ -337,7 +338,7 @@ kda_status kda_cp_finish(const float *maps, int rank, int world, const float *h0
  *               (sequence, head) (d_k d_v / 16 bytes per token-head) plus 8 states per
  *               (sequence, head).  The gradients stored in fp32 match an fp64
  *               evaluation to about 1e-7.
- *   segmented:  (bf16, d_k = d_v = 128, fixed-length input, grad_o, grad_q and grad_k
+ *   segmented:  (bf16, d_k = d_v = 128, fixed-length input, grad_q and grad_k
  *               16-byte aligned) the chain cut into segments of whole 64-token chunks,
  *               all run at once.  A segment's starting state comes from the tensor-core
  *               forward (kda_fwd's records and state pass, with a checkpoint at every
@@ -363,7 +364,7 @@ kda_status kda_bwd(const void *q, const void *k, const void *v, const float *g,
  * kda_bwd with the schedule chosen by the caller: num_segments = 0 as kda_bwd, 1 the
  * per-chain pass (any input kda_bwd takes), n >= 2 the segmented pass with n segments
  * per sequence (n must divide ceil(T / 64); bf16, d = 128, fixed-length input, else
- * KDA_ERR_UNSUPPORTED_SHAPE; grad_o, grad_q, grad_k 16-byte aligned, else
+ * KDA_ERR_UNSUPPORTED_SHAPE; grad_q, grad_k 16-byte aligned, else
  * KDA_ERR_MISALIGNED).  The workspace must hold
  * kda_bwd_segmented_workspace_size(..., num_segments) bytes (0 when the request cannot
  * be met).

@@ -376,6 +376,8 @@ static kda_status validate_fwd(const void *q, const void *k, const void *v, cons
         !aligned_to(workspace, 16) || !aligned_to(h0, 16) || !aligned_to(hT, 16) ||
         !aligned_to(g, 8) || !aligned_to(beta, 4) || !aligned_to(cu, 4) || !aligned_to(o, 2 * es))
         return KDA_ERR_MISALIGNED;
+    // the tensor-core path loads g by tensor copies: a 16-byte aligned base
+    if (is_tc_path(dtype, dk) && !aligned_to(g, 16)) return KDA_ERR_MISALIGNED;
     // outputs must not alias inputs (hT == h0 is the one allowed overlap)
     if (o && (o == q || o == k || o == v || o == g || o == beta)) return KDA_ERR_INVALID_ARG;
     if (nseg_req < 0 || nseg_req > kMaxSegmentsExplicit) return KDA_ERR_INVALID_ARG;
@@ -996,9 +998,10 @@ static kda_status bwd_impl(const void *q, const void *k, const void *v, const fl
     const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
     if (ntok > 0 && (!grad_o || !grad_q || !grad_k || !grad_v || !grad_g || !grad_beta))
         return KDA_ERR_INVALID_ARG;
-    if (!aligned_to(grad_o, es) || !aligned_to(grad_q, es) || !aligned_to(grad_k, es) ||
-        !aligned_to(grad_v, es) || !aligned_to(grad_g, 4) || !aligned_to(grad_beta, 4) ||
-        !aligned_to(grad_hT, 16) || !aligned_to(grad_h0, 16))
+    // the slice kernel stages rows of g and grad_o with 16-byte copies
+    if (!aligned_to(grad_o, 16) || !aligned_to(g, 16) || !aligned_to(grad_q, es) ||
+        !aligned_to(grad_k, es) || !aligned_to(grad_v, es) || !aligned_to(grad_g, 4) ||
+        !aligned_to(grad_beta, 4) || !aligned_to(grad_hT, 16) || !aligned_to(grad_h0, 16))
         return KDA_ERR_MISALIGNED;
     const void *ins[] = {q, k, v, g, beta, h0, grad_o, grad_hT};
     const void *outs[] = {grad_q, grad_k, grad_v, grad_g, grad_beta, grad_h0};
@@ -1012,8 +1015,7 @@ static kda_status bwd_impl(const void *q, const void *k, const void *v, const fl
         if (!cu_seqlens && T > 0 && cps % nseg_req == 0)
             SL = bwd_seg_layout(B, T, H, dk, dtype, cps / nseg_req);
         if (!SL.sc) return KDA_ERR_UNSUPPORTED_SHAPE;
-        if (!aligned_to(grad_o, 16) || !aligned_to(grad_q, 16) || !aligned_to(grad_k, 16))
-            return KDA_ERR_MISALIGNED;
+        if (!aligned_to(grad_q, 16) || !aligned_to(grad_k, 16)) return KDA_ERR_MISALIGNED;
     } else if (nseg_req == 0 && !cu_seqlens) {
         SL = bwd_seg_layout(B, T, H, dk, dtype);
     }
@@ -1038,8 +1040,9 @@ static kda_status bwd_impl(const void *q, const void *k, const void *v, const fl
     // goes to grad_q), the reversed records, the chunk-level gradient chain over them
     // from dL/dhT with dL/dS at every segment end (its o goes to grad_k), then the
     // per-token backward on all segments at once, which overwrites grad_q and grad_k.
-    // 16-byte vector accesses of grad_o, grad_q and grad_k; else the per-chain pass.
-    if (SL.sc && aligned_to(grad_o, 16) && aligned_to(grad_q, 16) && aligned_to(grad_k, 16)) {
+    // 16-byte vector stores of grad_q and grad_k (the state passes' o); else the
+    // per-chain pass.
+    if (SL.sc && aligned_to(grad_q, 16) && aligned_to(grad_k, 16)) {
         using namespace kda::bwd;
         float *fck = reinterpret_cast<float *>(ws + SL.fck);
         float *rck = reinterpret_cast<float *>(ws + SL.rck);

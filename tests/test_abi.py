@@ -173,6 +173,8 @@ def test_bwd_segmented_validation_before_launch(lib):
     assert _bwd(lib, 2, dk=64, dv=64, dtype=F32) == UNSUPPORTED
     assert _bwd(lib, 2, cu=0x30000, num_seqs=2, B=1) == UNSUPPORTED
     assert _bwd(lib, 2, do=0x10002) == MISALIGNED            # 16-byte vector reads of dO
+    assert _bwd(lib, 1, do=0x10008) == MISALIGNED            # every schedule stages dO rows
+    assert _bwd(lib, 1, g=0x10008, dtype=F32, dk=64, dv=64) == MISALIGNED   # ... and g rows
     assert _bwd(lib, 2, dq=0x200002) == MISALIGNED
     assert _bwd(lib, 2, dk_=0x300008) == MISALIGNED
     assert _bwd(lib, 2, ws=1024) == WS_SMALL
@@ -200,6 +202,8 @@ def test_fwd_validation_before_launch(lib):
     assert _fwd(lib, q=0x10004) == MISALIGNED
     assert _fwd(lib, hT=0x20008) == MISALIGNED           # states are read as float4
     assert _fwd(lib, g=0x10004) == MISALIGNED            # g is read as float pairs
+    assert _fwd(lib, g=0x10008) == MISALIGNED            # ... and by tensor copies (bf16, d=128)
+    assert _fwd(lib, g=0x10008, dtype=F32, dk=64, dv=64, B=0) == OK   # CUDA-core path: 8 bytes
     assert _fwd(lib, o=0x20002) == MISALIGNED            # bf16 o needs 4 bytes
     assert _fwd(lib, o=0x10000) == INVALID               # output aliases an input
     assert _fwd(lib, ws=16) == WS_SMALL
