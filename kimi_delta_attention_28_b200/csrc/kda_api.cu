@@ -567,6 +567,10 @@ static kda_status tc_inter(const float *h0, const int32_t *cu, int N, int T, int
 // Below 128 chunks per chain the two were measured equal or the single launch slower
 // (B=2, H=8, T=4,096: 0.110 against 0.107 ms), so the single launch needs at least that
 // many (B=1, H=16, T=16,384: 0.380 against 0.416 ms; T=1M: 19.5 against 23.8 ms).
+// The constants were fitted before the state pass had a producer warp per ring and the
+// record window its 32 MiB (one launch at T=1M: 15.9 against 22.5 ms now; a 64-column
+// chunk about 0.93 us inside it): the model errs toward the two launches, and picks the
+// single launch for about 12 or more chains, where it was measured faster.
 constexpr double kPrepUsTwo = 12.2, kState32Us = 0.79;
 constexpr double kPrepUsOne = 14.5, kState64OneUs = 1.19, kRampUs = 5.0;
 constexpr long long kMinOverlapChunks = 128;
