@@ -527,6 +527,23 @@ def measure_e2e(kda, w, inp, o, hT, ws, dev, stream, world, ntok, n_steps):
                     "pipelined on 3 streams with 2 device buffer sets"}
 
 
+def workload_shapes(w):
+    """The prefill inputs of workload `w` as meta tensors: shapes and dtypes, no data."""
+    import torch
+    from kimi_delta_attention_28_b200 import workloads as W
+    meta = torch.device("meta")
+    if w.varlen_seqs:
+        lengths = W.varlen_lengths(w.varlen_seqs, *w.varlen_range, seed=w.seed)
+        B, T, N = 1, int(sum(lengths)), len(lengths)
+    else:
+        B, T, N = w.B, w.T, w.B
+    mk = lambda *s, dt=torch.float32: torch.empty(*s, dtype=dt, device=meta)  # noqa: E731
+    return {"q": mk(B, T, w.H, w.dk, dt=w.dtype), "k": mk(B, T, w.H, w.dk, dt=w.dtype),
+            "v": mk(B, T, w.H, w.dv, dt=w.dtype), "g": mk(B, T, w.H, w.dk),
+            "beta": mk(B, T, w.H), "h0": mk(N, w.H, w.dk, w.dv) if w.h0 else None,
+            "cu_seqlens": mk(N + 1, dt=torch.int32) if w.varlen_seqs else None}
+
+
 def host_f64(inp):
     import numpy as np
     out = {}
@@ -998,12 +1015,15 @@ def run_reference(args, world, rank):
     import oracle
     from kimi_delta_attention_28_b200 import workloads as W
     w = workload_of(args.workload)
-    inp = W.make_workload(w, "cpu")
-    h = host_f64(inp)
-    B, T, H, dk = h["q"].shape
-    # sample: whole (sequence, head) chains over the first Ts tokens of sequence 0,
-    # sized so warmup + steps finish in about args.ref_seconds
-    Ts = min(T, 4096)
+    # The sample only: whole (sequence, head) chains over Ts tokens of one sequence,
+    # drawn by the workload's generator at that size (the whole workload, converted to
+    # fp64 on the host, would take about 90 GB at T = 1M), sized below so that warmup +
+    # steps finish in about args.ref_seconds.  The config reports the whole workload.
+    shapes = workload_shapes(w)
+    B, T, H, dk = shapes["q"].shape
+    Ts = min(T if w.varlen_seqs == 0 else
+             W.varlen_lengths(w.varlen_seqs, *w.varlen_range, seed=w.seed)[0], 4096)
+    h = host_f64(W.make_prefill_inputs(1, Ts, H, dk, w.dv, w.dtype, w.h0, w.seed, "cpu"))
     one = lambda n: np.ascontiguousarray(h[n][0, :Ts, :1])  # noqa: E731
     t0 = time.perf_counter()
     oracle.kda_fwd_packed(one("q"), one("k"), one("v"), one("g"), one("beta"), None,
@@ -1028,13 +1048,13 @@ def run_reference(args, world, rank):
     ms = 1e3 * statistics.mean(times)
     tokens = Ts * chains / H          # tokens-with-H-heads equivalent of the sample
     value = tokens / (ms * 1e-3)
-    sample = (f"{chains} of {H} heads x {Ts} tokens of sequence 0 per step "
+    sample = (f"{chains} of {H} heads x {Ts} tokens of one sequence per step "
               f"(fp64 token-by-token C oracle)")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded), same generator as the GPU arm",
-            "config": prefill_config(w, inp, world),
+            "config": prefill_config(w, shapes, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": int(used),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
