@@ -1,6 +1,7 @@
 """Host-side bookkeeping of bench.py (CPU): the byte counts behind the roofline and
 the rule that a stored ncu traffic figure is reported only for the kernel sources it
 was taken on."""
+import pytest
 import json
 import os
 
@@ -82,3 +83,16 @@ def test_headline_workload_is_the_largest_single_gpu_prefill():
     from kimi_delta_attention_28_b200 import workloads as W
     assert bench.HEADLINE == "long" and bench.workload_of(bench.HEADLINE) is W.LONG
     assert bench.default_steps("long") >= 3
+
+
+@pytest.mark.parametrize("name", ["prefill", "profile"])
+def test_reference_arm_config_from_shapes_alone(name):
+    """The reference arm reports the whole workload's config from shape-only (meta)
+    tensors, drawing only its sample: the config must equal the GPU arm's."""
+    import bench
+    from kimi_delta_attention_28_b200 import workloads as W
+    w = bench.workload_of(name)
+    real = W.make_workload(w, "cpu")
+    assert bench.prefill_config(w, bench.workload_shapes(w), 1) == bench.prefill_config(w, real, 1)
+    shapes = bench.workload_shapes(bench.workload_of("long"))
+    assert tuple(shapes["q"].shape) == (1, 1 << 20, 16, 128) and shapes["q"].device.type == "meta"
