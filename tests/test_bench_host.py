@@ -1,10 +1,10 @@
 """Host-side bookkeeping of bench.py (CPU): the byte counts behind the roofline and
 the rule that a stored ncu traffic figure is reported only for the kernel sources it
 was taken on."""
-import pytest
 import json
 import os
 
+import pytest
 import torch
 
 import bench
