@@ -348,6 +348,10 @@ kda_status kda_cp_finish(const float *maps, int rank, int world, const float *h0
  *               the bf16 records' rounding, so every gradient is held to the bf16
  *               prefill bound (rel-L2 <= 1e-2).  grad_q and grad_k serve as scratch for
  *               the two state passes' outputs before they receive the gradients.
+ *               Workspace: the chunk records twice (forward and reversed, 1,544 bytes
+ *               per token-head each at d = 128), a state and a state gradient per
+ *               segment boundary, the 64-token checkpoints as above and 8 states per
+ *               (sequence, head, segment).
  * kda_bwd takes the segmented schedule whenever it applies and some cut leaves at least
  * two segments: one chunk per segment, or the fewest chunks (a power of two dividing
  * the chunks per sequence) that keep (sequences x heads x segments) <= 1024.
